@@ -1,0 +1,308 @@
+"""CPU oracle for the QLoRA linear layer (blockwise NF4 + double quantisation +
+LoRA forward/backward).
+
+TEST INFRASTRUCTURE ONLY.  This is a plain, slow, obviously correct numpy
+restatement of what the layer computes.  It shares no code with the CUDA
+library and imports nothing from it.  Only the test suite, the smoke check in
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of ``bench.py`` may
+import it; the product path never calls it.
+
+Sources, cited by page title and section:
+
+* [QLoRA-chkda] "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora) -- the
+  most precise page; it wins every conflict.
+* [FromZero2AI] "LoRA and QLoRA: Efficient Fine-Tuning of Large Language
+  Models" (fromzero2ai.dev).
+* [CodeThePapers] "Democratizing LLM Finetuning: A Deep Dive into QLoRA".
+
+Precision: the pages fix bf16 storage for W-hat, X, A, B (section "Double
+quantization and double dequantization", QLoRA expression) and an fp32 scale
+per block (section "First, how does k-bit quantization work?").  Quantisation
+arithmetic is therefore carried out in fp32 with IEEE round-to-nearest, each
+operation rounded once, exactly as written.  Matrix products, whose
+accumulation precision the pages leave open, are done in fp64 on the exact
+fp32 images of the bf16 inputs.
+
+Readings of passages that are silent or ambiguous:
+
+R1  Codebook: C = {Phi^-1(p_i)/Phi^-1(p*)} with 8 positive p_i evenly spaced on
+    (1/2, p*] and 7 negative values mirrored from 7 evenly spaced p on
+    (1/2, p*], plus an exact 0.  The tail cutoff p* is the midpoint of the
+    interval of cutoffs that reproduces all 16 printed 4-decimal values.
+R2  Nearest code: distances |RN32(xn - C[j])| in fp32, first minimum wins
+    (the page's "choose the smaller index").
+R3  xn = RN32(w / s) with IEEE division; codes use the exact block absmax.
+R4  Packing: byte t = code[2t] | code[2t+1] << 4, an odd tail padded with 0.
+R5  Double quantisation: the page's only spelled-out 8-bit scheme (symmetric
+    Int8 absmax, Q = 127) with c1 = RN32(127 / absmax) stored in fp32,
+    "round" = round half to even, an all-zero group stored as zeros with
+    c1 = 1.  One mean per tensor, mu = RN32(RN64(RN64(sum s_j) / M_b)).
+R6  Scale reconstruction s^_j = RN32(RN32(c2_j / c1_g) + mu);
+    weight reconstruction w^ = BF16_RNE(RN32(C[q] * s^)).
+R7  Forward Y = X W^T + (alpha/r) (X A^T) B^T with W^ the reconstructed bf16
+    weights; backward derived by calculus (the pages print no formulas):
+    U = dY B, dX = dY W^ + s U A, dA = s U^T X, dB = s dY^T T, T = X A^T.
+"""
+from __future__ import annotations
+
+import math
+from statistics import NormalDist
+
+import numpy as np
+
+__all__ = [
+    "TAIL_CUTOFF", "codebook_values", "nf4_codebook", "bf16_round_bits", "bf16_bits_to_f32",
+    "nearest_code", "nf4_quantize", "pack_codes", "unpack_codes", "int8_absmax_quantize",
+    "int8_dequantize", "exact_mean_f32", "double_quantize", "double_dequantize_scales",
+    "nf4_dequantize", "quantize_tensor", "dequantize_tensor", "storage_bits_per_weight",
+    "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale",
+]
+
+BLOCK = 64          # weights per NF4 block ([QLoRA-chkda] "QLoRA uses blocks of 64 weights")
+DQ_GROUP = 256      # block scales per second-level group ([QLoRA-chkda] double quantization)
+INT8_Q = 127        # symmetric Int8 range [-127, 127] ([QLoRA-chkda] k-bit quantization)
+
+# Interval of tail cutoffs p* that reproduce every printed 4-decimal NF4 value
+# ([QLoRA-chkda] "NF4: Choose the codebook to fit the distribution"); found by
+# bisection on codebook_values(p) against the printed table.  Entry 4 (-0.2844)
+# binds the lower end, entry 6 (-0.0911) the upper end.
+TAIL_CUTOFF_INTERVAL = (0.9677023838639995, 0.9677082837944422)
+TAIL_CUTOFF = 0.9677053338292209  # midpoint (reading R1)
+
+
+# ----------------------------------------------------------------------------
+# bf16 helpers (storage rounding written out on the bit pattern)
+# ----------------------------------------------------------------------------
+def bf16_round_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bits, round to nearest, ties to even (finite inputs)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (u >> np.uint64(16)) & np.uint64(1)
+    return ((u + np.uint64(0x7FFF) + lsb) >> np.uint64(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# NF4 codebook  ([QLoRA-chkda] "NF4: Choose the codebook to fit the
+# distribution" and "Building the NF4 codebook")
+# ----------------------------------------------------------------------------
+def codebook_values(p_star: float = TAIL_CUTOFF) -> list[float]:
+    """The 16 NF4 values in float64 for a given tail cutoff p* (reading R1).
+
+    Evenly spaced probabilities on (1/2, p*] become normal quantiles; the
+    largest is normalised to 1.  Eight positive and seven negative values plus
+    an exact zero, as the page requires.
+    """
+    inv = NormalDist().inv_cdf
+    top = inv(p_star)
+    pos = [inv(0.5 + (p_star - 0.5) * i / 8) / top for i in range(1, 9)]
+    neg = [-inv(0.5 + (p_star - 0.5) * i / 7) / top for i in range(1, 8)]
+    return sorted(neg) + [0.0] + pos
+
+
+def nf4_codebook() -> np.ndarray:
+    """The frozen fp32 NF4 table C[0..15], ascending."""
+    return np.array(codebook_values(TAIL_CUTOFF), dtype=np.float64).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# NF4 blockwise quantisation  ([QLoRA-chkda] "Quantizing and dequantizing with
+# the codebook")
+# ----------------------------------------------------------------------------
+def nearest_code(xn: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """argmin_j |xn - C[j]| with fp32 distances; the first minimum wins (R2)."""
+    xn = np.asarray(xn, dtype=np.float32)
+    dist = np.abs(xn[..., None] - C.astype(np.float32))          # fp32 subtract, exact abs
+    return np.argmin(dist, axis=-1).astype(np.uint8)             # argmin returns the first minimum
+
+
+def nf4_quantize(w: np.ndarray, blocksize: int = BLOCK, C: np.ndarray | None = None):
+    """Blockwise NF4 quantisation of a flat fp32 array (values exact in bf16).
+
+    Per block: scale = |w[argmax |w|]|; if scale == 0 every code is the
+    argmin of |C| (the exact zero); otherwise code = nearest(w / scale).
+    The last block may be shorter.  Returns (codes uint8[N], absmax f32[M_b]).
+    """
+    C = nf4_codebook() if C is None else C
+    w = np.asarray(w, dtype=np.float32).ravel()
+    n = w.size
+    nblk = -(-n // blocksize)
+    codes = np.empty(n, dtype=np.uint8)
+    absmax = np.empty(nblk, dtype=np.float32)
+    zero_code = int(np.argmin(np.abs(C)))
+    step = 4096 * blocksize                     # chunk only to bound memory
+    for c0 in range(0, n, step):
+        seg = w[c0:c0 + step]
+        nb = -(-seg.size // blocksize)
+        padded = np.zeros(nb * blocksize, dtype=np.float32)
+        padded[:seg.size] = seg
+        blocks = padded.reshape(nb, blocksize)
+        s = np.max(np.abs(blocks), axis=1)      # |w[argmax]| equals the max magnitude
+        absmax[c0 // blocksize:c0 // blocksize + nb] = s
+        safe = np.where(s == 0, np.float32(1), s)
+        xn = (blocks / safe[:, None]).astype(np.float32)   # IEEE fp32 division (R3)
+        q = nearest_code(xn, C)
+        q[s == 0, :] = zero_code
+        codes[c0:c0 + seg.size] = q.ravel()[:seg.size]
+    return codes, absmax
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte, element 2t in the low nibble (reading R4)."""
+    codes = np.asarray(codes, dtype=np.uint8).ravel()
+    if codes.size % 2:
+        codes = np.concatenate([codes, np.zeros(1, np.uint8)])
+    return (codes[0::2] | (codes[1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray, n: int) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(packed.size * 2, dtype=np.uint8)
+    out[0::2] = packed & 0x0F
+    out[1::2] = packed >> 4
+    return out[:n]
+
+
+# ----------------------------------------------------------------------------
+# Symmetric Int8 absmax quantisation  ([QLoRA-chkda] "First, how does k-bit
+# quantization work?")
+# ----------------------------------------------------------------------------
+def int8_absmax_quantize(x: np.ndarray):
+    """c = 127 / absmax(x) in fp32; q = round(c * x) with round-half-even.
+
+    An all-zero input is stored as zeros with the nonzero scale c = 1.
+    Returns (q int8, c float32).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    a = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    if a == 0:
+        return np.zeros(x.shape, np.int8), np.float32(1.0)
+    c = np.float32(INT8_Q) / a                                   # fp32 division
+    q = np.rint((c * x).astype(np.float32))                      # fp32 product, ties to even
+    q = np.clip(q, -INT8_Q, INT8_Q).astype(np.int8)
+    return q, np.float32(c)
+
+
+def int8_dequantize(q: np.ndarray, c) -> np.ndarray:
+    """x^ = q / c in fp32."""
+    return (np.asarray(q).astype(np.float32) / np.float32(c)).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# Double quantisation  ([QLoRA-chkda] "Double quantization and double
+# dequantization")
+# ----------------------------------------------------------------------------
+def exact_mean_f32(s: np.ndarray) -> np.float32:
+    """mu = RN32(RN64(RN64(sum s) / M)), the sum correctly rounded (math.fsum)."""
+    s = np.asarray(s, dtype=np.float32)
+    total = math.fsum(float(v) for v in s.tolist())
+    return np.float32(total / s.size)
+
+
+def double_quantize(absmax: np.ndarray, group: int = DQ_GROUP):
+    """Quantise the block scales: subtract the tensor mean, then Int8 absmax per
+    group of 256 scales.  Returns (c2 int8[M_b], c1 f32[G], mean f32)."""
+    absmax = np.asarray(absmax, dtype=np.float32)
+    mu = exact_mean_f32(absmax)
+    v = (absmax - mu).astype(np.float32)
+    ng = -(-absmax.size // group)
+    c2 = np.empty(absmax.size, np.int8)
+    c1 = np.empty(ng, np.float32)
+    for g in range(ng):
+        q, c = int8_absmax_quantize(v[g * group:(g + 1) * group])
+        c2[g * group:(g + 1) * group] = q
+        c1[g] = c
+    return c2, c1, mu
+
+
+def double_dequantize_scales(c2: np.ndarray, c1: np.ndarray, mean, group: int = DQ_GROUP) -> np.ndarray:
+    """scales[j] = dequantize(c2[j], c1[j // 256]) + mean, each op rounded to fp32."""
+    c2 = np.asarray(c2, dtype=np.int8)
+    g = np.arange(c2.size) // group
+    deq = (c2.astype(np.float32) / np.asarray(c1, np.float32)[g]).astype(np.float32)
+    return (deq + np.float32(mean)).astype(np.float32)
+
+
+def nf4_dequantize(codes: np.ndarray, scales: np.ndarray, blocksize: int = BLOCK,
+                   C: np.ndarray | None = None) -> np.ndarray:
+    """weights[i] = BF16(C[codes[i]] * scales[i // 64]); returns bf16 bits."""
+    C = nf4_codebook() if C is None else C
+    codes = np.asarray(codes, dtype=np.uint8).ravel()
+    blk = np.arange(codes.size) // blocksize
+    prod = (C[codes].astype(np.float32) * np.asarray(scales, np.float32)[blk]).astype(np.float32)
+    return bf16_round_bits(prod)
+
+
+def quantize_tensor(w_bits: np.ndarray, double_quant: bool = True, blocksize: int = BLOCK) -> dict:
+    """Full quantisation of a bf16 weight (bits): codes, packed bytes and constants."""
+    w = bf16_bits_to_f32(np.asarray(w_bits).ravel())
+    codes, absmax = nf4_quantize(w, blocksize)
+    out = {"n": w.size, "codes": codes, "packed": pack_codes(codes), "absmax": absmax,
+           "double_quant": bool(double_quant)}
+    if double_quant:
+        c2, c1, mu = double_quantize(absmax)
+        out.update(c2=c2, c1=c1, mean=mu)
+    return out
+
+
+def dequantize_tensor(q: dict, blocksize: int = BLOCK) -> np.ndarray:
+    """doubleDequant (or single dequant when DQ is off); returns bf16 bits."""
+    if q["double_quant"]:
+        scales = double_dequantize_scales(q["c2"], q["c1"], q["mean"])
+    else:
+        scales = q["absmax"]
+    codes = unpack_codes(q["packed"], q["n"])
+    return nf4_dequantize(codes, scales, blocksize)
+
+
+def storage_bits_per_weight(double_quant: bool, blocksize: int = BLOCK, group: int = DQ_GROUP) -> float:
+    """Scale overhead in bits per weight ([QLoRA-chkda] 0.373-bit accounting)."""
+    if not double_quant:
+        return 32.0 / blocksize
+    return 8.0 / blocksize + 32.0 / (group * blocksize)
+
+
+# ----------------------------------------------------------------------------
+# LoRA / QLoRA linear layer  ([QLoRA-chkda] "How does it work?", "How does
+# alpha/r control adapter strength?", QLoRA expression; [FromZero2AI] "Low-Rank
+# Matrix Factorization")
+# ----------------------------------------------------------------------------
+def lora_trainable_params(d: int, k: int, r: int) -> int:
+    """(r x k) + (d x r) trainable entries for one adapted matrix."""
+    return r * k + d * r
+
+
+def lora_scale(alpha: float, r: int) -> np.float32:
+    return np.float32(np.float32(alpha) / np.float32(r))
+
+
+def _f64(a):
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        a = bf16_bits_to_f32(a)
+    return a.astype(np.float64)
+
+
+def qlora_forward(X, W_hat, A, B, alpha: float, r: int):
+    """Y = X W^T + s (X A^T) B^T, s = alpha / r; returns (Y, T) in fp64.
+
+    X (M x k), W_hat (d x k), A (r x k), B (d x r); bf16-bit arrays or floats.
+    """
+    X, W_hat, A, B = map(_f64, (X, W_hat, A, B))
+    s = float(lora_scale(alpha, r))
+    T = X @ A.T
+    return X @ W_hat.T + s * (T @ B.T), T
+
+
+def qlora_backward(dY, X, W_hat, A, B, alpha: float, r: int):
+    """Gradients of the forward for the frozen base (no dW0): returns dX, dA, dB."""
+    dY, X, W_hat, A, B = map(_f64, (dY, X, W_hat, A, B))
+    s = float(lora_scale(alpha, r))
+    T = X @ A.T
+    U = dY @ B
+    dX = dY @ W_hat + s * (U @ A)
+    dA = s * (U.T @ X)
+    dB = s * (dY.T @ T)
+    return dX, dA, dB
