@@ -1,0 +1,231 @@
+"""QLoRA linear layer for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding of ``libqlora.so`` (C ABI in ``include/qlora.h``).  The
+functions below only marshal arguments: every step of quantisation,
+dequantisation, forward and backward runs in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  There is no fallback: if the
+library is missing or a call fails, a ``QLoRAError`` is raised.
+
+Names follow the C ABI: ``nf4_quantize``, ``nf4_dequantize``,
+``qlora_linear_fwd``, ``qlora_linear_bwd``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_OK = 0
+_STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTED", -3: "QLORA_ERR_ALIGNMENT",
+           -4: "QLORA_ERR_WORKSPACE", -5: "QLORA_ERR_CUDA", -6: "QLORA_ERR_DEVICE"}
+
+EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_rank_pad", "qlora_linear_workspace_size",
+           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error")
+
+
+class QLoRAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{_STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class QloraNF4(ctypes.Structure):
+    """Mirror of ``qlora_nf4_t``."""
+    _fields_ = [("d", ctypes.c_int64), ("k", ctypes.c_int64), ("blocksize", ctypes.c_int32),
+                ("double_quant", ctypes.c_int32), ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
+                ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mean", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqlora.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise QLoRAError(-5, f"{LIB_PATH} is missing; build it with `python -m bit_quantized_lora_02_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    c_i64, c_i32, c_sz, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
+    L.qlora_nf4_sizes.argtypes = [c_i64, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz), ctypes.POINTER(c_sz)]
+    L.nf4_quantize.argtypes = [vp, ctypes.POINTER(QloraNF4), vp, c_sz, vp]
+    L.nf4_dequantize.argtypes = [ctypes.POINTER(QloraNF4), vp, vp]
+    L.qlora_rank_pad.argtypes = [c_i32]
+    L.qlora_rank_pad.restype = c_i32
+    L.qlora_linear_workspace_size.argtypes = [c_i64, c_i64, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz)]
+    L.qlora_linear_fwd.argtypes = [vp, c_i64, ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float, vp, vp, vp,
+                                   c_sz, vp]
+    L.qlora_linear_bwd.argtypes = [vp, vp, c_i64, ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float, vp, vp,
+                                   vp, vp, vp, c_sz, vp]
+    L.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
+    L.qlora_device_status.argtypes = [vp, ctypes.POINTER(c_i32)]
+    L.qlora_last_error.restype = ctypes.c_char_p
+    for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_linear_workspace_size",
+                 "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status"):
+        getattr(L, name).restype = c_i32
+    _lib = L
+    return L
+
+
+def _check(rc: int) -> None:
+    if rc != QLORA_OK:
+        raise QLoRAError(rc, lib().qlora_last_error().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# quantized weight container
+# ---------------------------------------------------------------------------
+@dataclass
+class NF4Weight:
+    """Device buffers of one quantized weight (layout of ``qlora_nf4_t``)."""
+    d: int
+    k: int
+    double_quant: bool
+    codes: torch.Tensor
+    absmax: Optional[torch.Tensor] = None
+    c2: Optional[torch.Tensor] = None
+    c1: Optional[torch.Tensor] = None
+    mean: Optional[torch.Tensor] = None
+    blocksize: int = 64
+
+    def struct(self) -> QloraNF4:
+        return QloraNF4(self.d, self.k, self.blocksize, int(self.double_quant), _ptr(self.codes), _ptr(self.absmax),
+                        _ptr(self.c2), _ptr(self.c1), _ptr(self.mean))
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.absmax, self.c2, self.c1, self.mean)
+                   if t is not None)
+
+
+def qlora_nf4_sizes(d: int, k: int, blocksize: int = 64, double_quant: bool = True):
+    """(sizes of codes, absmax, c2, c1, mean in bytes, quantize workspace bytes)."""
+    sizes = (ctypes.c_size_t * 5)()
+    ws = ctypes.c_size_t()
+    _check(lib().qlora_nf4_sizes(d, k, blocksize, int(double_quant), sizes, ctypes.byref(ws)))
+    return list(sizes), ws.value
+
+
+def nf4_alloc(d: int, k: int, double_quant: bool = True, device=None) -> NF4Weight:
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    sizes, _ = qlora_nf4_sizes(d, k, 64, double_quant)
+
+    def buf(n, dtype, esize):
+        # 16 extra bytes of slack keep vector accesses inside the allocation
+        return torch.empty(max(n // esize, 1) + 16 // esize, dtype=dtype, device=device)
+    codes = buf(sizes[0], torch.uint8, 1)
+    if double_quant:
+        return NF4Weight(d, k, True, codes, None, buf(sizes[2], torch.int8, 1), buf(sizes[3], torch.float32, 4),
+                         buf(sizes[4], torch.float32, 4))
+    return NF4Weight(d, k, False, codes, buf(sizes[1], torch.float32, 4))
+
+
+def nf4_quantize(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4Weight] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> NF4Weight:
+    """Blockwise NF4 (+ double quantisation) of a bf16 (d, k) weight."""
+    assert W0.dtype == torch.bfloat16 and W0.dim() == 2 and W0.is_contiguous()
+    d, k = W0.shape
+    q = out or nf4_alloc(d, k, double_quant, W0.device)
+    _, ws_bytes = qlora_nf4_sizes(d, k, 64, q.double_quant)
+    if workspace is None and ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=W0.device)
+    st = q.struct()
+    _check(lib().nf4_quantize(W0.data_ptr(), ctypes.byref(st), _ptr(workspace),
+                              0 if workspace is None else workspace.numel() * workspace.element_size(),
+                              _stream(stream)))
+    return q
+
+
+def nf4_dequantize(q: NF4Weight, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """doubleDequant into a bf16 (d, k) tensor."""
+    if out is None:
+        out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
+    st = q.struct()
+    _check(lib().nf4_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def qlora_rank_pad(r: int) -> int:
+    return int(lib().qlora_rank_pad(r))
+
+
+def qlora_linear_workspace_size(M: int, d: int, k: int, r: int, backward: bool) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().qlora_linear_workspace_size(M, d, k, r, int(backward), ctypes.byref(n)))
+    return n.value
+
+
+def qlora_linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     Y: Optional[torch.Tensor] = None, T_save: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None, save_T: bool = True):
+    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns (Y, T_save)."""
+    M, k = X.shape
+    r = A.shape[0]
+    dev = X.device
+    if Y is None:
+        Y = torch.empty(M, q.d, dtype=torch.bfloat16, device=dev)
+    if T_save is None and save_T:
+        T_save = torch.empty(M, qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        n = qlora_linear_workspace_size(M, q.d, q.k, r, False)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
+    st = q.struct()
+    _check(lib().qlora_linear_fwd(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha),
+                                  Y.data_ptr(), _ptr(T_save), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(), _stream(stream)))
+    return Y, T_save
+
+
+def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                     alpha: float, T_save: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,
+                     dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None, need_dX: bool = True):
+    """Gradients for the adapters and the input; returns (dX, dA, dB)."""
+    M = dY.shape[0]
+    r = A.shape[0]
+    dev = dY.device
+    if dX is None and need_dX:
+        dX = torch.empty(M, q.k, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(r, q.k, dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty(q.d, r, dtype=torch.float32, device=dev)
+    if workspace is None:
+        n = qlora_linear_workspace_size(M, q.d, q.k, r, True)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
+    st = q.struct()
+    _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
+                                  float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
+                                  _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
+    return dX, dA, dB
+
+
+def qlora_nf4_codebook():
+    buf = (ctypes.c_float * 16)()
+    _check(lib().qlora_nf4_codebook(buf))
+    return list(buf)
+
+
+def qlora_device_status(stream=None) -> int:
+    """Synchronize and return (and clear) the device status word; 0 = clean."""
+    s = ctypes.c_int32()
+    rc = lib().qlora_device_status(_stream(stream), ctypes.byref(s))
+    if rc not in (QLORA_OK, -6):
+        _check(rc)
+    return s.value

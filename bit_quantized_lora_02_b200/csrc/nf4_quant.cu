@@ -1,0 +1,445 @@
+// nf4_quant.cu -- blockwise NF4 quantisation with double quantisation of the
+// block constants, and the standalone double dequantisation.
+//
+// "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora):
+//   "Quantizing and dequantizing with the codebook"  (blocks of 64, absmax
+//      scale, nearest code with the smaller index on ties, exact-zero code for
+//      an all-zero block, reconstruction scale * C[code]);
+//   "First, how does k-bit quantization work?"       (Int8 absmax: c = 127 /
+//      absmax, q = round(c x), all-zero input -> zeros and a nonzero scale);
+//   "Double quantization and double dequantization"  (8-bit constants in groups
+//      of 256, one FP32 second-level scale per group, a stored mean;
+//      doubleDequant in BF16).
+//
+// Kernels (all memory-bound streaming kernels, no waits):
+//   k_nf4_quant    one pass over W0: block absmax (8-lane shuffle max), code
+//                  search, nibble packing; per-CTA exponent histogram of the
+//                  absmax values (for the exact mean) when DQ is on.
+//   k_dq_mean      one thread: exact sum of the histogram as a 320-bit
+//                  integer, correctly rounded to fp64, divided, rounded to fp32.
+//   k_dq_groups    one warp per group of 256 scales: subtract mean, absmax,
+//                  c1 = 127 / absmax, c2 = round-half-even(c1 * v).
+//   k_nf4_dequant  one pass over the codes: scale reconstruction and
+//                  BF16(C[q] * s^), 16-byte vector stores.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "nf4_table.h"
+#include "qlora_device.cuh"
+#include "qlora_internal.h"
+
+namespace qlora {
+
+__constant__ uint32_t c_nf4_bits[16] = {QLORA_NF4_TABLE_BITS};
+static const uint32_t h_nf4_bits[16] = {QLORA_NF4_TABLE_BITS};
+
+void host_codebook(float out[16]) { std::memcpy(out, h_nf4_bits, sizeof(h_nf4_bits)); }
+
+// ----------------------------------------------------------------------------
+// Code search table.
+//
+// The nearest-code rule compares fp32 distances |RN32(xn - C[j])| with the
+// smaller index winning ties.  Both distances are monotone in xn, so between
+// neighbours C[j] and C[j+1] the choice flips exactly once: t_j is the largest
+// fp32 xn for which C[j] still wins, and code(xn) = #{ j : xn > t_j }.
+//
+// To find which t_j to compare against with one lookup, xn is bucketed into 33
+// cells by cell(xn) = RN_even(16 xn + 16) (one FFMA against a 1.5 * 2^23 bias,
+// read off the low mantissa bits).  cell() is monotone, each cell holds at
+// most one threshold (neighbouring t_j are > 1/16 apart), so
+//     code(xn) = base[cell] + (xn > thr[cell])
+// with base[c] = #{ j : cell(t_j) < c } and thr[c] the threshold in cell c
+// (3.0, never exceeded, when the cell has none).  This is exact for every fp32
+// xn in [-1, 1]; the host builds the table once from C with IEEE fp32
+// arithmetic.
+// ----------------------------------------------------------------------------
+constexpr float kCellBias = 12582928.0f;   // 1.5 * 2^23 + 16
+constexpr uint32_t kCellBiasBits = 0x4B400000u;
+
+struct QuantLut {
+  float thr[33];
+  float base[33];  // integer counts stored as fp32 bit patterns
+};
+
+static float f_of(uint32_t u) {
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+static bool left_wins(float x, float a, float b) {
+  volatile float da = x - a;   // each difference rounded to fp32 once
+  volatile float db = x - b;
+  return std::fabs(da) <= std::fabs(db);
+}
+
+static int host_cell(float x) {
+  float y = std::fmaf(x, 16.0f, kCellBias);
+  uint32_t u;
+  std::memcpy(&u, &y, 4);
+  return static_cast<int>(u - kCellBiasBits);
+}
+
+static bool g_lut_ok = false;
+
+static QuantLut build_lut() {
+  QuantLut L;
+  float C[16];
+  for (int j = 0; j < 16; ++j) C[j] = f_of(h_nf4_bits[j]);
+  float t[15];
+  for (int j = 0; j < 15; ++j) {
+    float x = static_cast<float>((static_cast<double>(C[j]) + static_cast<double>(C[j + 1])) * 0.5);
+    while (!left_wins(x, C[j], C[j + 1])) x = std::nextafterf(x, -2.0f);
+    for (;;) {
+      float up = std::nextafterf(x, 2.0f);
+      if (!left_wins(up, C[j], C[j + 1])) break;
+      x = up;
+    }
+    t[j] = x;
+  }
+  int cell_of[15];
+  bool ok = true;
+  for (int j = 0; j < 15; ++j) {
+    cell_of[j] = host_cell(t[j]);
+    if (cell_of[j] < 0 || cell_of[j] > 32) ok = false;
+    if (j && cell_of[j] <= cell_of[j - 1]) ok = false;     // at most one threshold per cell
+    if (j && !(t[j] > t[j - 1])) ok = false;
+  }
+  for (int c = 0; c <= 32; ++c) {
+    uint32_t base = 0;
+    float thr = 3.0f;
+    for (int j = 0; j < 15; ++j) {
+      if (cell_of[j] < c) ++base;
+      if (cell_of[j] == c) thr = t[j];
+    }
+    L.thr[c] = thr;
+    std::memcpy(&L.base[c], &base, 4);
+  }
+  g_lut_ok = ok;
+  return L;
+}
+
+static const QuantLut& quant_lut() {
+  static QuantLut lut;
+  static std::once_flag once;
+  std::call_once(once, [] { lut = build_lut(); });
+  return lut;
+}
+
+bool quant_lut_valid() {
+  quant_lut();
+  return g_lut_ok;
+}
+
+void quant_thresholds(float out[15]) {
+  // the decision thresholds t_j, recovered from the cell table (host only)
+  const QuantLut& L = quant_lut();
+  int j = 0;
+  for (int c = 0; c <= 32 && j < 15; ++c)
+    if (L.thr[c] < 2.0f) out[j++] = L.thr[c];
+}
+
+// ----------------------------------------------------------------------------
+// Quantisation kernel
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// xn = RN32(w / s).  For a block scale in [2^-60, 2^60] this uses the
+// correctly rounded reciprocal r = RN32(1/s) and one residual correction
+// (Markstein's final division step: y = RN(w r); e = fma(-s, y, w);
+// q = fma(e, r, y)).  For bf16 operands this equals IEEE division whenever
+// |w/s| >= 2^-102 (checked exhaustively over all bf16 significand pairs);
+// smaller quotients all map to the exact-zero code either way.  Outside that
+// scale range the kernel falls back to IEEE division.
+__device__ __forceinline__ float quotient(float w, float s, float r, bool fast) {
+  if (fast) {
+    float y = __fmul_rn(w, r);
+    float e = __fmaf_rn(-s, y, w);
+    return __fmaf_rn(e, r, y);
+  }
+  return __fdiv_rn(w, s);
+}
+
+template <bool kDQ>
+__global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ W, int64_t N,
+                                                   uint8_t* __restrict__ codes, float* __restrict__ absmax_f32,
+                                                   uint16_t* __restrict__ absmax_bf16,
+                                                   unsigned long long* __restrict__ hist, const QuantLut lut) {
+  __shared__ float2 s_lut[33];
+  __shared__ uint32_t s_hist[256];
+  const int tid = threadIdx.x;
+  if (tid < 33) s_lut[tid] = make_float2(lut.thr[tid], lut.base[tid]);
+  if (kDQ) s_hist[tid] = 0;
+  __syncthreads();
+
+  const int lane = tid & 31;
+  const int64_t ngroups = (N + 7) >> 3;                      // groups of 8 elements
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+  for (int64_t g0 = static_cast<int64_t>(blockIdx.x) * 256 + (tid & ~31); g0 < ngroups; g0 += stride) {
+    const int64_t g = g0 + lane;
+    const int64_t e0 = g << 3;
+    float w[8];
+    const bool full = (e0 + 8 <= N);
+    if (full) {
+      uint4 v = ldg_nc_v4(W + e0);
+      w[0] = bf16_lo(v.x); w[1] = bf16_hi(v.x); w[2] = bf16_lo(v.y); w[3] = bf16_hi(v.y);
+      w[4] = bf16_lo(v.z); w[5] = bf16_hi(v.z); w[6] = bf16_lo(v.w); w[7] = bf16_hi(v.w);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = (e0 + i < N) ? __uint_as_float(static_cast<uint32_t>(W[e0 + i]) << 16) : 0.0f;
+    }
+    float am = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(w[i]));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
+    const float s = am;   // block absmax (bf16-exact)
+
+    uint32_t packed = 0x77777777u;   // exact-zero code for an all-zero block
+    if (s != 0.0f) {
+      const bool fast = (s >= 0x1p-60f) && (s <= 0x1p60f);
+      const float r = __frcp_rn(s);
+      packed = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float xn = quotient(w[i], s, r, fast);
+        const float y = __fmaf_rn(xn, 16.0f, kCellBias);
+        const float2 e = s_lut[__float_as_uint(y) - kCellBiasBits];
+        const uint32_t q = __float_as_uint(e.y) + (xn > e.x ? 1u : 0u);
+        packed |= q << (4 * i);
+      }
+    }
+    if (e0 < N) {
+      if (full) {
+        *reinterpret_cast<uint32_t*>(codes + (e0 >> 1)) = packed;
+      } else {
+        const int valid = static_cast<int>(N - e0);            // 1..7
+        const uint32_t keep = (1u << (4 * valid)) - 1u;          // pad nibbles are 0
+        packed &= keep;
+        const int nbytes = (valid + 1) >> 1;
+        for (int b = 0; b < nbytes; ++b) codes[(e0 >> 1) + b] = static_cast<uint8_t>(packed >> (8 * b));
+      }
+      if ((g & 7) == 0) {
+        const int64_t blk = e0 >> 6;
+        if (kDQ) {
+          const uint32_t bits = __float_as_uint(s);
+          absmax_bf16[blk] = static_cast<uint16_t>(bits >> 16);
+          const uint32_t E = (bits >> 23) & 0xFFu;
+          const uint32_t m = (bits >> 16) & 0x7Fu;
+          atomicAdd(&s_hist[E], E ? (128u + m) : m);
+        } else {
+          absmax_f32[blk] = s;
+        }
+      }
+    }
+  }
+  if (kDQ) {
+    __syncthreads();
+    const uint32_t h = s_hist[tid];
+    if (h) atomicAdd(&hist[tid], static_cast<unsigned long long>(h));
+  }
+}
+
+__global__ void k_zero_u64(unsigned long long* p, int n) {
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0ull;
+}
+
+// ----------------------------------------------------------------------------
+// Exact mean of the block scales.  Each scale is a bf16 value
+// sig * 2^(max(E,1) - 134) with an 8-bit significand; the histogram holds, per
+// exponent field E, the exact integer sum of significands.  The total is an
+// integer multiple of 2^-133 that fits in 5 64-bit limbs; it is rounded once
+// to fp64 (nearest, ties to even), divided by M_b in fp64 and rounded to fp32:
+// mean = RN32(RN64(RN64(sum) / M_b)).
+// ----------------------------------------------------------------------------
+__global__ void k_dq_mean(const unsigned long long* __restrict__ hist, int64_t nblocks, float* __restrict__ mean) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  // 32-bit limbs held in 64-bit words; limb i covers bits [32 i, 32 i + 32).
+  unsigned long long A[12];
+  for (int i = 0; i < 12; ++i) A[i] = 0ull;
+  for (int E = 0; E < 256; ++E) {
+    const unsigned long long v = hist[E];   // < 2^51
+    if (!v) continue;
+    const int sh = (E ? E : 1) - 1;        // position of 2^(max(E,1) - 134) in units of 2^-133
+    const int li = sh >> 5, bo = sh & 31;
+    A[li] += (v << bo) & 0xFFFFFFFFull;
+    A[li + 1] += (v >> (32 - bo)) & 0xFFFFFFFFull;
+    if (bo) A[li + 2] += v >> (64 - bo);
+  }
+  for (int i = 0; i < 11; ++i) {
+    A[i + 1] += A[i] >> 32;
+    A[i] &= 0xFFFFFFFFull;
+  }
+  auto bit = [&](int p) -> unsigned long long { return (p < 0) ? 0ull : ((A[p >> 5] >> (p & 31)) & 1ull); };
+  int top = -1;
+  for (int p = 12 * 32 - 1; p >= 0; --p)
+    if (bit(p)) { top = p; break; }
+  double S = 0.0;
+  if (top >= 0) {
+    if (top < 53) {
+      S = ldexp(static_cast<double>(A[0] | (A[1] << 32)), -133);    // exact
+    } else {
+      unsigned long long m = 0;
+      for (int p = top; p > top - 53; --p) m = (m << 1) | bit(p);
+      const int rpos = top - 53;
+      bool sticky = false;
+      for (int p = rpos - 1; p >= 0 && !sticky; --p) sticky = bit(p) != 0;
+      if (bit(rpos) && (sticky || (m & 1ull))) ++m;   // ties to even; 2^53 stays exact
+      S = ldexp(static_cast<double>(m), top - 52 - 133);
+    }
+  }
+  *mean = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblocks)));
+}
+
+// ----------------------------------------------------------------------------
+// Double quantisation of the scales: one warp per group of 256.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ absmax_bf16, int64_t nblocks,
+                                                   const float* __restrict__ mean, int8_t* __restrict__ c2,
+                                                   float* __restrict__ c1) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int64_t ngroups = (nblocks + 255) >> 8;
+  if (g >= ngroups) return;
+  const float mu = *mean;
+  const int64_t j0 = g * 256 + lane * 8;
+  float v[8];
+  float am = 0.0f;
+  if (j0 + 8 <= nblocks) {
+    uint4 raw = ldg_nc_v4(absmax_bf16 + j0);
+    const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __fsub_rn(bf16_lo(r4[i]), mu);
+      v[2 * i + 1] = __fsub_rn(bf16_hi(r4[i]), mu);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[i] = (j0 + i < nblocks) ? __fsub_rn(__uint_as_float(static_cast<uint32_t>(absmax_bf16[j0 + i]) << 16), mu)
+                                : 0.0f;
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const float c = (am == 0.0f) ? 1.0f : __fdiv_rn(127.0f, am);
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int q = 0;
+    if (am != 0.0f) {
+      q = __float2int_rn(__fmul_rn(c, v[i]));
+      q = max(-127, min(127, q));
+    }
+    const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
+    if (i < 4) lo |= b << (8 * i);
+    else hi |= b << (8 * (i - 4));
+  }
+  if (j0 + 8 <= nblocks) {
+    *reinterpret_cast<uint2*>(c2 + j0) = make_uint2(lo, hi);
+  } else {
+    for (int i = 0; i < 8; ++i)
+      if (j0 + i < nblocks) c2[j0 + i] = static_cast<int8_t>(((i < 4) ? (lo >> (8 * i)) : (hi >> (8 * (i - 4)))) & 0xFFu);
+  }
+  if (lane == 0) c1[g] = c;
+}
+
+// ----------------------------------------------------------------------------
+// Standalone double dequantisation: W_out[i] = BF16(RN32(C[q_i] * s^_j)).
+// ----------------------------------------------------------------------------
+template <bool kDQ>
+__global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__ codes, int64_t N,
+                                                     const float* __restrict__ absmax, const int8_t* __restrict__ c2,
+                                                     const float* __restrict__ c1, const float* __restrict__ mean,
+                                                     uint16_t* __restrict__ out) {
+  __shared__ float s_C[16];
+  if (threadIdx.x < 16) s_C[threadIdx.x] = __uint_as_float(c_nf4_bits[threadIdx.x]);
+  __syncthreads();
+  const float mu = kDQ ? *mean : 0.0f;
+  const int64_t ngroups = (N + 7) >> 3;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
+    const int64_t e0 = g << 3;
+    const int64_t blk = e0 >> 6;
+    float sh;
+    if (kDQ) sh = __fadd_rn(__fdiv_rn(static_cast<float>(c2[blk]), c1[blk >> 8]), mu);
+    else sh = absmax[blk];
+    const bool full = (e0 + 8 <= N);
+    uint32_t cw;
+    if (full) {
+      cw = __ldg(reinterpret_cast<const unsigned int*>(codes + (e0 >> 1)));
+    } else {
+      cw = 0;
+      const int nbytes = static_cast<int>((N - e0 + 1) >> 1);
+      for (int b = 0; b < nbytes; ++b) cw |= static_cast<uint32_t>(codes[(e0 >> 1) + b]) << (8 * b);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float a = __fmul_rn(s_C[(cw >> (8 * i)) & 15u], sh);
+      const float b = __fmul_rn(s_C[(cw >> (8 * i + 4)) & 15u], sh);
+      o[i] = pack_bf16x2(a, b);
+    }
+    if (full) {
+      *reinterpret_cast<uint4*>(out + e0) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      for (int i = 0; e0 + i < N; ++i) out[e0 + i] = static_cast<uint16_t>(o[i >> 1] >> (16 * (i & 1)));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host launchers
+// ----------------------------------------------------------------------------
+static int grid_for(int64_t ngroups8) {
+  int64_t ctas = (ngroups8 + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (ctas > cap) ctas = cap;
+  if (ctas < 1) ctas = 1;
+  return static_cast<int>(ctas);
+}
+
+size_t quant_workspace_bytes(int64_t N, bool dq) {
+  if (!dq) return 0;
+  const int64_t nblk = (N + 63) / 64;
+  return 256 * sizeof(unsigned long long) + align_up(static_cast<size_t>(nblk) * 2 + 16, 256);
+}
+
+cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, void* ws, cudaStream_t st) {
+  const int64_t ng8 = (N + 7) / 8;
+  const int grid = grid_for(ng8);
+  const int64_t nblk = (N + 63) / 64;
+  if (!q.double_quant) {
+    k_nf4_quant<false><<<grid, 256, 0, st>>>(W, N, q.codes, q.absmax, nullptr, nullptr, quant_lut());
+    return cudaGetLastError();
+  }
+  auto* hist = static_cast<unsigned long long*>(ws);
+  auto* amax16 = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256 * sizeof(unsigned long long));
+  k_zero_u64<<<1, 256, 0, st>>>(hist, 256);
+  k_nf4_quant<true><<<grid, 256, 0, st>>>(W, N, q.codes, nullptr, amax16, hist, quant_lut());
+  k_dq_mean<<<1, 32, 0, st>>>(hist, nblk, q.mean);
+  const int64_t ngroups = (nblk + 255) / 256;
+  k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, q.mean, q.c2, q.c1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st) {
+  const int grid = grid_for((N + 7) / 8);
+  if (q.double_quant)
+    k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
+  else
+    k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
+  return cudaGetLastError();
+}
+
+}  // namespace qlora

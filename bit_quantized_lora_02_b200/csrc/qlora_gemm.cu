@@ -1,0 +1,1132 @@
+// qlora_gemm.cu -- the QLoRA linear layer's forward and backward on tcgen05
+// tensor cores.
+//
+// "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora):
+//   "How does it work?" / "How does alpha/r control adapter strength?"
+//       h = W0 x + (alpha/r) B (A x), A r x k, B d x r;
+//   "Double quantization and double dequantization"
+//       Y = X doubleDequant(c1, c2, W_NF4) + X L1 L2 in BF16, and the backward
+//       that flows "through the reconstructed base transformations" into the
+//       adapters only (no gradient for the 4-bit weights).
+//
+// With s = alpha / r (fp32) the library computes
+//     T_s = BF16(s X A^T)                 (M x rp, rp = r padded to 64)
+//     Y   = X W^T + T_s B^T               (one GEMM: [X | T_s] [W | B]^T)
+//     U_s = BF16(s dY B)                  (M x rp)
+//     dX  = dY W + U_s A                  (one GEMM: [dY | U_s] [W ; A])
+//     dA  = U_s^T X,   dB = dY^T T_s      (fp32)
+// where W = doubleDequant(...) is rebuilt tile by tile in shared memory and
+// never written to device memory.
+//
+// Kernels
+//   k_qlora_main<Fwd>     Y tile 128 tokens x 256 weight rows.  TMA stages X
+//                         and the packed codes; 8 dequant warps expand the codes
+//                         to bf16 in the 128-byte-swizzled K-major layout the
+//                         tensor core reads; one thread issues tcgen05.mma into
+//                         a 128 x 256 fp32 TMEM accumulator; the LoRA term is
+//                         one (or more) extra 64-wide K steps.
+//   k_qlora_main<Bwd>     dX tile 128 tokens x 256 input columns; the dequant
+//                         warps write W in the MN-major swizzled layout (the
+//                         reduction runs over W's rows).
+//   k_qlora_main<FwdSwap> few tokens (M <= 128): W rows are the MMA's M side
+//                         (128 per tile), the tokens its N side, so the tensor
+//                         core is not padded to 128 tokens; split over K.
+//   k_thin<false,false>   T_s and U_s partial sums (K-major operands).
+//   k_thin<true,true>     dA^T and dB partial sums (MN-major operands, the
+//                         reduction runs over tokens).
+//   k_reduce_*            deterministic sums of split-K partials.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nf4_table.h"
+#include "qlora_device.cuh"
+#include "qlora_internal.h"
+
+namespace qlora {
+
+__constant__ uint32_t c_nf4_gemm[16] = {QLORA_NF4_TABLE_BITS};
+
+// ============================================================================
+// Tensor maps
+// ============================================================================
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor: `inner` elements per row (contiguous), `outer` rows,
+// `row_bytes` between rows.  Box = box_inner x box_outer.
+static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                     uint32_t box_rows) {
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows, true);
+}
+
+// ============================================================================
+// Dequantisation of one 64-weight NF4 block into a 128-byte swizzled row.
+//
+// The block's 16 reconstruction values T[j] = BF16(RN32(C[j] * s^)) are built
+// once per block (bit-identical to BF16(C[q] * s^) per weight), split into four
+// registers of low bytes and four of high bytes, and every 4-bit code is then
+// resolved with byte permutes: PRMT selects by the code's low 3 bits from each
+// half of the table and a sign-replicated mask of the code's top bit picks the
+// half.  About 2.75 integer instructions per weight, no shared-memory lookups.
+// ============================================================================
+struct Nf4Tab {
+  uint32_t L[4], H[4];
+};
+
+__device__ __forceinline__ Nf4Tab make_tab(float sh, const float (&C)[16]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(C[2 * i], sh), __fmul_rn(C[2 * i + 1], sh));
+  Nf4Tab t;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    t.L[i] = prmt(P[2 * i], P[2 * i + 1], 0x6420u);
+    t.H[i] = prmt(P[2 * i], P[2 * i + 1], 0x7531u);
+  }
+  return t;
+}
+
+// 8 codes (code i in bits 4i..4i+3) -> 8 bf16 (element i in halfword i).
+__device__ __forceinline__ uint4 dq8(uint32_t c, const Nf4Tab& t) {
+  const uint32_t xl = c & 0x7777u;
+  const uint32_t xh = (c >> 16) & 0x7777u;
+  const uint32_t d4 = c << 4;
+  const uint32_t ml = prmt(d4, c, 0xD9C8u);   // 0xFF in byte i iff code i >= 8 (i = 0..3)
+  const uint32_t mh = prmt(d4, c, 0xFBEAu);   // same for codes 4..7
+  uint4 o;
+  {
+    const uint32_t la = prmt(t.L[0], t.L[1], xl), lb = prmt(t.L[2], t.L[3], xl);
+    const uint32_t ha = prmt(t.H[0], t.H[1], xl), hb = prmt(t.H[2], t.H[3], xl);
+    const uint32_t lo = (la & ~ml) | (lb & ml);
+    const uint32_t hi = (ha & ~ml) | (hb & ml);
+    o.x = prmt(lo, hi, 0x5140u);
+    o.y = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t la = prmt(t.L[0], t.L[1], xh), lb = prmt(t.L[2], t.L[3], xh);
+    const uint32_t ha = prmt(t.H[0], t.H[1], xh), hb = prmt(t.H[2], t.H[3], xh);
+    const uint32_t lo = (la & ~mh) | (lb & mh);
+    const uint32_t hi = (ha & ~mh) | (hb & mh);
+    o.z = prmt(lo, hi, 0x5140u);
+    o.w = prmt(lo, hi, 0x7362u);
+  }
+  return o;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+// Block scale s^ for NF4 block `blk`.
+struct ScaleSrc {
+  const float* absmax;   // DQ off
+  const int8_t* c2;      // DQ on
+  const float* c1;
+  const float* mean;     // device scalar, DQ on
+  int dq;
+};
+
+struct ScaleRaw {
+  float a;   // absmax (DQ off) or c1 (DQ on)
+  int b;     // c2
+};
+
+__device__ __forceinline__ ScaleRaw scale_fetch(const ScaleSrc& s, int64_t blk) {
+  ScaleRaw r;
+  if (s.dq) {
+    r.b = __ldg(s.c2 + blk);
+    r.a = __ldg(s.c1 + (blk >> 8));
+  } else {
+    r.a = __ldg(s.absmax + blk);
+    r.b = 0;
+  }
+  return r;
+}
+
+// s^ = RN32(RN32(c2 / c1) + mean) with DQ, else the stored absmax.
+__device__ __forceinline__ float scale_value(int dq, float mean, ScaleRaw r) {
+  return dq ? __fadd_rn(__fdiv_rn(static_cast<float>(r.b), r.a), mean) : r.a;
+}
+
+// ============================================================================
+// Main fused kernel
+// ============================================================================
+enum class Mode : int { Fwd = 0, Bwd = 1, FwdSwap = 2 };
+
+struct MainParams {
+  int64_t M, d, k;
+  int32_t r, rp;
+  int32_t kpb;              // NF4 blocks per weight row (k / 64)
+  ScaleSrc sc;
+  const uint16_t* lora;     // Fwd/FwdSwap: B (d x r); Bwd: A (r x k)
+  uint16_t* out;            // bf16 output (splits == 1)
+  float* partial;           // fp32 [splits][M][n_out] (splits > 1)
+  int64_t n_out;            // output columns: d (Fwd/FwdSwap) or k (Bwd)
+  int32_t steps_main;       // main K steps in total
+  int32_t steps_per_split;
+  int32_t ext_steps;        // rp / 64
+  int32_t splits;
+};
+
+template <Mode MODE, int NT>
+struct MainCfg {
+  static constexpr bool kSwap = MODE == Mode::FwdSwap;
+  static constexpr bool kBwd = MODE == Mode::Bwd;
+  static constexpr int kWRows = kSwap ? 128 : (kBwd ? 64 : 256);      // W rows per K step
+  static constexpr int kWCols = kBwd ? 256 : 64;                       // W columns per K step
+  static constexpr int kActRows = kSwap ? NT : 128;                    // token rows per K step
+  static constexpr int kMmaN = kSwap ? NT : 256;
+  static constexpr uint32_t kActBytes = kActRows * 128;
+  static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
+  static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
+  static constexpr uint32_t kStageBytes = kActBytes + kWBytes + kCodeBytes;
+  static constexpr int kStagesRaw = static_cast<int>((200u * 1024u) / kStageBytes);
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr uint32_t kTmemCols = kMmaN <= 32 ? 32 : (kMmaN <= 64 ? 64 : (kMmaN <= 128 ? 128 : 256));
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kThreads = 384;
+  static constexpr uint32_t kIdesc = make_idesc_bf16(128, kMmaN, false, kBwd);
+};
+
+template <Mode MODE, int NT>
+__global__ void __launch_bounds__(384, 1)
+    k_qlora_main(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+                 const __grid_constant__ CUtensorMap tm_ext, const MainParams p) {
+  using Cfg = MainCfg<MODE, NT>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;            // TMA data landed (act + codes)
+  uint64_t* deq_bar = bars + S;         // dequant warps finished the W tile
+  uint64_t* empty_bar = bars + 2 * S;   // MMAs reading the stage completed
+  uint64_t* tmem_full = bars + 3 * S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // tile coordinates
+  int64_t m0 = 0, n0 = 0;   // token row / output column of the tile (non-swap); W row (swap)
+  if (Cfg::kSwap) {
+    n0 = static_cast<int64_t>(blockIdx.x) * 128;
+  } else {
+    n0 = static_cast<int64_t>(blockIdx.x) * 256;
+    m0 = static_cast<int64_t>(blockIdx.y) * 128;
+  }
+  const int split = blockIdx.z;
+  const int s_begin = split * p.steps_per_split;
+  const int s_end = min(p.steps_main, s_begin + p.steps_per_split);
+  const int n_main = max(0, s_end - s_begin);
+  const int n_local = n_main + (split == 0 ? p.ext_steps : 0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&deq_bar[i], 8);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(tmem_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_ext);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
+  auto w_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
+  auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes + Cfg::kWBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int l = 0; l < n_local; ++l) {
+        const int st = l % S;
+        const uint32_t ph = (l / S) & 1;
+        if (!mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
+        if (l < n_main) {
+          const int i = s_begin + l;
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes + Cfg::kCodeBytes);
+          if (Cfg::kSwap) {
+            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, 0);
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(n0));
+          } else if (Cfg::kBwd) {
+            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], static_cast<int>(n0 / 2), 64 * i);
+          } else {
+            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(n0));
+          }
+        } else {
+          const int e = l - n_main;
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes);
+          tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, Cfg::kSwap ? 0 : static_cast<int>(m0));
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let every copy still in flight land before the CTA exits
+        const int first = issued > S ? issued - S : 0;
+        for (int l = first; l < issued; ++l) {
+          const uint32_t a = smem_u32(&full_bar[l % S]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, (l / S) & 1) && globaltimer_ns() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int l = 0;
+      for (; l < n_local; ++l) {
+        const int st = l % S;
+        const uint32_t ph = (l / S) & 1;
+        if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
+        if (!mbar_wait(&deq_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
+        tc_fence_after();
+        const uint32_t a_act = smem_u32(act_tile(st));
+        const uint32_t a_w = smem_u32(w_tile(st));
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          uint64_t da, db;
+          const uint64_t d_act = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
+          if (Cfg::kSwap) {
+            da = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
+            db = d_act;
+          } else if (Cfg::kBwd) {
+            da = d_act;
+            db = make_sdesc_sw128(a_w + 2048u * kk, 8192u, 1024u);
+          } else {
+            da = d_act;
+            db = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
+          }
+          umma_bf16(tmem_base, da, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty_bar[st]);
+      }
+      umma_commit(tmem_full);   // also drains MMAs on the abort path
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ dequant warps
+    const int t = threadIdx.x - 128;   // 0..255
+    float C[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(c_nf4_gemm[j]);
+    const ScaleSrc sc = p.sc;
+    const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
+    // this thread's W row and block column inside the tile
+    int row, sub;   // Fwd: row = t; Swap: row = t >> 1, sub = half; Bwd: row = t & 63 (K row), sub = chunk
+    if (Cfg::kSwap) {
+      row = t >> 1;
+      sub = t & 1;
+    } else if (Cfg::kBwd) {
+      row = t & 63;
+      sub = t >> 6;
+    } else {
+      row = t;
+      sub = 0;
+    }
+    auto block_of = [&](int i, bool& valid) -> int64_t {
+      int64_t wr, bc;
+      if (Cfg::kBwd) {
+        wr = 64ll * i + row;
+        bc = n0 / 64 + sub;
+        valid = (wr < p.d) && (bc < p.kpb);
+      } else {
+        wr = n0 + row;
+        bc = i;
+        valid = wr < p.d;
+      }
+      return wr * p.kpb + bc;
+    };
+    ScaleRaw pre{};
+    bool pre_valid = false;
+    if (n_main > 0) {
+      int64_t b0 = block_of(s_begin, pre_valid);
+      if (pre_valid) pre = scale_fetch(sc, b0);
+    }
+    for (int l = 0; l < n_local; ++l) {
+      const int st = l % S;
+      const uint32_t ph = (l / S) & 1;
+      bool okw = mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
+      okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      const uint32_t wt = smem_u32(w_tile(st));
+      if (l < n_main) {
+        const ScaleRaw cur = pre;
+        const bool cur_valid = pre_valid;
+        if (l + 1 < n_main) {   // prefetch the next step's constants
+          int64_t bn = block_of(s_begin + l + 1, pre_valid);
+          if (pre_valid) pre = scale_fetch(sc, bn);
+        }
+        const uint32_t ct = smem_u32(code_tile(st));
+        if (Cfg::kSwap) {
+          uint4 cw = lds128(ct + row * 32 + sub * 16);
+          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
+          if (cur_valid) {
+            const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sts128(wt + sw128_offset(row, 4 * sub + c), dq8(w4[c], tab));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) sts128(wt + sw128_offset(row, 4 * sub + c), make_uint4(0, 0, 0, 0));
+          }
+        } else {
+          const uint32_t src = Cfg::kBwd ? (ct + row * 128 + sub * 32) : (ct + row * 32);
+          const uint32_t dst = Cfg::kBwd ? (wt + sub * 8192) : wt;
+          uint4 c0 = lds128(src), c1 = lds128(src + 16);
+          const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+          if (cur_valid) {
+            const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sts128(dst + sw128_offset(row, c), dq8(w8[c], tab));
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) sts128(dst + sw128_offset(row, c), make_uint4(0, 0, 0, 0));
+          }
+        }
+      } else {
+        // LoRA extension step: copy 64 columns of the adapter into the W tile
+        const int e = l - n_main;
+        if (Cfg::kBwd) {
+          // A (r x k): K row j = 64e + row, N columns n0 + 64 sub + [0, 64)
+          const int64_t j = 64ll * e + row;
+          const int64_t c0 = n0 + 64 * sub;
+          const bool v = (j < p.r) && (c0 < p.k);
+          const uint16_t* src = p.lora + j * p.k + c0;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (v) val = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
+            sts128(wt + sub * 8192 + sw128_offset(row, c), val);
+          }
+        } else {
+          // B (d x r): row n, columns 64e + [0, 64) (Fwd) or a half of them (Swap)
+          const int64_t n = n0 + row;
+          const int cbeg = Cfg::kSwap ? 4 * sub : 0;
+          const int cnum = Cfg::kSwap ? 4 : 8;
+          for (int c = cbeg; c < cbeg + cnum; ++c) {
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int64_t j = 64ll * e + 8 * c + q;
+              h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
+            }
+            sts128(wt + sw128_offset(row, c),
+                   make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&deq_bar[st]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
+    tc_fence_after();
+    if (ok) {
+      const int q = warp & 3;          // TMEM lane quarter this warp may access
+      const int half = (warp - 4) >> 2;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+      if (!Cfg::kSwap) {
+        const int64_t m = m0 + 32 * q + lane;
+        for (int cb = 0; cb < 4; ++cb) {
+          const int col0 = 128 * half + 32 * cb;
+          uint32_t v[32];
+          tmem_ld32(lane_base + col0, v);
+          tmem_ld_wait();
+          if (m < p.M) {
+            const int64_t n = n0 + col0;
+            if (p.splits == 1) {
+              uint16_t* dst = p.out + m * p.n_out + n;
+#pragma unroll
+              for (int g = 0; g < 4; ++g) {
+                if (n + 8 * g + 8 <= p.n_out) {
+                  uint4 o;
+                  o.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
+                  o.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
+                  o.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
+                  o.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
+                  *reinterpret_cast<uint4*>(dst + 8 * g) = o;
+                }
+              }
+            } else {
+              float* dst = p.partial + (static_cast<int64_t>(split) * p.M + m) * p.n_out + n;
+#pragma unroll
+              for (int g = 0; g < 8; ++g)
+                if (n + 4 * g + 4 <= p.n_out)
+                  *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            }
+          }
+        }
+      } else if (half == 0) {
+        // lanes = W rows n, columns = tokens
+        const int64_t n = n0 + 32 * q + lane;
+        for (int cb = 0; cb < NT / 16; ++cb) {
+          uint32_t v[16];
+          tmem_ld16(lane_base + 16 * cb, v);
+          tmem_ld_wait();
+          if (n < p.d) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int64_t tok = 16 * cb + j;
+              if (tok < p.M) {
+                if (p.splits == 1) {
+                  const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f);
+                  p.out[tok * p.n_out + n] = static_cast<uint16_t>(b & 0xFFFFu);
+                } else {
+                  p.partial[(static_cast<int64_t>(split) * p.M + tok) * p.n_out + n] = __uint_as_float(v[j]);
+                }
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  if (warp == 1 && lane == 0) {
+    // the accumulator must be idle before its columns are released
+    const uint32_t a = smem_u32(tmem_full);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(a, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ============================================================================
+// Thin GEMM: D[128 x rp] += A_tile * B_tile^T over a K range, fp32 partials.
+//   kMN = false: A, B K-major (T_s: X and A; U_s: dY and B^T).
+//   kMN = true : A, B MN-major, reduction over tokens (dA^T: X^T and U_s;
+//                dB: dY^T and T_s).
+// ============================================================================
+struct ThinParams {
+  int64_t rows;          // output rows in total (M, k or d)
+  int32_t rp;            // output columns (multiple of 64)
+  int32_t steps;         // K steps in total
+  int32_t steps_per_split;
+  float* partial;        // [splits][rows][rp]
+};
+
+template <bool kMN>
+struct ThinCfg {
+  static constexpr int kStages = 4;
+  static constexpr uint32_t kABytes = 128 * 128;      // 128 rows x 64 K (K-major) or 2 x (64 K x 64 MN)
+  static constexpr uint32_t kBBytesMax = 256 * 128;   // rp <= 256
+  static constexpr uint32_t kStageBytes = kABytes + kBBytesMax;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+};
+
+template <bool kMN>
+__global__ void __launch_bounds__(128, 1)
+    k_thin(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const ThinParams p) {
+  using Cfg = ThinCfg<kMN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + S;
+  uint64_t* tmem_full = bars + 2 * S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * 128;
+  const int split = blockIdx.y;
+  const int s_begin = split * p.steps_per_split;
+  const int s_end = min(p.steps, s_begin + p.steps_per_split);
+  const int n_local = max(0, s_end - s_begin);
+  const int rp = p.rp;
+  const uint32_t tmem_cols = rp <= 64 ? 64u : (rp <= 128 ? 128u : 256u);
+  const uint32_t b_bytes = static_cast<uint32_t>(rp) * 128u;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    mbar_init(tmem_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_a);
+    tma_prefetch_desc(&tm_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  auto a_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
+  auto b_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kABytes; };
+
+  if (warp == 0 && lane == 0) {
+    int issued = 0;
+    for (int l = 0; l < n_local; ++l) {
+      const int st = l % S;
+      const uint32_t ph = (l / S) & 1;
+      if (!mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
+      const int i = s_begin + l;
+      mbar_arrive_expect_tx(&full_bar[st], Cfg::kABytes + b_bytes);
+      if (!kMN) {
+        tma_load_2d(a_tile(st), &tm_a, &full_bar[st], 64 * i, static_cast<int>(row0));
+        tma_load_2d(b_tile(st), &tm_b, &full_bar[st], 64 * i, 0);
+      } else {
+        tma_load_2d(a_tile(st), &tm_a, &full_bar[st], static_cast<int>(row0), 64 * i);
+        tma_load_2d(a_tile(st) + 8192, &tm_a, &full_bar[st], static_cast<int>(row0) + 64, 64 * i);
+        for (int c = 0; c < rp / 64; ++c) tma_load_2d(b_tile(st) + 8192 * c, &tm_b, &full_bar[st], 64 * c, 64 * i);
+      }
+      ++issued;
+    }
+    if (*abort_flag) {
+      const int first = issued > S ? issued - S : 0;
+      for (int l = first; l < issued; ++l) {
+        const uint32_t a = smem_u32(&full_bar[l % S]);
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(a, (l / S) & 1) && globaltimer_ns() - t0 < 100000000ull) {
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = make_idesc_bf16(128, static_cast<uint32_t>(rp), kMN, kMN);
+    for (int l = 0; l < n_local; ++l) {
+      const int st = l % S;
+      const uint32_t ph = (l / S) & 1;
+      if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
+      tc_fence_after();
+      const uint32_t aa = smem_u32(a_tile(st));
+      const uint32_t bb = smem_u32(b_tile(st));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint64_t da, db;
+        if (!kMN) {
+          da = make_sdesc_sw128(aa + 32u * kk, 16u, 1024u);
+          db = make_sdesc_sw128(bb + 32u * kk, 16u, 1024u);
+        } else {
+          da = make_sdesc_sw128(aa + 2048u * kk, 8192u, 1024u);
+          db = make_sdesc_sw128(bb + 2048u * kk, 8192u, 1024u);
+        }
+        umma_bf16(tmem_base, da, db, idesc, (l > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&empty_bar[st]);
+    }
+    umma_commit(tmem_full);
+  }
+  __syncwarp();
+
+  // epilogue: all four warps (warp w owns TMEM lanes 32w..32w+31)
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
+  tc_fence_after();
+  if (ok) {
+    const int64_t row = row0 + 32 * warp + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
+    for (int cb = 0; cb < rp / 32; ++cb) {
+      uint32_t v[32];
+      tmem_ld32(lane_base + 32 * cb, v);
+      tmem_ld_wait();
+      if (row < p.rows) {
+        float* dst = p.partial + (static_cast<int64_t>(split) * p.rows + row) * rp + 32 * cb;
+        if (n_local == 0) {
+#pragma unroll
+          for (int g = 0; g < 8; ++g) *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(0, 0, 0, 0);
+        } else {
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, tmem_cols);
+  }
+}
+
+// ============================================================================
+// Reductions over split-K partials (fixed order: deterministic)
+// ============================================================================
+// out_bf16[i] = BF16(scale * sum_s partial[s][i]), n4 = count / 4
+__global__ void k_reduce_bf16(const float* __restrict__ partial, int splits, int64_t count, float scale,
+                              uint16_t* __restrict__ out) {
+  const int64_t n4 = count >> 2;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float4 acc = reinterpret_cast<const float4*>(partial)[i];
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = reinterpret_cast<const float4*>(partial + s * count)[i];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(acc.x * scale, acc.y * scale);
+    o.y = pack_bf16x2(acc.z * scale, acc.w * scale);
+    reinterpret_cast<uint2*>(out)[i] = o;
+  }
+}
+
+// dB[n][j] = sum_s partial[s][n][j] for j < r   (partial rows are rp wide)
+__global__ void k_reduce_dB(const float* __restrict__ partial, int splits, int64_t d, int rp, int r,
+                            float* __restrict__ dB) {
+  const int64_t count = d * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / r;
+    const int j = static_cast<int>(i - n * r);
+    float acc = 0.0f;
+    for (int s = 0; s < splits; ++s) acc += partial[(s * d + n) * rp + j];
+    dB[i] = acc;
+  }
+}
+
+// dA[j][c] = sum_s partial[s][c][j]  (partial holds dA^T, rows = k columns)
+__global__ void k_reduce_dA(const float* __restrict__ partial, int splits, int64_t k, int rp, int r,
+                            float* __restrict__ dA) {
+  __shared__ float tile[32][33];
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int j0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
+  for (int yy = ty; yy < 32; yy += 8) {
+    const int64_t c = c0 + yy;
+    const int j = j0 + tx;
+    float acc = 0.0f;
+    if (c < k && j < rp)
+      for (int s = 0; s < splits; ++s) acc += partial[(s * k + c) * rp + j];
+    tile[yy][tx] = acc;
+  }
+  __syncthreads();
+  for (int yy = ty; yy < 32; yy += 8) {
+    const int j = j0 + yy;
+    const int64_t c = c0 + tx;
+    if (j < r && c < k) dA[static_cast<int64_t>(j) * k + c] = tile[tx][yy];
+  }
+}
+
+// Bt[j][n] = B[n][j] for j < r, 0 for r <= j < rp
+__global__ void k_transpose_B(const uint16_t* __restrict__ B, int64_t d, int r, int rp, uint16_t* __restrict__ Bt) {
+  __shared__ uint16_t tile[32][34];
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int j0 = blockIdx.y * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int yy = ty; yy < 32; yy += 8) {
+    const int64_t n = n0 + yy;
+    const int j = j0 + tx;
+    tile[yy][tx] = (n < d && j < r) ? B[n * r + j] : static_cast<uint16_t>(0);
+  }
+  __syncthreads();
+  for (int yy = ty; yy < 32; yy += 8) {
+    const int j = j0 + yy;
+    const int64_t n = n0 + tx;
+    if (j < rp && n < d) Bt[static_cast<int64_t>(j) * d + n] = tile[tx][yy];
+  }
+}
+
+// ============================================================================
+// Host side: split heuristics, workspace layout, launches
+// ============================================================================
+constexpr int kSms = 148;   // B200: split counts are planned for 148 SMs
+
+// Number of K splits so that `tiles * splits` fills the machine, each split
+// keeping at least `min_steps` K steps.
+static int plan_splits(int64_t tiles, int steps, int min_steps, int slots_per_sm) {
+  const int64_t slots = static_cast<int64_t>(kSms) * slots_per_sm;
+  if (tiles >= slots || steps <= min_steps) return 1;
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 32; ++s) {
+    const int per = static_cast<int>(ceil_div(steps, s));
+    if (per < min_steps && s > 1) break;
+    const int real = static_cast<int>(ceil_div(steps, per));
+    const int64_t ctas = tiles * real;
+    const int64_t waves = ceil_div(ctas, slots);
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * slots);
+    // prefer filling the machine; among similar fills prefer fewer splits
+    const double score = eff * (ctas >= slots ? 1.0 : static_cast<double>(ctas) / slots);
+    if (score > best_eff + 0.02) {
+      best_eff = score;
+      best = real;
+    }
+  }
+  return best;
+}
+
+struct Plan {
+  // thin GEMMs
+  int splits_T, splits_U, splits_dA, splits_dB;
+  // main
+  int main_splits;
+  int nt;   // swap token tile (0 = non-swap)
+  // workspace offsets (bytes)
+  size_t off_T, off_partT, off_Bt, off_U, off_partU, off_partA, off_partB, off_main, total;
+};
+
+static int swap_nt(int64_t M) {
+  if (M <= 16) return 16;
+  if (M <= 32) return 32;
+  if (M <= 64) return 64;
+  if (M <= 128) return 128;
+  return 0;
+}
+
+static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool need_T) {
+  Plan pl{};
+  const int rp = qlora_rank_pad(r);
+  const int64_t mt = ceil_div(M, 128);
+  pl.splits_T = plan_splits(mt, static_cast<int>(k / 64), 4, 2);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align_up(bytes, 256);
+    return o;
+  };
+  pl.off_T = need_T ? take(static_cast<size_t>(M) * rp * 2) : 0;
+  pl.off_partT = need_T ? take(static_cast<size_t>(pl.splits_T) * M * rp * 4) : 0;
+  if (!bwd) {
+    pl.nt = swap_nt(M);
+    const int steps = static_cast<int>(k / 64);
+    if (pl.nt) {
+      pl.main_splits = plan_splits(ceil_div(d, 128), steps, 8, 1);
+    } else {
+      pl.main_splits = plan_splits(ceil_div(d, 256) * mt, steps, 8, 1);
+    }
+    pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * d * 4) : 0;
+  } else {
+    pl.nt = 0;
+    const int dsteps = static_cast<int>(ceil_div(d, 64));
+    pl.splits_U = plan_splits(mt, dsteps, 4, 2);
+    pl.off_Bt = take(static_cast<size_t>(rp) * d * 2);
+    pl.off_U = take(static_cast<size_t>(M) * rp * 2);
+    pl.off_partU = take(static_cast<size_t>(pl.splits_U) * M * rp * 4);
+    const int msteps = static_cast<int>(ceil_div(M, 64));
+    pl.splits_dA = plan_splits(ceil_div(k, 128), msteps, 4, 2);
+    pl.splits_dB = plan_splits(ceil_div(d, 128), msteps, 4, 2);
+    pl.off_partA = take(static_cast<size_t>(pl.splits_dA) * k * rp * 4);
+    pl.off_partB = take(static_cast<size_t>(pl.splits_dB) * d * rp * 4);
+    pl.main_splits = plan_splits(ceil_div(k, 256) * mt, dsteps, 8, 1);
+    pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * k * 4) : 0;
+  }
+  pl.total = off;
+  return pl;
+}
+
+size_t fwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
+  // T_s always has a workspace home so the caller may pass T_save == NULL
+  return make_plan(M, d, k, r, false, true).total;
+}
+size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
+  return make_plan(M, d, k, r, true, true).total;
+}
+
+template <typename K>
+static cudaError_t set_smem(K kernel, uint32_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+static int grid1d(int64_t work, int per_block) {
+  int64_t g = ceil_div(work, per_block);
+  const int64_t cap = static_cast<int64_t>(kSms) * 16;
+  if (g > cap) g = cap;
+  return static_cast<int>(g < 1 ? 1 : g);
+}
+
+#define QL_CHECK_LAUNCH(what)                    \
+  do {                                           \
+    cudaError_t e_ = cudaGetLastError();         \
+    if (e_ != cudaSuccess) {                     \
+      *why = what;                               \
+      return QLORA_ERR_CUDA;                     \
+    }                                            \
+  } while (0)
+
+// T_s = BF16(s X A^T) (or U_s = BF16(s dY B) with `act` = dY and `bmat` = B^T)
+static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uint16_t* bmat, int64_t brows,
+                            int rp, float s, int splits, float* partial, uint16_t* out, cudaStream_t st,
+                            const char** why) {
+  CUtensorMap ta, tb;
+  if (!map_bf16(&ta, act, K, M, 64, 128) || !map_bf16(&tb, bmat, K, brows, 64, rp)) {
+    *why = "tensor map encoding failed (thin GEMM)";
+    return QLORA_ERR_CUDA;
+  }
+  ThinParams tp{};
+  tp.rows = M;
+  tp.rp = rp;
+  tp.steps = static_cast<int>(ceil_div(K, 64));
+  tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, splits));
+  tp.partial = partial;
+  const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
+  if (set_smem(k_thin<false>, ThinCfg<false>::kSmemBytes) != cudaSuccess) {
+    *why = "smem attribute";
+    return QLORA_ERR_CUDA;
+  }
+  dim3 grid(static_cast<unsigned>(ceil_div(M, 128)), static_cast<unsigned>(real));
+  k_thin<false><<<grid, 128, ThinCfg<false>::kSmemBytes, st>>>(ta, tb, tp);
+  QL_CHECK_LAUNCH("thin GEMM launch");
+  const int64_t count = M * rp;
+  k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(partial, real, count, s, out);
+  QL_CHECK_LAUNCH("reduce launch");
+  return 0;
+}
+
+template <Mode MODE, int NT>
+static int launch_main(const CUtensorMap& ta, const CUtensorMap& tc, const CUtensorMap& te, const MainParams& mp,
+                       dim3 grid, cudaStream_t st, const char** why) {
+  using Cfg = MainCfg<MODE, NT>;
+  if (set_smem(k_qlora_main<MODE, NT>, Cfg::kSmemBytes) != cudaSuccess) {
+    *why = "smem attribute (main)";
+    return QLORA_ERR_CUDA;
+  }
+  k_qlora_main<MODE, NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
+  QL_CHECK_LAUNCH("main GEMM launch");
+  return 0;
+}
+
+static ScaleSrc scale_src(const qlora_nf4_t& q) {
+  ScaleSrc s{};
+  s.dq = q.double_quant;
+  s.absmax = q.absmax;
+  s.c2 = q.c2;
+  s.c1 = q.c1;
+  s.mean = q.mean;
+  return s;
+}
+
+int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
+  const int64_t M = a.M, d = a.d, k = a.k;
+  const int rp = a.rp;
+  const bool own_T = (a.T == nullptr);
+  Plan pl = make_plan(M, d, k, a.r, false, true);
+  char* ws = static_cast<char*>(a.ws);
+  uint16_t* T = own_T ? reinterpret_cast<uint16_t*>(ws + pl.off_T) : a.T;
+  float* partT = reinterpret_cast<float*>(ws + pl.off_partT);
+  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, rp, a.s, pl.splits_T, partT, T, st, why);
+  if (rc) return rc;
+
+  const qlora_nf4_t& q = *a.q;
+  MainParams mp{};
+  mp.M = M; mp.d = d; mp.k = k; mp.r = a.r; mp.rp = rp;
+  mp.kpb = static_cast<int32_t>(k / 64);
+  mp.sc = scale_src(q);
+  mp.lora = a.B;
+  mp.n_out = d;
+  mp.steps_main = static_cast<int32_t>(k / 64);
+  mp.ext_steps = rp / 64;
+  mp.steps_per_split = static_cast<int32_t>(ceil_div(mp.steps_main, pl.main_splits));
+  mp.splits = static_cast<int32_t>(ceil_div(mp.steps_main, mp.steps_per_split));
+  mp.out = a.Y;
+  mp.partial = reinterpret_cast<float*>(ws + pl.off_main);
+  CUtensorMap t_act, t_codes, t_ext;
+  const int nt = pl.nt;
+  bool ok;
+  if (nt) {
+    ok = map_bf16(&t_act, a.X, k, M, 64, nt) &&
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 128, false) &&
+         map_bf16(&t_ext, T, rp, M, 64, nt);
+  } else {
+    ok = map_bf16(&t_act, a.X, k, M, 64, 128) &&
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 256, false) &&
+         map_bf16(&t_ext, T, rp, M, 64, 128);
+  }
+  if (!ok) {
+    *why = "tensor map encoding failed (forward)";
+    return QLORA_ERR_CUDA;
+  }
+  dim3 grid;
+  if (nt) {
+    grid = dim3(static_cast<unsigned>(ceil_div(d, 128)), 1, static_cast<unsigned>(mp.splits));
+  } else {
+    grid = dim3(static_cast<unsigned>(ceil_div(d, 256)), static_cast<unsigned>(ceil_div(M, 128)),
+                static_cast<unsigned>(mp.splits));
+  }
+  switch (nt) {
+    case 16: rc = launch_main<Mode::FwdSwap, 16>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 32: rc = launch_main<Mode::FwdSwap, 32>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 64: rc = launch_main<Mode::FwdSwap, 64>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 128: rc = launch_main<Mode::FwdSwap, 128>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    default: rc = launch_main<Mode::Fwd, 0>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+  }
+  if (rc) return rc;
+  if (mp.splits > 1) {
+    const int64_t count = M * d;
+    k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.Y);
+    QL_CHECK_LAUNCH("reduce launch (forward)");
+  }
+  return 0;
+}
+
+int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
+  const int64_t M = a.M, d = a.d, k = a.k;
+  const int rp = a.rp, r = a.r;
+  Plan pl = make_plan(M, d, k, r, true, true);
+  char* ws = static_cast<char*>(a.ws);
+  const qlora_nf4_t& q = *a.q;
+  int rc;
+  if (M == 0) {
+    cudaMemsetAsync(a.dA, 0, static_cast<size_t>(r) * k * 4, st);
+    cudaMemsetAsync(a.dB, 0, static_cast<size_t>(d) * r * 4, st);
+    return 0;
+  }
+  // T_s (recompute when not saved)
+  const uint16_t* T = a.Tin;
+  if (!T) {
+    uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + pl.off_T);
+    rc = run_lowrank_down(a.X, M, k, a.A, r, rp, a.s, pl.splits_T, reinterpret_cast<float*>(ws + pl.off_partT), Tw,
+                          st, why);
+    if (rc) return rc;
+    T = Tw;
+  }
+  // U_s = BF16(s dY B) through B^T (rp x d, K-major)
+  uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
+  k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
+      a.B, d, r, rp, Bt);
+  QL_CHECK_LAUNCH("transpose launch");
+  uint16_t* U = reinterpret_cast<uint16_t*>(ws + pl.off_U);
+  rc = run_lowrank_down(a.dY, M, d, Bt, rp, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU), U,
+                        st, why);
+  if (rc) return rc;
+
+  // dX = dY W + U_s A
+  if (a.dX) {
+    MainParams mp{};
+    mp.M = M; mp.d = d; mp.k = k; mp.r = r; mp.rp = rp;
+    mp.kpb = static_cast<int32_t>(k / 64);
+    mp.sc = scale_src(q);
+    mp.lora = a.A;
+    mp.n_out = k;
+    mp.steps_main = static_cast<int32_t>(ceil_div(d, 64));
+    mp.ext_steps = rp / 64;
+    mp.steps_per_split = static_cast<int32_t>(ceil_div(mp.steps_main, pl.main_splits));
+    mp.splits = static_cast<int32_t>(ceil_div(mp.steps_main, mp.steps_per_split));
+    mp.out = a.dX;
+    mp.partial = reinterpret_cast<float*>(ws + pl.off_main);
+    CUtensorMap t_act, t_codes, t_ext;
+    if (!map_bf16(&t_act, a.dY, d, M, 64, 128) ||
+        !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 64, false) ||
+        !map_bf16(&t_ext, U, rp, M, 64, 128)) {
+      *why = "tensor map encoding failed (backward)";
+      return QLORA_ERR_CUDA;
+    }
+    dim3 grid(static_cast<unsigned>(ceil_div(k, 256)), static_cast<unsigned>(ceil_div(M, 128)),
+              static_cast<unsigned>(mp.splits));
+    rc = launch_main<Mode::Bwd, 0>(t_act, t_codes, t_ext, mp, grid, st, why);
+    if (rc) return rc;
+    if (mp.splits > 1) {
+      const int64_t count = M * k;
+      k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.dX);
+      QL_CHECK_LAUNCH("reduce launch (dX)");
+    }
+  }
+
+  // dA^T = X^T U_s  and  dB = dY^T T_s  (reduction over tokens, MN-major operands)
+  {
+    CUtensorMap ta, tb;
+    if (!map_bf16(&ta, a.X, k, M, 64, 64) || !map_bf16(&tb, U, rp, M, 64, 64)) {
+      *why = "tensor map encoding failed (dA)";
+      return QLORA_ERR_CUDA;
+    }
+    ThinParams tp{};
+    tp.rows = k;
+    tp.rp = rp;
+    tp.steps = static_cast<int>(ceil_div(M, 64));
+    tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dA));
+    tp.partial = reinterpret_cast<float*>(ws + pl.off_partA);
+    const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
+    if (set_smem(k_thin<true>, ThinCfg<true>::kSmemBytes) != cudaSuccess) {
+      *why = "smem attribute (thin MN)";
+      return QLORA_ERR_CUDA;
+    }
+    k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
+                   ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+    QL_CHECK_LAUNCH("dA GEMM launch");
+    k_reduce_dA<<<dim3(static_cast<unsigned>(ceil_div(k, 32)), static_cast<unsigned>(ceil_div(r, 32))), 256, 0, st>>>(
+        tp.partial, real, k, rp, r, a.dA);
+    QL_CHECK_LAUNCH("dA reduce launch");
+  }
+  {
+    CUtensorMap ta, tb;
+    if (!map_bf16(&ta, a.dY, d, M, 64, 64) || !map_bf16(&tb, T, rp, M, 64, 64)) {
+      *why = "tensor map encoding failed (dB)";
+      return QLORA_ERR_CUDA;
+    }
+    ThinParams tp{};
+    tp.rows = d;
+    tp.rp = rp;
+    tp.steps = static_cast<int>(ceil_div(M, 64));
+    tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dB));
+    tp.partial = reinterpret_cast<float*>(ws + pl.off_partB);
+    const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
+    k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
+                   ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+    QL_CHECK_LAUNCH("dB GEMM launch");
+    k_reduce_dB<<<grid1d(d * r, 256), 256, 0, st>>>(tp.partial, real, d, rp, r, a.dB);
+    QL_CHECK_LAUNCH("dB reduce launch");
+  }
+  return 0;
+}
+
+}  // namespace qlora

@@ -1,0 +1,184 @@
+/*
+ * qlora.h -- C ABI of libqlora: the QLoRA linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer keeps a frozen weight W0 (d x k) as blockwise 4-bit NormalFloat
+ * (NF4) codes, optionally with double quantisation (DQ) of the per-block
+ * constants, and trains a rank-r LoRA adapter (A: r x k, B: d x r) beside it:
+ *
+ *     Y = X * deq(W0)^T + (alpha / r) * (X * A^T) * B^T
+ *
+ * Sources (page title, section):
+ *   "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora): sections
+ *     "How does it work?" (h = W0 x + (alpha/r) B (A x), A is r x k, B is d x r),
+ *     "First, how does k-bit quantization work?" (Int8 absmax),
+ *     "NF4: Choose the codebook to fit the distribution" (the 16-value table),
+ *     "Quantizing and dequantizing with the codebook" (blockwise NF4, blocks of 64),
+ *     "Double quantization and double dequantization" (8-bit block constants in
+ *       groups of 256 with an FP32 second-level scale and a stored mean; the
+ *       QLoRA expression; backpropagation through the reconstructed base).
+ *   "LoRA and QLoRA: Efficient Fine-Tuning of Large Language Models"
+ *     (fromzero2ai.dev): section "Low-Rank Matrix Factorization".
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers into caller-owned memory.  The
+ *     library never allocates device memory; scratch space is passed in as
+ *     `workspace`.  Host-side structs (qlora_nf4_t) are read during the call only.
+ *   - bf16 tensors are passed as uint16_t bit patterns, row-major, densely
+ *     packed, 16-byte aligned.  fp32 outputs are row-major, 16-byte aligned.
+ *   - Every compute call is asynchronous: it validates its arguments on the
+ *     host, enqueues kernels on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and returns.  Results are ready when the stream reaches them.
+ *   - Return value: QLORA_OK (0) or a negative qlora_status.  Nothing is
+ *     enqueued when a call returns an error.  qlora_last_error() gives a
+ *     human-readable reason (thread-local, valid until the next call on the
+ *     same thread).
+ *   - Kernels never trap.  A kernel that detects a failed internal check (a
+ *     bounded wait that ran out) records it in a per-device status word that
+ *     qlora_device_status() reads and clears.
+ *   - No NaN/Inf handling is promised: W0 and the activations must be finite;
+ *     non-finite inputs give unspecified (but memory-safe) results.
+ */
+#ifndef QLORA_H
+#define QLORA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = -1,  /* null pointer, negative size, mismatched struct  */
+  QLORA_ERR_UNSUPPORTED = -2,  /* valid but not implemented (blocksize != 64, ...) */
+  QLORA_ERR_ALIGNMENT = -3,    /* a pointer is not 16-byte aligned               */
+  QLORA_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required      */
+  QLORA_ERR_CUDA = -5,         /* a CUDA runtime/driver call failed               */
+  QLORA_ERR_DEVICE = -6        /* a kernel reported a failed check (see status)   */
+} qlora_status;
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA headers. */
+typedef void *qlora_stream_t;
+
+/* Quantized weight.  Element i of W0 (flat row-major index, N = d*k) lies in
+ * block j = i / 64 and DQ group g = j / 256.
+ *   codes : ceil(N/2) bytes; byte t = code[2t] | code[2t+1] << 4 (low nibble
+ *           first); an odd N pads the last high nibble with 0.
+ *   absmax: M_b = ceil(N/64) fp32 block scales (the block's max |w|); used and
+ *           written only when double_quant == 0 (may be NULL otherwise).
+ *   c2    : M_b int8 quantized deviations (s_j - mean) * c1[g], round half to
+ *           even; DQ only.
+ *   c1    : G = ceil(M_b/256) fp32 second-level scales, c1 = 127 / max|s - mean|
+ *           over the group (1.0 for an all-zero group); DQ only.
+ *   mean  : 1 fp32, the mean of all M_b block scales; DQ only.
+ * All pointers are device pointers; codes and c2 need no alignment beyond 4
+ * bytes, the fp32 arrays 4 bytes. */
+typedef struct {
+  int64_t d;
+  int64_t k;
+  int32_t blocksize;     /* weights per NF4 block; only 64 is supported       */
+  int32_t double_quant;  /* 0: fp32 absmax per block; 1: int8 c2 + fp32 c1    */
+  uint8_t *codes;
+  float *absmax;
+  int8_t *c2;
+  float *c1;
+  float *mean;
+} qlora_nf4_t;
+
+/* Index of each buffer in qlora_nf4_sizes()'s `sizes` array. */
+enum { QLORA_BUF_CODES = 0, QLORA_BUF_ABSMAX = 1, QLORA_BUF_C2 = 2, QLORA_BUF_C1 = 3, QLORA_BUF_MEAN = 4 };
+
+/* Byte sizes of the five quantized-weight buffers for a d x k weight, and the
+ * workspace nf4_quantize needs.  Buffers not used by the chosen mode get size
+ * 0.  With blocksize 64 and DQ on, sizes[1..4] add up to the page's
+ * 8/64 + 32/(256*64) bits per weight ("Double quantization and double
+ * dequantization", the 0.373-bit accounting) plus the 4-byte mean.
+ * Host-only; touches no GPU. */
+int qlora_nf4_sizes(int64_t d, int64_t k, int32_t blocksize, int32_t double_quant,
+                    size_t sizes[5], size_t *quant_workspace_bytes);
+
+/* Blockwise NF4 quantisation of W0 ("Quantizing and dequantizing with the
+ * codebook") followed, when q->double_quant, by double quantisation of the
+ * block scales ("Double quantization and double dequantization").
+ *   W0        : d*k bf16 (device, 16-byte aligned).
+ *   q         : host struct describing the output buffers (device pointers,
+ *               sizes from qlora_nf4_sizes).
+ *   workspace : device scratch of at least quant_workspace_bytes (16-byte
+ *               aligned); unused and may be NULL when DQ is off.
+ * Per block: s = max |w|; code = the index of the nearest NF4 value to
+ * RN32(w / s) measured by fp32 distance, the smaller index on ties; an
+ * all-zero block gets the exact-zero code 7.  DQ: mean = RN32(RN64(exact sum
+ * of s_j) / M_b); per group of 256, c1 = RN32(127 / max|RN32(s_j - mean)|),
+ * c2_j = round_half_even(RN32(c1 * RN32(s_j - mean))).  Deterministic and
+ * bit-reproducible. */
+int nf4_quantize(const uint16_t *W0, const qlora_nf4_t *q, void *workspace, size_t workspace_bytes,
+                 qlora_stream_t stream);
+
+/* doubleDequant ("Double quantization and double dequantization"): writes the
+ * reconstructed weights W_out[i] = BF16(RN32(C[code_i] * s^_j)) with
+ * s^_j = RN32(RN32(c2_j / c1_g) + mean) (DQ on) or s^_j = absmax_j (DQ off).
+ *   W_out : d*k bf16 (device, 16-byte aligned). */
+int nf4_dequantize(const qlora_nf4_t *q, uint16_t *W_out, qlora_stream_t stream);
+
+/* Columns of the saved adapter activation T_save (and of the internal U):
+ * r rounded up to a multiple of 64. */
+int32_t qlora_rank_pad(int32_t r);
+
+/* Workspace bytes needed by qlora_linear_fwd (backward == 0) or
+ * qlora_linear_bwd (backward == 1) for M tokens and a d x k weight of rank r.
+ * Host-only. */
+int qlora_linear_workspace_size(int64_t M, int64_t d, int64_t k, int32_t r, int32_t backward,
+                                size_t *bytes);
+
+/* Forward of the QLoRA linear layer (the QLoRA expression in "Double
+ * quantization and double dequantization"; scaling alpha/r from "How does
+ * alpha/r control adapter strength?"):
+ *     Y = X * W^T + s * (X * A^T) * B^T,  s = RN32(alpha / r),
+ * where W = doubleDequant(q) in bf16 is formed tile by tile in on-chip memory
+ * and never written to device memory.
+ *   X      : M x k bf16.        A : r x k bf16.       B : d x r bf16.
+ *   Y      : M x d bf16 (written, not accumulated).
+ *   T_save : M x qlora_rank_pad(r) bf16, receives BF16(s * X * A^T) with zero
+ *            padding columns, for reuse by qlora_linear_bwd; may be NULL.
+ *   workspace : qlora_linear_workspace_size(M, d, k, r, 0) bytes, 16-byte
+ *            aligned (may be NULL only when that size is 0).
+ * Requirements: k % 64 == 0, d % 8 == 0, 1 <= r <= 256, M >= 0 (M == 0 is a
+ * no-op).  Accumulation is fp32 on the tensor cores. */
+int qlora_linear_fwd(const uint16_t *X, int64_t M, const qlora_nf4_t *q, const uint16_t *A,
+                     const uint16_t *B, int32_t r, float alpha, uint16_t *Y, uint16_t *T_save,
+                     void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Backward of the QLoRA linear layer.  The base weight is frozen ("we
+ * backpropagate through the reconstructed base transformations to train those
+ * adapters; the stored 4-bit weights are not updated"), so there is no dW0:
+ *     U  = s * dY * B                    (M x r)
+ *     dX = dY * W + U * A                (M x k, bf16)
+ *     dA = U^T * X  = s * (dY B)^T X     (r x k, fp32)
+ *     dB = s * dY^T * (X A^T)            (d x r, fp32)
+ *   T_save : the buffer filled by qlora_linear_fwd with the same X, A, r,
+ *            alpha; NULL recomputes it into the workspace.
+ *   dX, dA, dB are written, not accumulated.  dX may be NULL to skip it.
+ *   workspace : qlora_linear_workspace_size(M, d, k, r, 1) bytes. */
+int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t M, const qlora_nf4_t *q,
+                     const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                     const uint16_t *T_save, uint16_t *dX, float *dA, float *dB,
+                     void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* The library's NF4 table C[0..15] (fp32, ascending) copied to host memory. */
+int qlora_nf4_codebook(float out[16]);
+
+/* Synchronizes `stream`, then reads and clears the current device's status
+ * word: *status = 0 when no kernel reported a failed check since the last
+ * read, otherwise the code of the first failure.  Returns QLORA_ERR_DEVICE
+ * when *status != 0. */
+int qlora_device_status(qlora_stream_t stream, int32_t *status);
+
+/* Reason for the last error returned on this thread ("" if none). */
+const char *qlora_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H */

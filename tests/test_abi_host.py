@@ -1,0 +1,112 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and its host-only functions (sizes, validation, codebook)
+behave as documented."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_quantized_lora_02_b200 as Q
+from oracle import qlora_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_quantized_lora_02_b200 import build
+    build.build()
+    return Q.lib()
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = header_functions()
+    assert len(declared) >= 10
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(declared) == sorted(Q.EXPORTS)
+
+
+def test_codebook_matches_oracle_bitwise(L):
+    lib_table = np.array(Q.qlora_nf4_codebook(), np.float32)
+    assert np.array_equal(lib_table.view(np.uint32), O.nf4_codebook().view(np.uint32))
+
+
+def test_sizes_closed_form(golden):
+    g = golden("storage_accounting.json")
+    sizes, ws = Q.qlora_nf4_sizes(4096, 4096, 64, True)
+    assert sizes == [8388608, 0, 262144, 4096, 4]
+    assert sum(sizes) == 8654852
+    n = 4096 * 4096
+    bits_consts = (sizes[2] + sizes[3]) * 8 / n
+    assert bits_consts == g["bits_per_weight_after"]
+    sizes0, ws0 = Q.qlora_nf4_sizes(4096, 4096, 64, False)
+    assert sizes0 == [8388608, 4 * 262144, 0, 0, 0] and ws0 == 0
+    assert sizes0[1] * 8 / n == g["bits_per_weight_before"]
+    assert ws > 0
+
+
+def test_sizes_ragged():
+    sizes, _ = Q.qlora_nf4_sizes(3, 37, 64, True)   # N = 111 -> 2 blocks, 1 group
+    assert sizes == [56, 0, 2, 4, 4]
+    sizes, _ = Q.qlora_nf4_sizes(0, 5, 64, True)
+    assert sizes[0] == 0 and sizes[2] == 0
+
+
+def test_unsupported_blocksize_and_bad_args(L):
+    with pytest.raises(Q.QLoRAError) as e:
+        Q.qlora_nf4_sizes(64, 64, 32, True)
+    assert e.value.code == -2 and "blocksize" in str(e.value)
+    with pytest.raises(Q.QLoRAError) as e:
+        Q.qlora_nf4_sizes(-1, 64, 64, True)
+    assert e.value.code == -1
+
+
+def test_quantize_rejects_null_and_misaligned_without_gpu(L):
+    st = Q.QloraNF4(64, 64, 64, 1, None, None, None, None, None)
+    rc = L.nf4_quantize(None, ctypes.byref(st), None, 0, None)
+    assert rc == -1 and b"codes" in L.qlora_last_error()
+    st = Q.QloraNF4(64, 64, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+    rc = L.nf4_quantize(0x1001, ctypes.byref(st), 0x5000, 1 << 20, None)
+    assert rc == -3 and b"W0" in L.qlora_last_error()
+    rc = L.nf4_quantize(0x1000, ctypes.byref(st), 0x5000, 4, None)
+    assert rc == -4 and b"workspace" in L.qlora_last_error()
+    st = Q.QloraNF4(64, 64, 64, 1, 0x1000, None, 0x2001, 0x3000, 0x4000)
+    assert L.nf4_quantize(0x1000, ctypes.byref(st), 0x5000, 1 << 20, None) == -3
+
+
+def test_linear_shape_validation(L):
+    n = ctypes.c_size_t()
+    assert L.qlora_linear_workspace_size(16, 512, 512, 8, 0, ctypes.byref(n)) == 0 and n.value > 0
+    assert L.qlora_linear_workspace_size(16, 512, 500, 8, 0, ctypes.byref(n)) == -2      # k % 64
+    assert L.qlora_linear_workspace_size(16, 510, 512, 8, 0, ctypes.byref(n)) == -2      # d % 8
+    assert L.qlora_linear_workspace_size(16, 512, 512, 0, 0, ctypes.byref(n)) == -2      # r
+    assert L.qlora_linear_workspace_size(16, 512, 512, 257, 0, ctypes.byref(n)) == -2
+    assert L.qlora_linear_workspace_size(-1, 512, 512, 8, 0, ctypes.byref(n)) == -1
+    assert L.qlora_rank_pad(8) == 64 and L.qlora_rank_pad(64) == 64 and L.qlora_rank_pad(65) == 128
+
+
+def test_linear_rejects_null_inputs_without_gpu(L):
+    st = Q.QloraNF4(512, 512, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+    rc = L.qlora_linear_fwd(None, 16, ctypes.byref(st), 0x10000, 0x20000, 8, 16.0, 0x30000, None, 0x40000,
+                            1 << 30, None)
+    assert rc == -1 and b"X" in L.qlora_last_error()
+    rc = L.qlora_linear_fwd(0x10000, 16, ctypes.byref(st), 0x10000, 0x20000, 8, 16.0, 0x30000, None, None, 0, None)
+    assert rc == -4
+    # M == 0 is a no-op that succeeds without touching memory
+    assert L.qlora_linear_fwd(None, 0, ctypes.byref(st), None, None, 8, 16.0, None, None, None, 0, None) == 0
+
+
+def test_param_count_matches_buffer_shapes(golden):
+    g = golden("lora_param_count.json")
+    # A is r x k and B is d x r: the entries the backward writes
+    assert g["r"] * g["k"] + g["d"] * g["r"] == g["trainable"]
