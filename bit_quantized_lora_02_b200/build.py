@@ -47,6 +47,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     os.makedirs(BUILD, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra += os.environ.get("QLORA_NVCC_EXTRA", "").split()
     procs = []
     objs = []
     for src in SOURCES:

@@ -32,7 +32,6 @@
 
 namespace qlora {
 
-__constant__ uint32_t c_nf4_bits[16] = {QLORA_NF4_TABLE_BITS};
 static const uint32_t h_nf4_bits[16] = {QLORA_NF4_TABLE_BITS};
 
 void host_codebook(float out[16]) { std::memcpy(out, h_nf4_bits, sizeof(h_nf4_bits)); }
@@ -363,7 +362,11 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
                                                      const float* __restrict__ c1, const float* __restrict__ mean,
                                                      uint16_t* __restrict__ out) {
   __shared__ float s_C[16];
-  if (threadIdx.x < 16) s_C[threadIdx.x] = __uint_as_float(c_nf4_bits[threadIdx.x]);
+  constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) s_C[j] = __uint_as_float(kCB[j]);
+  }
   __syncthreads();
   const float mu = kDQ ? *mean : 0.0f;
   const int64_t ngroups = (N + 7) >> 3;

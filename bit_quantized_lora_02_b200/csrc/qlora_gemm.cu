@@ -45,7 +45,7 @@
 
 namespace qlora {
 
-__constant__ uint32_t c_nf4_gemm[16] = {QLORA_NF4_TABLE_BITS};
+
 
 // ============================================================================
 // Tensor maps
@@ -358,9 +358,11 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ dequant warps
     const int t = threadIdx.x - 128;   // 0..255
+    // the codebook as register immediates (no memory traffic)
+    constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
     float C[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(c_nf4_gemm[j]);
+    for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
     const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
     // this thread's W row and block column inside the tile
@@ -1128,5 +1130,6 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   }
   return 0;
 }
+
 
 }  // namespace qlora
