@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Benchmark of the QLoRA linear layer on B200.
+
+One step = the whole hot path over one batch of synthetic input, for every
+projection of the workload: blockwise NF4 quantisation with double
+quantisation of W0, the fused forward (Y = X W^T + s X A^T B^T, W rebuilt in
+shared memory) and the backward (dX, dA, dB).  With several ranks each rank
+runs the layer set on its own token batch (data parallel, weak scaling) and the
+adapter gradients dA, dB are summed over ranks with NCCL, as a data-parallel
+training step would.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints one JSON line on rank 0.  `value` is the fwd+bwd TFLOP/s of the whole
+job (algorithmic flops 4Mdk + 6Mr(d+k) per projection, summed over ranks,
+divided by the device time of K steps, max over ranks).  `--impl reference`
+times the CPU oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from bit_quantized_lora_02_b200 import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# workload arithmetic
+# ---------------------------------------------------------------------------
+def flops_fwd(M, d, k, r):
+    return 2 * M * d * k + 2 * M * r * (d + k)
+
+
+def flops_bwd(M, d, k, r):
+    return 2 * M * d * k + 4 * M * r * (d + k)
+
+
+def main_fwd_flops(M, d, k, r):      # the fused forward GEMM: X W^T + T_s B^T
+    return 2 * M * d * k + 2 * M * d * r
+
+
+def main_bwd_flops(M, d, k, r):      # the fused backward GEMM: dY W + U_s A
+    return 2 * M * d * k + 2 * M * k * r
+
+
+def nf4_bytes(d, k):
+    n = d * k
+    nb = -(-n // 64)
+    return (n + 1) // 2 + nb + 4 * (-(-nb // 256)) + 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for name in ("qlora_gemm.cu", "qlora_device.cuh", "nf4_quant.cu"):
+        with open(os.path.join(ROOT, "bit_quantized_lora_02_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel_class):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since those counters were taken."""
+    p = os.path.join(ROOT, "profiles", f"traffic_{kernel_class}.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                key, v = line.split("=", 1)
+                vals[key.strip()] = v.strip()
+    if vals.get("source_hash") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for rec in csv.reader(io.StringIO(out)):
+            if len(rec) < 10:
+                continue
+            rec = [x.strip() for x in rec]
+            try:
+                ts = time.mktime(time.strptime(rec[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + rec[0].split(".")[1]) if "." in rec[0] else 0.0
+                rows.append((ts + frac, float(rec[2]), float(rec[3]), rec[6:10]))
+            except (ValueError, IndexError):
+                continue
+        inside = [r for r in rows if self.t0 is not None and self.t0 - 0.06 <= r[0] <= self.t1 + 0.06]
+        use = inside or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median([r[1] for r in use]) if use else None,
+                "sm_max_mhz": max(r[2] for r in use) if use else None,
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """The CPU oracle on `frac` of one step: per projection it quantises frac
+    of W0's rows (NF4 + double quantisation + dequantisation) and runs the fp64
+    forward+backward on frac of the tokens against the full W-hat (built once,
+    outside the timed region)."""
+
+    def __init__(self, work, frac=0.125):
+        from oracle import qlora_oracle as O
+        self.O = O
+        self.M, self.r, self.alpha = work["m"], work["r"], work["alpha"]
+        self.frac = frac
+        self.Ms = max(1, int(self.M * frac))
+        self.prepared = []
+        for pi, (name, d, k) in enumerate(work["proj"]):
+            W0 = synth.weight(d, k, seed=pi)
+            What = O.dequantize_tensor(O.quantize_tensor(W0.reshape(-1), True)).reshape(d, k)
+            self.prepared.append((d, k, W0, What, synth.activations(self.Ms, k, pi), synth.grad_output(self.Ms, d, pi),
+                                  synth.lora_a(self.r, k, pi), synth.lora_b(d, self.r, pi)))
+        self.desc = (f"{frac:g} of one step: per projection NF4+DQ quantise/dequantise of {frac:g} of W0's rows and "
+                     f"fp64 fwd+bwd of {self.Ms} of {self.M} tokens (numpy)")
+
+    def run(self):
+        """Returns (seconds, credited fwd+bwd flops)."""
+        O, r, alpha = self.O, self.r, self.alpha
+        t0 = time.perf_counter()
+        flops = 0.0
+        for d, k, W0, What, X, dY, A, B in self.prepared:
+            rows = max(1, int(d * self.frac))
+            O.dequantize_tensor(O.quantize_tensor(W0[:rows].reshape(-1), True))
+            O.qlora_forward(X, What, A, B, alpha, r)
+            O.qlora_backward(dY, X, What, A, B, alpha, r)
+            flops += flops_fwd(self.Ms, d, k, r) + flops_bwd(self.Ms, d, k, r)
+        return time.perf_counter() - t0, flops
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, work, wl_name):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_lora_02_b200 as Q
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    M, r, alpha = work["m"], work["r"], work["alpha"]
+    projs = work["proj"]
+    bufs = []
+    h2d_bytes = d2h_bytes = 0
+    for pi, (name, d, k) in enumerate(projs):
+        tok_seed = pi + 1000 * rank         # each rank has its own token batch
+        host = {"W0": synth.weight(d, k, seed=pi), "A": synth.lora_a(r, k, seed=pi), "B": synth.lora_b(d, r, seed=pi),
+                "X": synth.activations(M, k, seed=tok_seed), "dY": synth.grad_output(M, d, seed=tok_seed)}
+        b = {"d": d, "k": k, "name": name}
+        for key, arr in host.items():
+            pinned = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).pin_memory()
+            b["h_" + key] = pinned
+            b[key] = pinned.to(dev, non_blocking=True)
+            h2d_bytes += pinned.numel() * 2
+        b["q"] = Q.nf4_alloc(d, k, True, dev)
+        b["qws"] = torch.empty(max(Q.qlora_nf4_sizes(d, k, 64, True)[1], 16), dtype=torch.uint8, device=dev)
+        b["Y"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+        b["T"] = torch.empty(M, Q.qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
+        b["dX"] = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
+        b["dA"] = torch.empty(r, k, dtype=torch.float32, device=dev)
+        b["dB"] = torch.empty(d, r, dtype=torch.float32, device=dev)
+        nws = max(Q.qlora_linear_workspace_size(M, d, k, r, False), Q.qlora_linear_workspace_size(M, d, k, r, True))
+        b["ws"] = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        for key in ("Y", "dX", "dA", "dB"):
+            b["h_" + key] = torch.empty(b[key].shape, dtype=b[key].dtype, pin_memory=True)
+            d2h_bytes += b[key].numel() * b[key].element_size()
+        bufs.append(b)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for b in bufs:
+            Q.nf4_quantize(b["W0"], True, out=b["q"], workspace=b["qws"], stream=stream)
+            Q.qlora_linear_fwd(b["X"], b["q"], b["A"], b["B"], alpha, Y=b["Y"], T_save=b["T"], workspace=b["ws"],
+                               stream=stream)
+            Q.qlora_linear_bwd(b["dY"], b["X"], b["q"], b["A"], b["B"], alpha, T_save=b["T"], dX=b["dX"],
+                               dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream)
+        if world > 1:
+            for b in bufs:
+                dist.all_reduce(b["dA"])
+                dist.all_reduce(b["dB"])
+
+    def h2d():
+        for b in bufs:
+            for key in ("W0", "A", "B", "X", "dY"):
+                b[key].copy_(b["h_" + key], non_blocking=True)
+
+    def d2h():
+        for b in bufs:
+            for key in ("Y", "dX", "dA", "dB"):
+                b["h_" + key].copy_(b[key], non_blocking=True)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # correctness guard before timing: the device status word must be clean
+    step()
+    torch.cuda.synchronize()
+    assert Q.qlora_device_status() == 0
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    Q.qlora_profile_read()                  # reset launch counters
+    Q.qlora_profile_enable(True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark("t0")
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    barrier()
+    clk = clocks.stop()
+    Q.qlora_profile_enable(False)
+    kms, klaunch = Q.qlora_profile_read()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms_total / args.steps
+    assert Q.qlora_device_status() == 0
+
+    step_flops = sum(flops_fwd(M, d, k, r) + flops_bwd(M, d, k, r) for _, d, k in projs)
+    value = world * step_flops / (ms_step * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers
+    e2e_steps = max(1, min(args.steps, 5))
+    step_e2e = lambda: (h2d(), step(), d2h())  # noqa: E731
+    step_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        step_e2e()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (device time over the timed region)
+    peaks, peaks_src = load_peaks()
+    algo = {
+        "fwd_gemm": sum(main_fwd_flops(M, d, k, r) for _, d, k in projs) * args.steps,
+        "bwd_gemm": sum(main_bwd_flops(M, d, k, r) for _, d, k in projs) * args.steps,
+    }
+    dom = max(kms, key=lambda c: kms[c])
+    roofline = None
+    if dom in algo and kms[dom] > 0:
+        achieved = algo[dom] / (kms[dom] * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        launches = max(klaunch[dom], 1)
+        traffic = read_traffic(dom)
+        roofline = {"kernel": dom, "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                    "peak_source": f"{peaks_src} bf16 dense, sustained",
+                    "frac_of_burst": round(achieved / peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]), 4),
+                    "traffic": traffic, "launches": klaunch[dom],
+                    "avg_launch_ms": round(kms[dom] / launches, 4)}
+
+    result = {
+        "metric": "QLoRA linear fwd+bwd TFLOP/s (NF4 double-quant base, LoRA adapters), step = quantize+fwd+bwd",
+        "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded numpy: W0~N(0,0.02), A~N(0,1/r), B~N(0,0.01), X,dY~N(0,1))",
+        "config": {"workload": wl_name, "tokens_per_rank": M, "rank": r, "alpha": alpha,
+                   "projections": [f"{n}:{d}x{k}" for n, d, k in projs], "nf4_blocksize": 64,
+                   "double_quant": True, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": "working set per step larger than L2 (no explicit flush)"},
+        "breakdown_ms_per_step": {c: round(v / args.steps, 4) for c, v in kms.items()},
+        "gpu_launches": int(sum(klaunch.values())),
+        "roofline": roofline,
+        "clocks": clk,
+        "e2e": {"value": round(e2e_value, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+                "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sample = OracleSample(work)
+        dt, fl = sample.run()
+        result["cpu_baseline"] = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_cores(),
+                                  "kind": "oracle", "sample": sample.desc, "seconds": round(dt, 3)}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def run_reference(args, work, wl_name):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sample = OracleSample(work)
+    desc = sample.desc
+    times, fl = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, fl = sample.run()
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    value = fl / (ms * 1e-3) / 1e12
+    result = {
+        "impl": "reference",
+        "metric": "QLoRA linear fwd+bwd TFLOP/s (NF4 double-quant base, LoRA adapters), step = quantize+fwd+bwd",
+        "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy)",
+        "config": {"workload": wl_name, "tokens_per_rank": work["m"], "rank": work["r"], "alpha": work["alpha"],
+                   "projections": [f"{n}:{d}x{k}" for n, d, k in work["proj"]], "sample": desc},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(result), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="llama7b_proj_set_m4096",
+                    choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "tiny_512"))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    work = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, work, args.workload)
+    else:
+        run_ours(args, work, args.workload)
+
+
+if __name__ == "__main__":
+    main()

@@ -26,7 +26,10 @@ _STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTE
            -4: "QLORA_ERR_WORKSPACE", -5: "QLORA_ERR_CUDA", -6: "QLORA_ERR_DEVICE"}
 
 EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_rank_pad", "qlora_linear_workspace_size",
-           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error")
+           "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error",
+           "qlora_profile_enable", "qlora_profile_read")
+
+KERNEL_CLASSES = ("quant", "dq_const", "dequant", "fwd_gemm", "bwd_gemm", "lora_gemm", "aux")
 
 
 class QLoRAError(RuntimeError):
@@ -67,8 +70,11 @@ def lib() -> ctypes.CDLL:
     L.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
     L.qlora_device_status.argtypes = [vp, ctypes.POINTER(c_i32)]
     L.qlora_last_error.restype = ctypes.c_char_p
+    L.qlora_profile_enable.argtypes = [c_i32]
+    L.qlora_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
     for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_linear_workspace_size",
-                 "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status"):
+                 "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
+                 "qlora_profile_enable", "qlora_profile_read"):
         getattr(L, name).restype = c_i32
     _lib = L
     return L
@@ -229,3 +235,15 @@ def qlora_device_status(stream=None) -> int:
     if rc not in (QLORA_OK, -6):
         _check(rc)
     return s.value
+
+
+def qlora_profile_enable(on: bool = True) -> None:
+    _check(lib().qlora_profile_enable(int(on)))
+
+
+def qlora_profile_read():
+    """Returns ({class: device ms}, {class: launches}) since the last read."""
+    ms = (ctypes.c_double * len(KERNEL_CLASSES))()
+    n = (ctypes.c_int64 * len(KERNEL_CLASSES))()
+    _check(lib().qlora_profile_read(ms, n))
+    return dict(zip(KERNEL_CLASSES, list(ms))), dict(zip(KERNEL_CLASSES, list(n)))

@@ -423,25 +423,46 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
   const int grid = grid_for(ng8);
   const int64_t nblk = (N + 63) / 64;
   if (!q.double_quant) {
-    k_nf4_quant<false><<<grid, 256, 0, st>>>(W, N, q.codes, q.absmax, nullptr, nullptr, quant_lut());
+    {
+      ProfScope ps_(QLORA_KC_QUANT, st);
+      k_nf4_quant<false><<<grid, 256, 0, st>>>(W, N, q.codes, q.absmax, nullptr, nullptr, quant_lut());
+    }
     return cudaGetLastError();
   }
   auto* hist = static_cast<unsigned long long*>(ws);
   auto* amax16 = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256 * sizeof(unsigned long long));
-  k_zero_u64<<<1, 256, 0, st>>>(hist, 256);
-  k_nf4_quant<true><<<grid, 256, 0, st>>>(W, N, q.codes, nullptr, amax16, hist, quant_lut());
-  k_dq_mean<<<1, 32, 0, st>>>(hist, nblk, q.mean);
+  {
+    ProfScope ps_(QLORA_KC_DQ_CONST, st);
+    k_zero_u64<<<1, 256, 0, st>>>(hist, 256);
+  }
+  {
+    ProfScope ps_(QLORA_KC_QUANT, st);
+    k_nf4_quant<true><<<grid, 256, 0, st>>>(W, N, q.codes, nullptr, amax16, hist, quant_lut());
+  }
+  {
+    ProfScope ps_(QLORA_KC_DQ_CONST, st);
+    k_dq_mean<<<1, 32, 0, st>>>(hist, nblk, q.mean);
+  }
   const int64_t ngroups = (nblk + 255) / 256;
-  k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, q.mean, q.c2, q.c1);
+  {
+    ProfScope ps_(QLORA_KC_DQ_CONST, st);
+    k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, q.mean, q.c2, q.c1);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st) {
   const int grid = grid_for((N + 7) / 8);
   if (q.double_quant)
-    k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
+    {
+      ProfScope ps_(QLORA_KC_DEQUANT, st);
+      k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
+    }
   else
-    k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
+    {
+      ProfScope ps_(QLORA_KC_DEQUANT, st);
+      k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
+    }
   return cudaGetLastError();
 }
 

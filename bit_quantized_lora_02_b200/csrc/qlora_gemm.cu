@@ -927,10 +927,16 @@ static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uin
     return QLORA_ERR_CUDA;
   }
   dim3 grid(static_cast<unsigned>(ceil_div(M, 128)), static_cast<unsigned>(real));
-  k_thin<false><<<grid, 128, ThinCfg<false>::kSmemBytes, st>>>(ta, tb, tp);
+  {
+    ProfScope ps_(QLORA_KC_LORA_GEMM, st);
+    k_thin<false><<<grid, 128, ThinCfg<false>::kSmemBytes, st>>>(ta, tb, tp);
+  }
   QL_CHECK_LAUNCH("thin GEMM launch");
   const int64_t count = M * rp;
-  k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(partial, real, count, s, out);
+  {
+    ProfScope ps_(QLORA_KC_AUX, st);
+    k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(partial, real, count, s, out);
+  }
   QL_CHECK_LAUNCH("reduce launch");
   return 0;
 }
@@ -943,7 +949,10 @@ static int launch_main(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
     *why = "smem attribute (main)";
     return QLORA_ERR_CUDA;
   }
-  k_qlora_main<MODE, NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
+  {
+    ProfScope ps_((MODE == Mode::Bwd ? QLORA_KC_BWD_GEMM : QLORA_KC_FWD_GEMM), st);
+    k_qlora_main<MODE, NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
+  }
   QL_CHECK_LAUNCH("main GEMM launch");
   return 0;
 }
@@ -1015,7 +1024,10 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   if (rc) return rc;
   if (mp.splits > 1) {
     const int64_t count = M * d;
-    k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.Y);
+    {
+      ProfScope ps_(QLORA_KC_AUX, st);
+      k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.Y);
+    }
     QL_CHECK_LAUNCH("reduce launch (forward)");
   }
   return 0;
@@ -1044,8 +1056,11 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   }
   // U_s = BF16(s dY B) through B^T (rp x d, K-major)
   uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
-  k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
+  {
+    ProfScope ps_(QLORA_KC_AUX, st);
+    k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
       a.B, d, r, rp, Bt);
+  }
   QL_CHECK_LAUNCH("transpose launch");
   uint16_t* U = reinterpret_cast<uint16_t*>(ws + pl.off_U);
   rc = run_lowrank_down(a.dY, M, d, Bt, rp, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU), U,
@@ -1079,7 +1094,10 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     if (rc) return rc;
     if (mp.splits > 1) {
       const int64_t count = M * k;
-      k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.dX);
+      {
+        ProfScope ps_(QLORA_KC_AUX, st);
+        k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.dX);
+      }
       QL_CHECK_LAUNCH("reduce launch (dX)");
     }
   }
@@ -1102,11 +1120,17 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
       *why = "smem attribute (thin MN)";
       return QLORA_ERR_CUDA;
     }
-    k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
+    {
+      ProfScope ps_(QLORA_KC_LORA_GEMM, st);
+      k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
                    ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+    }
     QL_CHECK_LAUNCH("dA GEMM launch");
-    k_reduce_dA<<<dim3(static_cast<unsigned>(ceil_div(k, 32)), static_cast<unsigned>(ceil_div(r, 32))), 256, 0, st>>>(
+    {
+      ProfScope ps_(QLORA_KC_AUX, st);
+      k_reduce_dA<<<dim3(static_cast<unsigned>(ceil_div(k, 32)), static_cast<unsigned>(ceil_div(r, 32))), 256, 0, st>>>(
         tp.partial, real, k, rp, r, a.dA);
+    }
     QL_CHECK_LAUNCH("dA reduce launch");
   }
   {
@@ -1122,10 +1146,16 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dB));
     tp.partial = reinterpret_cast<float*>(ws + pl.off_partB);
     const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-    k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
+    {
+      ProfScope ps_(QLORA_KC_LORA_GEMM, st);
+      k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
                    ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+    }
     QL_CHECK_LAUNCH("dB GEMM launch");
-    k_reduce_dB<<<grid1d(d * r, 256), 256, 0, st>>>(tp.partial, real, d, rp, r, a.dB);
+    {
+      ProfScope ps_(QLORA_KC_AUX, st);
+      k_reduce_dB<<<grid1d(d * r, 256), 256, 0, st>>>(tp.partial, real, d, rp, r, a.dB);
+    }
     QL_CHECK_LAUNCH("dB reduce launch");
   }
   return 0;

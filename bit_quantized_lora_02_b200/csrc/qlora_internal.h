@@ -51,6 +51,17 @@ size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r);
 int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why);
 int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why);
 
+// tracing (qlora_prof.cu): construct around each kernel launch
+struct ProfScope {
+  int kc;
+  cudaStream_t st;
+  void* a;
+  ProfScope(int kc, cudaStream_t st);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+};
+
 // status word (qlora_abi.cu)
 cudaError_t read_and_clear_status(int* out);
 

@@ -174,6 +174,29 @@ int qlora_nf4_codebook(float out[16]);
  * when *status != 0. */
 int qlora_device_status(qlora_stream_t stream, int32_t *status);
 
+/* Tracing: every kernel launch of the library belongs to one class. */
+enum {
+  QLORA_KC_QUANT = 0,      /* blockwise NF4 code search + packing            */
+  QLORA_KC_DQ_CONST = 1,   /* exact mean and 8-bit quantisation of the scales */
+  QLORA_KC_DEQUANT = 2,    /* standalone doubleDequant                         */
+  QLORA_KC_FWD_GEMM = 3,   /* fused dequant + LoRA forward GEMM                */
+  QLORA_KC_BWD_GEMM = 4,   /* fused dequant + LoRA backward (dX) GEMM          */
+  QLORA_KC_LORA_GEMM = 5,  /* low-rank GEMMs: s X A^T, s dY B, dA, dB          */
+  QLORA_KC_AUX = 6,        /* split-K reductions, transposes                   */
+  QLORA_KC_COUNT = 7
+};
+
+/* Turn per-launch device timing on (1) or off (0).  While on, each launch is
+ * bracketed by two CUDA events on the call's stream (pooled; no allocation in
+ * steady state).  Launch counting is always on.  Host-only. */
+int qlora_profile_enable(int on);
+
+/* Wait for the recorded events, write the summed device milliseconds per
+ * kernel class (ms, may be NULL) and the launches per class since the last
+ * read (launches, may be NULL), then reset both.  Not a paper operation: a
+ * tracing aid for benchmarks. */
+int qlora_profile_read(double ms[QLORA_KC_COUNT], int64_t launches[QLORA_KC_COUNT]);
+
 /* Reason for the last error returned on this thread ("" if none). */
 const char *qlora_last_error(void);
 
