@@ -414,7 +414,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b_proj_set_m4096",
-                    choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "tiny_512"))
+                    choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
