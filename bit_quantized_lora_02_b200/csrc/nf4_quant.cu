@@ -12,13 +12,13 @@
 //      doubleDequant in BF16).
 //
 // Kernels (all memory-bound streaming kernels, no waits):
-//   k_nf4_quant    one pass over W0: block absmax (8-lane shuffle max), code
+//   k_nf4_quant    one pass over W0: block absmax (4-lane shuffle max), code
 //                  search, nibble packing; per-CTA exponent histogram of the
 //                  absmax values (for the exact mean) when DQ is on.
-//   k_dq_mean      one thread: exact sum of the histogram as a 320-bit
-//                  integer, correctly rounded to fp64, divided, rounded to fp32.
-//   k_dq_groups    one warp per group of 256 scales: subtract mean, absmax,
-//                  c1 = 127 / absmax, c2 = round-half-even(c1 * v).
+//   k_dq_groups    warp 0 of each CTA: exact sum of the histogram in 32-bit
+//                  limbs, rounded once to fp64, divided, rounded to fp32 (the
+//                  mean); then one warp per group of 256 scales: subtract the
+//                  mean, absmax, c1 = 127 / absmax, c2 = round-half-even(c1 v).
 //   k_nf4_dequant  one pass over the codes: scale reconstruction and
 //                  BF16(C[q] * s^), 16-byte vector stores.
 #include <cmath>
@@ -167,67 +167,83 @@ __device__ __forceinline__ float quotient(float w, float s, float r, bool fast) 
   return __fdiv_rn(w, s);
 }
 
+// One thread handles 16 consecutive weights (two 16-byte loads); 4 lanes share
+// a 64-weight block.  The cell table is replicated 16 times with a stride that
+// puts copy i on bank pair i, and lane l reads copy l % 16, so every lookup of
+// a half-warp hits 16 distinct bank pairs (no bank conflicts).
 template <bool kDQ>
 __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ W, int64_t N,
                                                    uint8_t* __restrict__ codes, float* __restrict__ absmax_f32,
                                                    uint16_t* __restrict__ absmax_bf16,
                                                    unsigned long long* __restrict__ hist, const QuantLut lut) {
-  __shared__ float2 s_lut[33];
+  __shared__ float2 s_lut[33 * 16];
   __shared__ uint32_t s_hist[256];
   const int tid = threadIdx.x;
-  if (tid < 33) s_lut[tid] = make_float2(lut.thr[tid], lut.base[tid]);
+  for (int i = tid; i < 33 * 16; i += 256) s_lut[i] = make_float2(lut.thr[i >> 4], lut.base[i >> 4]);
   if (kDQ) s_hist[tid] = 0;
   __syncthreads();
 
   const int lane = tid & 31;
-  const int64_t ngroups = (N + 7) >> 3;                      // groups of 8 elements
+  const uint32_t lut_lane = smem_u32(s_lut) + 8u * static_cast<uint32_t>(lane & 15);
+  const int64_t ngroups = (N + 15) >> 4;                     // groups of 16 elements
   const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
   for (int64_t g0 = static_cast<int64_t>(blockIdx.x) * 256 + (tid & ~31); g0 < ngroups; g0 += stride) {
     const int64_t g = g0 + lane;
-    const int64_t e0 = g << 3;
-    float w[8];
-    const bool full = (e0 + 8 <= N);
+    const int64_t e0 = g << 4;
+    float w[16];
+    const bool full = (e0 + 16 <= N);
     if (full) {
-      uint4 v = ldg_nc_v4(W + e0);
-      w[0] = bf16_lo(v.x); w[1] = bf16_hi(v.x); w[2] = bf16_lo(v.y); w[3] = bf16_hi(v.y);
-      w[4] = bf16_lo(v.z); w[5] = bf16_hi(v.z); w[6] = bf16_lo(v.w); w[7] = bf16_hi(v.w);
+      const uint4 v0 = ldg_nc_v4(W + e0);
+      const uint4 v1 = ldg_nc_v4(W + e0 + 8);
+      const uint32_t u[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        w[2 * i] = bf16_lo(u[i]);
+        w[2 * i + 1] = bf16_hi(u[i]);
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) w[i] = (e0 + i < N) ? __uint_as_float(static_cast<uint32_t>(W[e0 + i]) << 16) : 0.0f;
+      for (int i = 0; i < 16; ++i)
+        w[i] = (e0 + i < N) ? __uint_as_float(static_cast<uint32_t>(W[e0 + i]) << 16) : 0.0f;
     }
     float am = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(w[i]));
+    for (int i = 0; i < 16; ++i) am = fmaxf(am, fabsf(w[i]));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
     am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
-    am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 4));
     const float s = am;   // block absmax (bf16-exact)
 
-    uint32_t packed = 0x77777777u;   // exact-zero code for an all-zero block
+    uint32_t lo = 0x77777777u, hi = 0x77777777u;   // exact-zero code for an all-zero block
     if (s != 0.0f) {
       const bool fast = (s >= 0x1p-60f) && (s <= 0x1p60f);
       const float r = __frcp_rn(s);
-      packed = 0;
+      lo = 0;
+      hi = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float xn = quotient(w[i], s, r, fast);
         const float y = __fmaf_rn(xn, 16.0f, kCellBias);
-        const float2 e = s_lut[__float_as_uint(y) - kCellBiasBits];
+        const uint32_t cell = __float_as_uint(y) - kCellBiasBits;
+        float2 e;
+        asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(e.x), "=f"(e.y) : "r"(lut_lane + cell * 128u));
         const uint32_t q = __float_as_uint(e.y) + (xn > e.x ? 1u : 0u);
-        packed |= q << (4 * i);
+        if (i < 8) lo |= q << (4 * i);
+        else hi |= q << (4 * (i - 8));
       }
     }
     if (e0 < N) {
       if (full) {
-        *reinterpret_cast<uint32_t*>(codes + (e0 >> 1)) = packed;
+        uint32_t* c32 = reinterpret_cast<uint32_t*>(codes + (e0 >> 1));
+        c32[0] = lo;
+        c32[1] = hi;
       } else {
-        const int valid = static_cast<int>(N - e0);            // 1..7
-        const uint32_t keep = (1u << (4 * valid)) - 1u;          // pad nibbles are 0
-        packed &= keep;
+        const int valid = static_cast<int>(N - e0);             // 1..15
+        const uint64_t all = (static_cast<uint64_t>(hi) << 32) | lo;
+        const uint64_t packed = all & ((1ull << (4 * valid)) - 1ull);   // pad nibbles are 0
         const int nbytes = (valid + 1) >> 1;
         for (int b = 0; b < nbytes; ++b) codes[(e0 >> 1) + b] = static_cast<uint8_t>(packed >> (8 * b));
       }
-      if ((g & 7) == 0) {
+      if ((g & 3) == 0) {
         const int64_t blk = e0 >> 6;
         if (kDQ) {
           const uint32_t bits = __float_as_uint(s);
@@ -256,60 +272,100 @@ __global__ void k_zero_u64(unsigned long long* p, int n) {
 // Exact mean of the block scales.  Each scale is a bf16 value
 // sig * 2^(max(E,1) - 134) with an 8-bit significand; the histogram holds, per
 // exponent field E, the exact integer sum of significands.  The total is an
-// integer multiple of 2^-133 that fits in 5 64-bit limbs; it is rounded once
-// to fp64 (nearest, ties to even), divided by M_b in fp64 and rounded to fp32:
-// mean = RN32(RN64(RN64(sum) / M_b)).
+// integer multiple of 2^-133 below 2^384: one warp accumulates it in twelve
+// 32-bit limbs (each lane takes the exponents lane + 32m, whose limb index is
+// m or m - 1, so the limb array stays in registers), reduces the limbs across
+// the warp, and lane 0 propagates carries and rounds once to fp64 (nearest,
+// ties to even); then mean = RN32(RN64(sum) / M_b).
 // ----------------------------------------------------------------------------
-__global__ void k_dq_mean(const unsigned long long* __restrict__ hist, int64_t nblocks, float* __restrict__ mean) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  // 32-bit limbs held in 64-bit words; limb i covers bits [32 i, 32 i + 32).
-  unsigned long long A[12];
-  for (int i = 0; i < 12; ++i) A[i] = 0ull;
-  for (int E = 0; E < 256; ++E) {
-    const unsigned long long v = hist[E];   // < 2^51
-    if (!v) continue;
-    const int sh = (E ? E : 1) - 1;        // position of 2^(max(E,1) - 134) in units of 2^-133
-    const int li = sh >> 5, bo = sh & 31;
-    A[li] += (v << bo) & 0xFFFFFFFFull;
-    A[li + 1] += (v >> (32 - bo)) & 0xFFFFFFFFull;
-    if (bo) A[li + 2] += v >> (64 - bo);
-  }
-  for (int i = 0; i < 11; ++i) {
-    A[i + 1] += A[i] >> 32;
-    A[i] &= 0xFFFFFFFFull;
-  }
-  auto bit = [&](int p) -> unsigned long long { return (p < 0) ? 0ull : ((A[p >> 5] >> (p & 31)) & 1ull); };
-  int top = -1;
-  for (int p = 12 * 32 - 1; p >= 0; --p)
-    if (bit(p)) { top = p; break; }
-  double S = 0.0;
-  if (top >= 0) {
-    if (top < 53) {
-      S = ldexp(static_cast<double>(A[0] | (A[1] << 32)), -133);    // exact
-    } else {
-      unsigned long long m = 0;
-      for (int p = top; p > top - 53; --p) m = (m << 1) | bit(p);
-      const int rpos = top - 53;
-      bool sticky = false;
-      for (int p = rpos - 1; p >= 0 && !sticky; --p) sticky = bit(p) != 0;
-      if (bit(rpos) && (sticky || (m & 1ull))) ++m;   // ties to even; 2^53 stays exact
-      S = ldexp(static_cast<double>(m), top - 52 - 133);
+__device__ float exact_mean_warp(const unsigned long long* __restrict__ hist, int64_t nblocks) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long acc[12];
+#pragma unroll
+  for (int j = 0; j < 12; ++j) acc[j] = 0ull;
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    const int E = lane + 32 * m;
+    const unsigned long long v = __ldcg(hist + E);
+    const int sh = (E ? E : 1) - 1;
+    const int bo = sh & 31;
+    const unsigned long long p0 = (v << bo) & 0xFFFFFFFFull;
+    const unsigned long long p1 = (v >> (32 - bo)) & 0xFFFFFFFFull;
+    const unsigned long long p2 = bo ? (v >> (64 - bo)) : 0ull;
+    if ((sh >> 5) == m) {
+      acc[m] += p0;
+      acc[m + 1] += p1;
+      acc[m + 2] += p2;
+    } else if (m > 0) {   // lane 0, m >= 1: limb index m - 1
+      acc[m - 1] += p0;
+      acc[m] += p1;
+      acc[m + 1] += p2;
     }
   }
-  *mean = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblocks)));
+#pragma unroll
+  for (int j = 0; j < 12; ++j)
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], o);
+  float mean = 0.0f;
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < 11; ++j) {
+      acc[j + 1] += acc[j] >> 32;
+      acc[j] &= 0xFFFFFFFFull;
+    }
+    unsigned long long Wd[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) Wd[i] = acc[2 * i] | (acc[2 * i + 1] << 32);
+    int top = -1;
+#pragma unroll
+    for (int i = 5; i >= 0; --i)
+      if (top < 0 && Wd[i]) top = 64 * i + 63 - __clzll(static_cast<long long>(Wd[i]));
+    double S = 0.0;
+    if (top >= 0 && top < 53) {
+      S = ldexp(static_cast<double>(Wd[0]), -133);   // exact
+    } else if (top >= 53) {
+      auto bits = [&](int lo) -> unsigned long long {   // 64 bits starting at bit `lo`
+        const int w = lo >> 6, b = lo & 63;
+        unsigned long long x = Wd[w] >> b;
+        if (b && w + 1 < 6) x |= Wd[w + 1] << (64 - b);
+        return x;
+      };
+      unsigned long long m = bits(top - 52) & ((1ull << 53) - 1ull);
+      const int rpos = top - 53;
+      const bool rbit = (bits(rpos) & 1ull) != 0;
+      bool sticky = false;
+      const int rw = rpos >> 6;
+      for (int i = 0; i < rw; ++i) sticky |= (Wd[i] != 0);
+      sticky |= (Wd[rw] & ((1ull << (rpos & 63)) - 1ull)) != 0;
+      if (rbit && (sticky || (m & 1ull))) ++m;   // ties to even; 2^53 stays exact
+      S = ldexp(static_cast<double>(m), top - 52 - 133);
+    }
+    mean = __double2float_rn(__ddiv_rn(S, static_cast<double>(nblocks)));
+  }
+  return __shfl_sync(0xffffffffu, mean, 0);
 }
 
 // ----------------------------------------------------------------------------
 // Double quantisation of the scales: one warp per group of 256.
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ absmax_bf16, int64_t nblocks,
-                                                   const float* __restrict__ mean, int8_t* __restrict__ c2,
+                                                   const unsigned long long* __restrict__ hist,
+                                                   float* __restrict__ mean_out, int8_t* __restrict__ c2,
                                                    float* __restrict__ c1) {
+  __shared__ float s_mean;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x < 32) {
+    const float m = exact_mean_warp(hist, nblocks);   // every CTA derives the same value
+    if (lane == 0) {
+      s_mean = m;
+      if (blockIdx.x == 0) *mean_out = m;
+    }
+  }
+  __syncthreads();
   const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int64_t ngroups = (nblocks + 255) >> 8;
   if (g >= ngroups) return;
-  const float mu = *mean;
+  const float mu = s_mean;
   const int64_t j0 = g * 256 + lane * 8;
   float v[8];
   float am = 0.0f;
@@ -404,8 +460,8 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
 // ----------------------------------------------------------------------------
 // Host launchers
 // ----------------------------------------------------------------------------
-static int grid_for(int64_t ngroups8) {
-  int64_t ctas = (ngroups8 + 255) / 256;
+static int grid_for(int64_t nthreads) {
+  int64_t ctas = (nthreads + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (ctas > cap) ctas = cap;
   if (ctas < 1) ctas = 1;
@@ -419,8 +475,7 @@ size_t quant_workspace_bytes(int64_t N, bool dq) {
 }
 
 cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, void* ws, cudaStream_t st) {
-  const int64_t ng8 = (N + 7) / 8;
-  const int grid = grid_for(ng8);
+  const int grid = grid_for((N + 15) / 16);
   const int64_t nblk = (N + 63) / 64;
   if (!q.double_quant) {
     {
@@ -439,30 +494,21 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
     ProfScope ps_(QLORA_KC_QUANT, st);
     k_nf4_quant<true><<<grid, 256, 0, st>>>(W, N, q.codes, nullptr, amax16, hist, quant_lut());
   }
-  {
-    ProfScope ps_(QLORA_KC_DQ_CONST, st);
-    k_dq_mean<<<1, 32, 0, st>>>(hist, nblk, q.mean);
-  }
   const int64_t ngroups = (nblk + 255) / 256;
   {
     ProfScope ps_(QLORA_KC_DQ_CONST, st);
-    k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, q.mean, q.c2, q.c1);
+    k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, hist, q.mean, q.c2, q.c1);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st) {
   const int grid = grid_for((N + 7) / 8);
+  ProfScope ps_(QLORA_KC_DEQUANT, st);
   if (q.double_quant)
-    {
-      ProfScope ps_(QLORA_KC_DEQUANT, st);
-      k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
-    }
+    k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
   else
-    {
-      ProfScope ps_(QLORA_KC_DEQUANT, st);
-      k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
-    }
+    k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
   return cudaGetLastError();
 }
 

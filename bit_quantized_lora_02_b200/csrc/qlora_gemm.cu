@@ -209,15 +209,17 @@ struct MainCfg {
   static constexpr bool kBwd = MODE == Mode::Bwd;
   static constexpr int kWRows = kSwap ? 128 : (kBwd ? 64 : 256);      // W rows per K step
   static constexpr int kWCols = kBwd ? 256 : 64;                       // W columns per K step
-  static constexpr int kActRows = kSwap ? NT : 128;                    // token rows per K step
+  static constexpr int kActRows = kSwap ? NT : 256;                    // token rows per K step
+  static constexpr int kAccs = kSwap ? 1 : 2;                          // M=128 accumulators per tile
   static constexpr int kMmaN = kSwap ? NT : 256;
   static constexpr uint32_t kActBytes = kActRows * 128;
   static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
   static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
   static constexpr uint32_t kStageBytes = kActBytes + kWBytes + kCodeBytes;
-  static constexpr int kStagesRaw = static_cast<int>((200u * 1024u) / kStageBytes);
+  static constexpr int kStagesRaw = static_cast<int>((218u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr uint32_t kTmemCols = kMmaN <= 32 ? 32 : (kMmaN <= 64 ? 64 : (kMmaN <= 128 ? 128 : 256));
+  static constexpr uint32_t kTmemCols =
+      kSwap ? (kMmaN <= 32 ? 32u : (kMmaN <= 64 ? 64u : 128u)) : 512u;   // two 128x256 fp32 accumulators
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr int kThreads = 384;
   static constexpr uint32_t kIdesc = make_idesc_bf16(128, kMmaN, false, kBwd);
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(384, 1)
     n0 = static_cast<int64_t>(blockIdx.x) * 128;
   } else {
     n0 = static_cast<int64_t>(blockIdx.x) * 256;
-    m0 = static_cast<int64_t>(blockIdx.y) * 128;
+    m0 = static_cast<int64_t>(blockIdx.y) * 256;
   }
   const int split = blockIdx.z;
   const int s_begin = split * p.steps_per_split;
@@ -350,6 +352,11 @@ __global__ void __launch_bounds__(384, 1)
             db = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
           }
           umma_bf16(tmem_base, da, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+          if (Cfg::kAccs == 2) {
+            // token rows 128..255 of the tile share the same W tile: second accumulator
+            const uint64_t da1 = make_sdesc_sw128(a_act + 16384u + 32u * kk, 16u, 1024u);
+            umma_bf16(tmem_base + 256u, da1, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&empty_bar[st]);
       }
@@ -390,11 +397,16 @@ __global__ void __launch_bounds__(384, 1)
       }
       return wr * p.kpb + bc;
     };
-    ScaleRaw pre{};
-    bool pre_valid = false;
+    // block constants are fetched two K steps ahead of their use
+    ScaleRaw pre0{}, pre1{};
+    bool pre0_valid = false, pre1_valid = false;
     if (n_main > 0) {
-      int64_t b0 = block_of(s_begin, pre_valid);
-      if (pre_valid) pre = scale_fetch(sc, b0);
+      const int64_t b0 = block_of(s_begin, pre0_valid);
+      if (pre0_valid) pre0 = scale_fetch(sc, b0);
+    }
+    if (n_main > 1) {
+      const int64_t b1 = block_of(s_begin + 1, pre1_valid);
+      if (pre1_valid) pre1 = scale_fetch(sc, b1);
     }
     for (int l = 0; l < n_local; ++l) {
       const int st = l % S;
@@ -404,11 +416,13 @@ __global__ void __launch_bounds__(384, 1)
       if (!__all_sync(0xffffffffu, okw)) break;
       const uint32_t wt = smem_u32(w_tile(st));
       if (l < n_main) {
-        const ScaleRaw cur = pre;
-        const bool cur_valid = pre_valid;
-        if (l + 1 < n_main) {   // prefetch the next step's constants
-          int64_t bn = block_of(s_begin + l + 1, pre_valid);
-          if (pre_valid) pre = scale_fetch(sc, bn);
+        const ScaleRaw cur = pre0;
+        const bool cur_valid = pre0_valid;
+        pre0 = pre1;
+        pre0_valid = pre1_valid;
+        if (l + 2 < n_main) {
+          const int64_t bn = block_of(s_begin + l + 2, pre1_valid);
+          if (pre1_valid) pre1 = scale_fetch(sc, bn);
         }
         const uint32_t ct = smem_u32(code_tile(st));
         if (Cfg::kSwap) {
@@ -478,14 +492,14 @@ __global__ void __launch_bounds__(384, 1)
     tc_fence_after();
     if (ok) {
       const int q = warp & 3;          // TMEM lane quarter this warp may access
-      const int half = (warp - 4) >> 2;
+      const int half = (warp - 4) >> 2;   // non-swap: which accumulator (token rows 128*half..)
       const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
       if (!Cfg::kSwap) {
-        const int64_t m = m0 + 32 * q + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 128 * half + 32 * cb;
+        const int64_t m = m0 + 128 * half + 32 * q + lane;
+        for (int cb = 0; cb < 8; ++cb) {
+          const int col0 = 32 * cb;
           uint32_t v[32];
-          tmem_ld32(lane_base + col0, v);
+          tmem_ld32(lane_base + 256u * half + col0, v);
           tmem_ld_wait();
           if (m < p.M) {
             const int64_t n = n0 + col0;
@@ -818,6 +832,17 @@ static int plan_splits(int64_t tiles, int steps, int min_steps, int slots_per_sm
   return best;
 }
 
+// Low-rank GEMMs are bound by reading their activation operand once: about one
+// CTA per SM, each streaming at least 8 K steps, keeps per-CTA fixed costs
+// (barrier set-up, TMEM allocation, the fp32 partial write) small.
+static int plan_thin_splits(int64_t tiles, int steps) {
+  int64_t s = tiles > 0 ? kSms / tiles : 1;
+  if (s < 1) s = 1;
+  const int64_t cap = steps / 8 > 1 ? steps / 8 : 1;
+  if (s > cap) s = cap;
+  return static_cast<int>(s);
+}
+
 struct Plan {
   // thin GEMMs
   int splits_T, splits_U, splits_dA, splits_dB;
@@ -840,7 +865,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
   Plan pl{};
   const int rp = qlora_rank_pad(r);
   const int64_t mt = ceil_div(M, 128);
-  pl.splits_T = plan_splits(mt, static_cast<int>(k / 64), 4, 2);
+  pl.splits_T = plan_thin_splits(mt, static_cast<int>(k / 64));
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -855,22 +880,22 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     if (pl.nt) {
       pl.main_splits = plan_splits(ceil_div(d, 128), steps, 8, 1);
     } else {
-      pl.main_splits = plan_splits(ceil_div(d, 256) * mt, steps, 8, 1);
+      pl.main_splits = plan_splits(ceil_div(d, 256) * ceil_div(M, 256), steps, 8, 1);
     }
     pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * d * 4) : 0;
   } else {
     pl.nt = 0;
     const int dsteps = static_cast<int>(ceil_div(d, 64));
-    pl.splits_U = plan_splits(mt, dsteps, 4, 2);
+    pl.splits_U = plan_thin_splits(mt, dsteps);
     pl.off_Bt = take(static_cast<size_t>(rp) * d * 2);
     pl.off_U = take(static_cast<size_t>(M) * rp * 2);
     pl.off_partU = take(static_cast<size_t>(pl.splits_U) * M * rp * 4);
     const int msteps = static_cast<int>(ceil_div(M, 64));
-    pl.splits_dA = plan_splits(ceil_div(k, 128), msteps, 4, 2);
-    pl.splits_dB = plan_splits(ceil_div(d, 128), msteps, 4, 2);
+    pl.splits_dA = plan_thin_splits(ceil_div(k, 128), msteps);
+    pl.splits_dB = plan_thin_splits(ceil_div(d, 128), msteps);
     pl.off_partA = take(static_cast<size_t>(pl.splits_dA) * k * rp * 4);
     pl.off_partB = take(static_cast<size_t>(pl.splits_dB) * d * rp * 4);
-    pl.main_splits = plan_splits(ceil_div(k, 256) * mt, dsteps, 8, 1);
+    pl.main_splits = plan_splits(ceil_div(k, 256) * ceil_div(M, 256), dsteps, 8, 1);
     pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * k * 4) : 0;
   }
   pl.total = off;
@@ -999,9 +1024,9 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
          make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 128, false) &&
          map_bf16(&t_ext, T, rp, M, 64, nt);
   } else {
-    ok = map_bf16(&t_act, a.X, k, M, 64, 128) &&
+    ok = map_bf16(&t_act, a.X, k, M, 64, 256) &&
          make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 256, false) &&
-         map_bf16(&t_ext, T, rp, M, 64, 128);
+         map_bf16(&t_ext, T, rp, M, 64, 256);
   }
   if (!ok) {
     *why = "tensor map encoding failed (forward)";
@@ -1011,7 +1036,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   if (nt) {
     grid = dim3(static_cast<unsigned>(ceil_div(d, 128)), 1, static_cast<unsigned>(mp.splits));
   } else {
-    grid = dim3(static_cast<unsigned>(ceil_div(d, 256)), static_cast<unsigned>(ceil_div(M, 128)),
+    grid = dim3(static_cast<unsigned>(ceil_div(d, 256)), static_cast<unsigned>(ceil_div(M, 256)),
                 static_cast<unsigned>(mp.splits));
   }
   switch (nt) {
@@ -1082,13 +1107,13 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     mp.out = a.dX;
     mp.partial = reinterpret_cast<float*>(ws + pl.off_main);
     CUtensorMap t_act, t_codes, t_ext;
-    if (!map_bf16(&t_act, a.dY, d, M, 64, 128) ||
+    if (!map_bf16(&t_act, a.dY, d, M, 64, 256) ||
         !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 64, false) ||
-        !map_bf16(&t_ext, U, rp, M, 64, 128)) {
+        !map_bf16(&t_ext, U, rp, M, 64, 256)) {
       *why = "tensor map encoding failed (backward)";
       return QLORA_ERR_CUDA;
     }
-    dim3 grid(static_cast<unsigned>(ceil_div(k, 256)), static_cast<unsigned>(ceil_div(M, 128)),
+    dim3 grid(static_cast<unsigned>(ceil_div(k, 256)), static_cast<unsigned>(ceil_div(M, 256)),
               static_cast<unsigned>(mp.splits));
     rc = launch_main<Mode::Bwd, 0>(t_act, t_codes, t_ext, mp, grid, st, why);
     if (rc) return rc;
