@@ -218,8 +218,12 @@ def run_ours(args, work, wl_name):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
+    from bit_quantized_lora_02_b200.dp import GradBucket, max_over_ranks as dp_max
+
     M, r, alpha = work["m"], work["r"], work["alpha"]
     projs = work["proj"]
+    # adapter gradients of every projection in one flat fp32 bucket (one all-reduce per step)
+    bucket = GradBucket([s_ for _, d, k in projs for s_ in ((r, k), (d, r))], dev)
     bufs = []
     h2d_bytes = d2h_bytes = 0
     for pi, (name, d, k) in enumerate(projs):
@@ -237,8 +241,8 @@ def run_ours(args, work, wl_name):
         b["Y"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
         b["T"] = torch.empty(M, Q.qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
         b["dX"] = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
-        b["dA"] = torch.empty(r, k, dtype=torch.float32, device=dev)
-        b["dB"] = torch.empty(d, r, dtype=torch.float32, device=dev)
+        b["dA"] = bucket.views[2 * pi]
+        b["dB"] = bucket.views[2 * pi + 1]
         nws = max(Q.qlora_linear_workspace_size(M, d, k, r, False), Q.qlora_linear_workspace_size(M, d, k, r, True))
         b["ws"] = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         for key in ("Y", "dX", "dA", "dB"):
@@ -256,9 +260,7 @@ def run_ours(args, work, wl_name):
             Q.qlora_linear_bwd(b["dY"], b["X"], b["q"], b["A"], b["B"], alpha, T_save=b["T"], dX=b["dX"],
                                dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream)
         if world > 1:
-            for b in bufs:
-                dist.all_reduce(b["dA"])
-                dist.all_reduce(b["dB"])
+            bucket.allreduce()
 
     def h2d():
         for b in bufs:
@@ -275,11 +277,7 @@ def run_ours(args, work, wl_name):
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return dp_max(x, dev)
 
     # correctness guard before timing: the device status word must be clean
     step()
