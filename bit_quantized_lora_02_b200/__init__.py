@@ -25,7 +25,7 @@ QLORA_OK = 0
 _STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTED", -3: "QLORA_ERR_ALIGNMENT",
            -4: "QLORA_ERR_WORKSPACE", -5: "QLORA_ERR_CUDA", -6: "QLORA_ERR_DEVICE"}
 
-EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_rank_pad", "qlora_linear_workspace_size",
+EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_rank_pad", "qlora_linear_workspace_size",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error",
            "qlora_profile_enable", "qlora_profile_read")
 
@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
     c_i64, c_i32, c_sz, vp = ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_void_p
     L.qlora_nf4_sizes.argtypes = [c_i64, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz), ctypes.POINTER(c_sz)]
     L.nf4_quantize.argtypes = [vp, ctypes.POINTER(QloraNF4), vp, c_sz, vp]
+    L.nf4_quantize_noalloc.argtypes = [vp, ctypes.POINTER(QloraNF4), vp]
     L.nf4_dequantize.argtypes = [ctypes.POINTER(QloraNF4), vp, vp]
     L.qlora_rank_pad.argtypes = [c_i32]
     L.qlora_rank_pad.restype = c_i32
@@ -72,7 +73,7 @@ def lib() -> ctypes.CDLL:
     L.qlora_last_error.restype = ctypes.c_char_p
     L.qlora_profile_enable.argtypes = [c_i32]
     L.qlora_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
-    for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_dequantize", "qlora_linear_workspace_size",
+    for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_workspace_size",
                  "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
                  "qlora_profile_enable", "qlora_profile_read"):
         getattr(L, name).restype = c_i32
@@ -155,6 +156,23 @@ def nf4_quantize(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4W
     _check(lib().nf4_quantize(W0.data_ptr(), ctypes.byref(st), _ptr(workspace),
                               0 if workspace is None else workspace.numel() * workspace.element_size(),
                               _stream(stream)))
+    return q
+
+
+NOALLOC_MAX_WEIGHTS = 1 << 28
+
+
+def nf4_quantize_noalloc(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4Weight] = None,
+                         stream=None) -> NF4Weight:
+    """nf4_quantize without a workspace: for callers that cannot allocate device
+    memory, the library uses its own fixed scratch (weights up to 2^28 elements).
+    Only `out`'s buffers are the caller's; pass them pre-allocated to allocate
+    nothing in this call."""
+    assert W0.dtype == torch.bfloat16 and W0.dim() == 2 and W0.is_contiguous()
+    d, k = W0.shape
+    q = out or nf4_alloc(d, k, double_quant, W0.device)
+    st = q.struct()
+    _check(lib().nf4_quantize_noalloc(W0.data_ptr(), ctypes.byref(st), _stream(stream)))
     return q
 
 

@@ -512,4 +512,49 @@ cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cu
   return cudaGetLastError();
 }
 
+// ----------------------------------------------------------------------------
+// Quantisation with library-owned scratch (nf4_quantize_noalloc).
+//
+// Double quantisation needs device scratch between its kernels: the 256-entry
+// exponent histogram of the block scales and a bf16 copy of every block scale.
+// nf4_quantize takes that scratch from the caller.  Some callers have no way to
+// provide it: a plugin running inside a host application whose memory manager
+// owns all device memory, or a service that reserves its memory up front and
+// must not call cudaMalloc later (it can synchronize the device and can fail
+// once memory is fragmented).  For them the scratch lives in the file-scope
+// array below, sized for QLORA_NOALLOC_MAX_WEIGHTS weights (about 8 MiB, held by
+// every GPU that loads the library until the process exits).
+//
+// Host code must not pass the array's name to a kernel: on the host that name
+// is only a stand-in, not a device address.  The first call on each device
+// (with that device current) asks the runtime for the real address with
+// cudaGetSymbolAddress and caches it.
+// ----------------------------------------------------------------------------
+constexpr size_t noalloc_scratch_bytes() {
+  return 256 * sizeof(unsigned long long) +
+         ((static_cast<size_t>(QLORA_NOALLOC_MAX_WEIGHTS / 64) * 2 + 16 + 255) / 256) * 256;
+}
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[noalloc_scratch_bytes()];
+
+static std::mutex g_noalloc_mu;
+static void* g_noalloc_addr[64] = {};
+
+cudaError_t noalloc_scratch(void** out, size_t* bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  *bytes = noalloc_scratch_bytes();
+  return cudaSuccess;
+}
+
 }  // namespace qlora

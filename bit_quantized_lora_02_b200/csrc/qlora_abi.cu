@@ -149,6 +149,32 @@ int nf4_quantize(const uint16_t* W0, const qlora_nf4_t* q, void* workspace, size
   return check_cuda(launch_quantize(W0, N, *q, workspace, static_cast<cudaStream_t>(stream)), "nf4_quantize launch");
 }
 
+int nf4_quantize_noalloc(const uint16_t* W0, const qlora_nf4_t* q, qlora_stream_t stream) {
+  int64_t N = 0;
+  int rc = check_nf4(q, &N);
+  if (rc) return rc;
+  if (N == 0) return ok();
+  if (!W0) return fail(QLORA_ERR_INVALID_ARG, "W0 is NULL");
+  if (!aligned(W0, 16)) return fail(QLORA_ERR_ALIGNMENT, "W0 must be 16-byte aligned");
+  if (N > QLORA_NOALLOC_MAX_WEIGHTS)
+    return fail(QLORA_ERR_UNSUPPORTED,
+                "nf4_quantize_noalloc: %lld weights exceed the built-in scratch limit of %lld; "
+                "use nf4_quantize with a workspace",
+                (long long)N, (long long)QLORA_NOALLOC_MAX_WEIGHTS);
+  if (!quant_lut_valid()) return fail(QLORA_ERR_UNSUPPORTED, "code-search table failed its self-check");
+  if ((rc = bind_device(W0))) return rc;
+  void* scratch = nullptr;
+  size_t scratch_bytes = 0;
+  if (q->double_quant) {
+    cudaError_t e = noalloc_scratch(&scratch, &scratch_bytes);
+    if (e != cudaSuccess) return fail(QLORA_ERR_CUDA, "scratch address lookup: %s", cudaGetErrorString(e));
+    if (scratch_bytes < quant_workspace_bytes(N, true))
+      return fail(QLORA_ERR_UNSUPPORTED, "built-in scratch too small");
+  }
+  return check_cuda(launch_quantize(W0, N, *q, scratch, static_cast<cudaStream_t>(stream)),
+                    "nf4_quantize_noalloc launch");
+}
+
 int nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_stream_t stream) {
   int64_t N = 0;
   int rc = check_nf4(q, &N);

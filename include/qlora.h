@@ -115,6 +115,27 @@ int qlora_nf4_sizes(int64_t d, int64_t k, int32_t blocksize, int32_t double_quan
 int nf4_quantize(const uint16_t *W0, const qlora_nf4_t *q, void *workspace, size_t workspace_bytes,
                  qlora_stream_t stream);
 
+/* Largest weight (d * k elements) that nf4_quantize_noalloc accepts. */
+#define QLORA_NOALLOC_MAX_WEIGHTS ((int64_t)1 << 28)
+
+/* nf4_quantize for callers that cannot allocate device memory.  The pages have
+ * no counterpart to this entry point; it is a convenience of this library.
+ * Callers such as a plugin inside an application whose memory manager owns all
+ * device memory, or a service that reserves its memory at start-up and must
+ * not call cudaMalloc afterwards, have no workspace to pass.  This variant
+ * needs none: the scratch that double quantisation uses lives in a fixed
+ * array inside the library (about 8 MiB on every GPU that loads the library,
+ * kept until the process exits).  Outputs are bit-identical to nf4_quantize.
+ *   - d * k above QLORA_NOALLOC_MAX_WEIGHTS returns QLORA_ERR_UNSUPPORTED;
+ *     use nf4_quantize with a workspace for larger weights.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the one array, and each call clears the part that must
+ *     start at zero.  Calls whose kernels may overlap on the GPU (for instance
+ *     on two streams without ordering) race on it and give wrong results. */
+int nf4_quantize_noalloc(const uint16_t *W0, const qlora_nf4_t *q, qlora_stream_t stream);
+
 /* doubleDequant ("Double quantization and double dequantization"): writes the
  * reconstructed weights W_out[i] = BF16(RN32(C[code_i] * s^_j)) with
  * s^_j = RN32(RN32(c2_j / c1_g) + mean) (DQ on) or s^_j = absmax_j (DQ off).
