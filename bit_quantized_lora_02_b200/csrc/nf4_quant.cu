@@ -362,51 +362,54 @@ __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ 
     }
   }
   __syncthreads();
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int64_t ngroups = (nblocks + 255) >> 8;
-  if (g >= ngroups) return;
   const float mu = s_mean;
-  const int64_t j0 = g * 256 + lane * 8;
-  float v[8];
-  float am = 0.0f;
-  if (j0 + 8 <= nblocks) {
-    uint4 raw = ldg_nc_v4(absmax_bf16 + j0);
-    const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); g < ngroups;
+       g += static_cast<int64_t>(gridDim.x) * 8) {
+    const int64_t j0 = g * 256 + lane * 8;
+    float v[8];
+    float am = 0.0f;
+    if (j0 + 8 <= nblocks) {
+      uint4 raw = ldg_nc_v4(absmax_bf16 + j0);
+      const uint32_t r4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __fsub_rn(bf16_lo(r4[i]), mu);
-      v[2 * i + 1] = __fsub_rn(bf16_hi(r4[i]), mu);
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __fsub_rn(bf16_lo(r4[i]), mu);
+        v[2 * i + 1] = __fsub_rn(bf16_hi(r4[i]), mu);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        v[i] = (j0 + i < nblocks)
+                   ? __fsub_rn(__uint_as_float(static_cast<uint32_t>(absmax_bf16[j0 + i]) << 16), mu)
+                   : 0.0f;
     }
-  } else {
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      v[i] = (j0 + i < nblocks) ? __fsub_rn(__uint_as_float(static_cast<uint32_t>(absmax_bf16[j0 + i]) << 16), mu)
-                                : 0.0f;
-  }
+    for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
 #pragma unroll
-  for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
+    for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    const float c = (am == 0.0f) ? 1.0f : __fdiv_rn(127.0f, am);
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  const float c = (am == 0.0f) ? 1.0f : __fdiv_rn(127.0f, am);
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    int q = 0;
-    if (am != 0.0f) {
-      q = __float2int_rn(__fmul_rn(c, v[i]));
-      q = max(-127, min(127, q));
+    for (int i = 0; i < 8; ++i) {
+      int q = 0;
+      if (am != 0.0f) {
+        q = __float2int_rn(__fmul_rn(c, v[i]));
+        q = max(-127, min(127, q));
+      }
+      const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
+      if (i < 4) lo |= b << (8 * i);
+      else hi |= b << (8 * (i - 4));
     }
-    const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
-    if (i < 4) lo |= b << (8 * i);
-    else hi |= b << (8 * (i - 4));
+    if (j0 + 8 <= nblocks) {
+      *reinterpret_cast<uint2*>(c2 + j0) = make_uint2(lo, hi);
+    } else {
+      for (int i = 0; i < 8; ++i)
+        if (j0 + i < nblocks)
+          c2[j0 + i] = static_cast<int8_t>(((i < 4) ? (lo >> (8 * i)) : (hi >> (8 * (i - 4)))) & 0xFFu);
+    }
+    if (lane == 0) c1[g] = c;
   }
-  if (j0 + 8 <= nblocks) {
-    *reinterpret_cast<uint2*>(c2 + j0) = make_uint2(lo, hi);
-  } else {
-    for (int i = 0; i < 8; ++i)
-      if (j0 + i < nblocks) c2[j0 + i] = static_cast<int8_t>(((i < 4) ? (lo >> (8 * i)) : (hi >> (8 * (i - 4)))) & 0xFFu);
-  }
-  if (lane == 0) c1[g] = c;
 }
 
 // ----------------------------------------------------------------------------
@@ -497,7 +500,10 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
   const int64_t ngroups = (nblk + 255) / 256;
   {
     ProfScope ps_(QLORA_KC_DQ_CONST, st);
-    k_dq_groups<<<static_cast<int>((ngroups + 7) / 8), 256, 0, st>>>(amax16, nblk, hist, q.mean, q.c2, q.c1);
+    // every CTA derives the mean itself, so keep the grid near one wave and loop over groups
+    const int64_t want = (ngroups + 7) / 8;
+    const int grid_g = static_cast<int>(want < 2 * num_sms() ? want : 2 * num_sms());
+    k_dq_groups<<<grid_g, 256, 0, st>>>(amax16, nblk, hist, q.mean, q.c2, q.c1);
   }
   return cudaGetLastError();
 }

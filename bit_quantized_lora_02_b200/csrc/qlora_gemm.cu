@@ -19,25 +19,28 @@
 // never written to device memory.
 //
 // Kernels
-//   k_qlora_main<Fwd>     Y tile 128 tokens x 256 weight rows.  TMA stages X
-//                         and the packed codes; 8 dequant warps expand the codes
+//   k_qlora_main<Fwd>     Y tile 256 tokens x 256 weight rows.  TMA stages X
+//                         and the packed codes; 16 dequant warps expand the codes
 //                         to bf16 in the 128-byte-swizzled K-major layout the
 //                         tensor core reads; one thread issues tcgen05.mma into
-//                         a 128 x 256 fp32 TMEM accumulator; the LoRA term is
+//                         two 128 x 256 fp32 TMEM accumulators; the LoRA term is
 //                         one (or more) extra 64-wide K steps.
-//   k_qlora_main<Bwd>     dX tile 128 tokens x 256 input columns; the dequant
+//   k_qlora_main<Bwd>     dX tile 256 tokens x 256 input columns; the dequant
 //                         warps write W in the MN-major swizzled layout (the
 //                         reduction runs over W's rows).
 //   k_qlora_main<FwdSwap> few tokens (M <= 128): W rows are the MMA's M side
 //                         (128 per tile), the tokens its N side, so the tensor
 //                         core is not padded to 128 tokens; split over K.
-//   k_thin<false,false>   T_s and U_s partial sums (K-major operands).
+//   k_thin<false,*>       T_s and U_s partial sums (K-major activations; A read
+//                         K-major, B read MN-major straight from its storage).
 //   k_thin<true,true>     dA^T and dB partial sums (MN-major operands, the
 //                         reduction runs over tokens).
 //   k_reduce_*            deterministic sums of split-K partials.
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "nf4_table.h"
 #include "qlora_device.cuh"
@@ -146,9 +149,15 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
   return v;
 }
 
@@ -221,12 +230,13 @@ struct MainCfg {
   static constexpr uint32_t kTmemCols =
       kSwap ? (kMmaN <= 32 ? 32u : (kMmaN <= 64 ? 64u : 128u)) : 512u;   // two 128x256 fp32 accumulators
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
-  static constexpr int kThreads = 384;
+  static constexpr int kDeqThreads = 512;     // 16 dequant warps (warps 2..17)
+  static constexpr int kThreads = 64 + kDeqThreads;
   static constexpr uint32_t kIdesc = make_idesc_bf16(128, kMmaN, false, kBwd);
 };
 
 template <Mode MODE, int NT>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(576, 1)
     k_qlora_main(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_ext, const MainParams p) {
   using Cfg = MainCfg<MODE, NT>;
@@ -263,7 +273,7 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&deq_bar[i], 8);
+      mbar_init(&deq_bar[i], 16);
       mbar_init(&empty_bar[i], 1);
     }
     mbar_init(tmem_full, 1);
@@ -362,9 +372,17 @@ __global__ void __launch_bounds__(384, 1)
       }
       umma_commit(tmem_full);   // also drains MMAs on the abort path
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------ dequant warps
-    const int t = threadIdx.x - 128;   // 0..255
+    // 16 warps; each NF4 block of the tile is shared by kTPB threads, each
+    // expanding kCPT 16-byte chunks (8 weights each) of the block's 128-byte row.
+    constexpr int kBlocks = Cfg::kWRows * Cfg::kWCols / 64;   // blocks per K step: 256 (Fwd, Bwd), 128 (Swap)
+    constexpr int kTPB = Cfg::kDeqThreads / kBlocks;
+    constexpr int kCPT = 8 / kTPB;
+    const int t = threadIdx.x - 64;   // 0..511
+    const int blk_id = t / kTPB;
+    const int part = t % kTPB;
+    const int c_first = part * kCPT;
     // the codebook as register immediates (no memory traffic)
     constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
     float C[16];
@@ -372,18 +390,10 @@ __global__ void __launch_bounds__(384, 1)
     for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
     const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
-    // this thread's W row and block column inside the tile
-    int row, sub;   // Fwd: row = t; Swap: row = t >> 1, sub = half; Bwd: row = t & 63 (K row), sub = chunk
-    if (Cfg::kSwap) {
-      row = t >> 1;
-      sub = t & 1;
-    } else if (Cfg::kBwd) {
-      row = t & 63;
-      sub = t >> 6;
-    } else {
-      row = t;
-      sub = 0;
-    }
+    // this thread's block inside the tile: Fwd/Swap: row = W row; Bwd: row =
+    // W row within the 64-row K step (MN-major K row), sub = 64-column chunk
+    const int row = Cfg::kBwd ? (blk_id & 63) : blk_id;
+    const int sub = Cfg::kBwd ? (blk_id >> 6) : 0;
     auto block_of = [&](int i, bool& valid) -> int64_t {
       int64_t wr, bc;
       if (Cfg::kBwd) {
@@ -414,7 +424,7 @@ __global__ void __launch_bounds__(384, 1)
       bool okw = mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
       okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
       if (!__all_sync(0xffffffffu, okw)) break;
-      const uint32_t wt = smem_u32(w_tile(st));
+      const uint32_t wt = smem_u32(w_tile(st)) + (Cfg::kBwd ? 8192u * sub : 0u);
       if (l < n_main) {
         const ScaleRaw cur = pre0;
         const bool cur_valid = pre0_valid;
@@ -424,31 +434,26 @@ __global__ void __launch_bounds__(384, 1)
           const int64_t bn = block_of(s_begin + l + 2, pre1_valid);
           if (pre1_valid) pre1 = scale_fetch(sc, bn);
         }
-        const uint32_t ct = smem_u32(code_tile(st));
-        if (Cfg::kSwap) {
-          uint4 cw = lds128(ct + row * 32 + sub * 16);
-          const uint32_t w4[4] = {cw.x, cw.y, cw.z, cw.w};
-          if (cur_valid) {
-            const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) sts128(wt + sw128_offset(row, 4 * sub + c), dq8(w4[c], tab));
-          } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) sts128(wt + sw128_offset(row, 4 * sub + c), make_uint4(0, 0, 0, 0));
-          }
+        // codes of this thread's chunks: 4 bytes per chunk
+        const uint32_t src = smem_u32(code_tile(st)) + (Cfg::kBwd ? (row * 128 + sub * 32) : (row * 32)) + 4 * c_first;
+        uint32_t w[kCPT];
+        if constexpr (kCPT == 4) {
+          const uint4 cw = lds128(src);
+          w[0] = cw.x;
+          w[1] = cw.y;
+          w[2] = cw.z;
+          w[3] = cw.w;
         } else {
-          const uint32_t src = Cfg::kBwd ? (ct + row * 128 + sub * 32) : (ct + row * 32);
-          const uint32_t dst = Cfg::kBwd ? (wt + sub * 8192) : wt;
-          uint4 c0 = lds128(src), c1 = lds128(src + 16);
-          const uint32_t w8[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-          if (cur_valid) {
-            const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) sts128(dst + sw128_offset(row, c), dq8(w8[c], tab));
-          } else {
+          for (int c = 0; c < kCPT; ++c) w[c] = lds32(src + 4 * c);
+        }
+        if (cur_valid) {
+          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) sts128(dst + sw128_offset(row, c), make_uint4(0, 0, 0, 0));
-          }
+          for (int c = 0; c < kCPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w[c], tab));
+        } else {
+#pragma unroll
+          for (int c = 0; c < kCPT; ++c) sts128(wt + sw128_offset(row, c_first + c), make_uint4(0, 0, 0, 0));
         }
       } else {
         // LoRA extension step: copy 64 columns of the adapter into the W tile
@@ -456,28 +461,27 @@ __global__ void __launch_bounds__(384, 1)
         if (Cfg::kBwd) {
           // A (r x k): K row j = 64e + row, N columns n0 + 64 sub + [0, 64)
           const int64_t j = 64ll * e + row;
-          const int64_t c0 = n0 + 64 * sub;
-          const bool v = (j < p.r) && (c0 < p.k);
-          const uint16_t* src = p.lora + j * p.k + c0;
+          const int64_t col = n0 + 64 * sub;
+          const bool v = (j < p.r) && (col < p.k);
+          const uint16_t* src = p.lora + j * p.k + col;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
+          for (int c = 0; c < kCPT; ++c) {
             uint4 val = make_uint4(0, 0, 0, 0);
-            if (v) val = __ldg(reinterpret_cast<const uint4*>(src + 8 * c));
-            sts128(wt + sub * 8192 + sw128_offset(row, c), val);
+            if (v) val = __ldg(reinterpret_cast<const uint4*>(src + 8 * (c_first + c)));
+            sts128(wt + sw128_offset(row, c_first + c), val);
           }
         } else {
-          // B (d x r): row n, columns 64e + [0, 64) (Fwd) or a half of them (Swap)
+          // B (d x r): row n, columns 64e + 8 (c_first + c) + [0, 8)
           const int64_t n = n0 + row;
-          const int cbeg = Cfg::kSwap ? 4 * sub : 0;
-          const int cnum = Cfg::kSwap ? 4 : 8;
-          for (int c = cbeg; c < cbeg + cnum; ++c) {
+#pragma unroll
+          for (int c = 0; c < kCPT; ++c) {
             uint32_t h[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              const int64_t j = 64ll * e + 8 * c + q;
+              const int64_t j = 64ll * e + 8 * (c_first + c) + q;
               h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
             }
-            sts128(wt + sw128_offset(row, c),
+            sts128(wt + sw128_offset(row, c_first + c),
                    make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
           }
         }
@@ -488,18 +492,21 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // ------------------------------------------------------------ epilogue
+    // warp w may read TMEM lanes 32 (w % 4) ..; the four warps sharing a lane
+    // quarter split the columns (idx = 0..3)
     const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
     tc_fence_after();
     if (ok) {
-      const int q = warp & 3;          // TMEM lane quarter this warp may access
-      const int half = (warp - 4) >> 2;   // non-swap: which accumulator (token rows 128*half..)
+      const int q = warp & 3;
+      const int idx = (warp - 2) >> 2;
       const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
       if (!Cfg::kSwap) {
-        const int64_t m = m0 + 128 * half + 32 * q + lane;
-        for (int cb = 0; cb < 8; ++cb) {
-          const int col0 = 32 * cb;
+        const int acc = idx >> 1;                       // which 128-token half of the tile
+        const int64_t m = m0 + 128 * acc + 32 * q + lane;
+        for (int cb = 0; cb < 4; ++cb) {
+          const int col0 = 128 * (idx & 1) + 32 * cb;
           uint32_t v[32];
-          tmem_ld32(lane_base + 256u * half + col0, v);
+          tmem_ld32(lane_base + 256u * acc + col0, v);
           tmem_ld_wait();
           if (m < p.M) {
             const int64_t n = n0 + col0;
@@ -525,10 +532,10 @@ __global__ void __launch_bounds__(384, 1)
             }
           }
         }
-      } else if (half == 0) {
+      } else {
         // lanes = W rows n, columns = tokens
         const int64_t n = n0 + 32 * q + lane;
-        for (int cb = 0; cb < NT / 16; ++cb) {
+        for (int cb = idx; cb < NT / 16; cb += 4) {
           uint32_t v[16];
           tmem_ld16(lane_base + 16 * cb, v);
           tmem_ld_wait();
@@ -582,25 +589,26 @@ struct ThinParams {
   float* partial;        // [splits][rows][rp]
 };
 
-template <bool kMN>
 struct ThinCfg {
   static constexpr int kStages = 4;
   static constexpr uint32_t kABytes = 128 * 128;      // 128 rows x 64 K (K-major) or 2 x (64 K x 64 MN)
-  static constexpr uint32_t kBBytesMax = 256 * 128;   // rp <= 256
-  static constexpr uint32_t kStageBytes = kABytes + kBBytesMax;
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 + 256;
+  // B holds rp x 64 bf16; shared memory is sized by rp so that two CTAs fit on
+  // an SM when rp <= 64 (one streams while the other sets up or drains)
+  __host__ __device__ static uint32_t stage_bytes(int rp) { return kABytes + 128u * static_cast<uint32_t>(rp); }
+  __host__ __device__ static uint32_t smem_bytes(int rp) { return kStages * stage_bytes(rp) + 1024 + 256; }
 };
 
-template <bool kMN>
-__global__ void __launch_bounds__(128, 1)
+template <bool kAMN, bool kBMN>
+__global__ void __launch_bounds__(128, 2)
     k_thin(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, const ThinParams p) {
-  using Cfg = ThinCfg<kMN>;
+  using Cfg = ThinCfg;
   constexpr int S = Cfg::kStages;
+  const uint32_t stage_bytes = Cfg::stage_bytes(p.rp);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * stage_bytes);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + S;
   uint64_t* tmem_full = bars + 2 * S;
@@ -637,8 +645,8 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  auto a_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
-  auto b_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kABytes; };
+  auto a_tile = [&](int st) { return base + st * stage_bytes; };
+  auto b_tile = [&](int st) { return base + st * stage_bytes + Cfg::kABytes; };
 
   if (warp == 0 && lane == 0) {
     int issued = 0;
@@ -648,12 +656,15 @@ __global__ void __launch_bounds__(128, 1)
       if (!mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
       const int i = s_begin + l;
       mbar_arrive_expect_tx(&full_bar[st], Cfg::kABytes + b_bytes);
-      if (!kMN) {
+      if (!kAMN) {
         tma_load_2d(a_tile(st), &tm_a, &full_bar[st], 64 * i, static_cast<int>(row0));
-        tma_load_2d(b_tile(st), &tm_b, &full_bar[st], 64 * i, 0);
       } else {
         tma_load_2d(a_tile(st), &tm_a, &full_bar[st], static_cast<int>(row0), 64 * i);
         tma_load_2d(a_tile(st) + 8192, &tm_a, &full_bar[st], static_cast<int>(row0) + 64, 64 * i);
+      }
+      if (!kBMN) {
+        tma_load_2d(b_tile(st), &tm_b, &full_bar[st], 64 * i, 0);
+      } else {
         for (int c = 0; c < rp / 64; ++c) tma_load_2d(b_tile(st) + 8192 * c, &tm_b, &full_bar[st], 64 * c, 64 * i);
       }
       ++issued;
@@ -668,7 +679,7 @@ __global__ void __launch_bounds__(128, 1)
       }
     }
   } else if (warp == 1 && lane == 0) {
-    const uint32_t idesc = make_idesc_bf16(128, static_cast<uint32_t>(rp), kMN, kMN);
+    const uint32_t idesc = make_idesc_bf16(128, static_cast<uint32_t>(rp), kAMN, kBMN);
     for (int l = 0; l < n_local; ++l) {
       const int st = l % S;
       const uint32_t ph = (l / S) & 1;
@@ -678,14 +689,10 @@ __global__ void __launch_bounds__(128, 1)
       const uint32_t bb = smem_u32(b_tile(st));
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        uint64_t da, db;
-        if (!kMN) {
-          da = make_sdesc_sw128(aa + 32u * kk, 16u, 1024u);
-          db = make_sdesc_sw128(bb + 32u * kk, 16u, 1024u);
-        } else {
-          da = make_sdesc_sw128(aa + 2048u * kk, 8192u, 1024u);
-          db = make_sdesc_sw128(bb + 2048u * kk, 8192u, 1024u);
-        }
+        const uint64_t da = kAMN ? make_sdesc_sw128(aa + 2048u * kk, 8192u, 1024u)
+                                 : make_sdesc_sw128(aa + 32u * kk, 16u, 1024u);
+        const uint64_t db = kBMN ? make_sdesc_sw128(bb + 2048u * kk, 8192u, 1024u)
+                                 : make_sdesc_sw128(bb + 32u * kk, 16u, 1024u);
         umma_bf16(tmem_base, da, db, idesc, (l > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(&empty_bar[st]);
@@ -835,8 +842,9 @@ static int plan_splits(int64_t tiles, int steps, int min_steps, int slots_per_sm
 // Low-rank GEMMs are bound by reading their activation operand once: about one
 // CTA per SM, each streaming at least 8 K steps, keeps per-CTA fixed costs
 // (barrier set-up, TMEM allocation, the fp32 partial write) small.
-static int plan_thin_splits(int64_t tiles, int steps) {
-  int64_t s = tiles > 0 ? kSms / tiles : 1;
+static int plan_thin_splits(int64_t tiles, int steps, int rp) {
+  const int64_t slots = static_cast<int64_t>(kSms) * (rp <= 64 ? 2 : 1);
+  int64_t s = tiles > 0 ? slots / tiles : 1;
   if (s < 1) s = 1;
   const int64_t cap = steps / 8 > 1 ? steps / 8 : 1;
   if (s > cap) s = cap;
@@ -865,7 +873,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
   Plan pl{};
   const int rp = qlora_rank_pad(r);
   const int64_t mt = ceil_div(M, 128);
-  pl.splits_T = plan_thin_splits(mt, static_cast<int>(k / 64));
+  pl.splits_T = plan_thin_splits(mt, static_cast<int>(k / 64), rp);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t o = off;
@@ -886,13 +894,13 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
   } else {
     pl.nt = 0;
     const int dsteps = static_cast<int>(ceil_div(d, 64));
-    pl.splits_U = plan_thin_splits(mt, dsteps);
+    pl.splits_U = plan_thin_splits(mt, dsteps, rp);
     pl.off_Bt = take(static_cast<size_t>(rp) * d * 2);
     pl.off_U = take(static_cast<size_t>(M) * rp * 2);
     pl.off_partU = take(static_cast<size_t>(pl.splits_U) * M * rp * 4);
     const int msteps = static_cast<int>(ceil_div(M, 64));
-    pl.splits_dA = plan_thin_splits(ceil_div(k, 128), msteps);
-    pl.splits_dB = plan_thin_splits(ceil_div(d, 128), msteps);
+    pl.splits_dA = plan_thin_splits(ceil_div(k, 128), msteps, rp);
+    pl.splits_dB = plan_thin_splits(ceil_div(d, 128), msteps, rp);
     pl.off_partA = take(static_cast<size_t>(pl.splits_dA) * k * rp * 4);
     pl.off_partB = take(static_cast<size_t>(pl.splits_dB) * d * rp * 4);
     pl.main_splits = plan_splits(ceil_div(k, 256) * ceil_div(M, 256), dsteps, 8, 1);
@@ -910,9 +918,23 @@ size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
   return make_plan(M, d, k, r, true, true).total;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device (the attribute
+// call costs host time on every launch otherwise).
+// The cache is keyed by the kernel's address: instantiations of one kernel
+// template share a function type but each needs its own attribute.
 template <typename K>
 static cudaError_t set_smem(K kernel, uint32_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, uint32_t> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
 }
 
 static int grid1d(int64_t work, int per_block) {
@@ -932,11 +954,15 @@ static int grid1d(int64_t work, int per_block) {
   } while (0)
 
 // T_s = BF16(s X A^T) (or U_s = BF16(s dY B) with `act` = dY and `bmat` = B^T)
+// b_mn = false: bmat is (brows x K) row-major, read K-major (A of the layer).
+// b_mn = true : bmat is (K x brows) row-major, read MN-major (B of the layer,
+//               K = d, N = r), which needs brows * 2 bytes to be a multiple of 16.
 static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uint16_t* bmat, int64_t brows,
-                            int rp, float s, int splits, float* partial, uint16_t* out, cudaStream_t st,
+                            bool b_mn, int rp, float s, int splits, float* partial, uint16_t* out, cudaStream_t st,
                             const char** why) {
   CUtensorMap ta, tb;
-  if (!map_bf16(&ta, act, K, M, 64, 128) || !map_bf16(&tb, bmat, K, brows, 64, rp)) {
+  const bool okb = b_mn ? map_bf16(&tb, bmat, brows, K, 64, 64) : map_bf16(&tb, bmat, K, brows, 64, rp);
+  if (!map_bf16(&ta, act, K, M, 64, 128) || !okb) {
     *why = "tensor map encoding failed (thin GEMM)";
     return QLORA_ERR_CUDA;
   }
@@ -947,14 +973,18 @@ static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uin
   tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, splits));
   tp.partial = partial;
   const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-  if (set_smem(k_thin<false>, ThinCfg<false>::kSmemBytes) != cudaSuccess) {
+  const uint32_t smem = ThinCfg::smem_bytes(rp);
+  if ((b_mn ? set_smem(k_thin<false, true>, smem) : set_smem(k_thin<false, false>, smem)) != cudaSuccess) {
     *why = "smem attribute";
     return QLORA_ERR_CUDA;
   }
   dim3 grid(static_cast<unsigned>(ceil_div(M, 128)), static_cast<unsigned>(real));
   {
     ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    k_thin<false><<<grid, 128, ThinCfg<false>::kSmemBytes, st>>>(ta, tb, tp);
+    if (b_mn)
+      k_thin<false, true><<<grid, 128, smem, st>>>(ta, tb, tp);
+    else
+      k_thin<false, false><<<grid, 128, smem, st>>>(ta, tb, tp);
   }
   QL_CHECK_LAUNCH("thin GEMM launch");
   const int64_t count = M * rp;
@@ -1000,7 +1030,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   char* ws = static_cast<char*>(a.ws);
   uint16_t* T = own_T ? reinterpret_cast<uint16_t*>(ws + pl.off_T) : a.T;
   float* partT = reinterpret_cast<float*>(ws + pl.off_partT);
-  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, rp, a.s, pl.splits_T, partT, T, st, why);
+  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, a.s, pl.splits_T, partT, T, st, why);
   if (rc) return rc;
 
   const qlora_nf4_t& q = *a.q;
@@ -1074,22 +1104,29 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   const uint16_t* T = a.Tin;
   if (!T) {
     uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + pl.off_T);
-    rc = run_lowrank_down(a.X, M, k, a.A, r, rp, a.s, pl.splits_T, reinterpret_cast<float*>(ws + pl.off_partT), Tw,
-                          st, why);
+    rc = run_lowrank_down(a.X, M, k, a.A, r, false, rp, a.s, pl.splits_T, reinterpret_cast<float*>(ws + pl.off_partT),
+                          Tw, st, why);
     if (rc) return rc;
     T = Tw;
   }
-  // U_s = BF16(s dY B) through B^T (rp x d, K-major)
-  uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
-  {
-    ProfScope ps_(QLORA_KC_AUX, st);
-    k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
-      a.B, d, r, rp, Bt);
-  }
-  QL_CHECK_LAUNCH("transpose launch");
+  // U_s = BF16(s dY B).  B (d x r) is read as an MN-major operand straight from
+  // its row-major storage when its rows are 16-byte multiples; otherwise a
+  // K-major copy B^T (rp x d) is made first.
   uint16_t* U = reinterpret_cast<uint16_t*>(ws + pl.off_U);
-  rc = run_lowrank_down(a.dY, M, d, Bt, rp, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU), U,
-                        st, why);
+  if (r % 8 == 0) {
+    rc = run_lowrank_down(a.dY, M, d, a.B, r, true, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU),
+                          U, st, why);
+  } else {
+    uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
+    {
+      ProfScope ps_(QLORA_KC_AUX, st);
+      k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
+          a.B, d, r, rp, Bt);
+    }
+    QL_CHECK_LAUNCH("transpose launch");
+    rc = run_lowrank_down(a.dY, M, d, Bt, rp, false, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU),
+                          U, st, why);
+  }
   if (rc) return rc;
 
   // dX = dY W + U_s A
@@ -1141,14 +1178,14 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dA));
     tp.partial = reinterpret_cast<float*>(ws + pl.off_partA);
     const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-    if (set_smem(k_thin<true>, ThinCfg<true>::kSmemBytes) != cudaSuccess) {
+    if (set_smem(k_thin<true, true>, ThinCfg::smem_bytes(rp)) != cudaSuccess) {
       *why = "smem attribute (thin MN)";
       return QLORA_ERR_CUDA;
     }
     {
       ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-      k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
-                   ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+      k_thin<true, true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
+                           ThinCfg::smem_bytes(rp), st>>>(ta, tb, tp);
     }
     QL_CHECK_LAUNCH("dA GEMM launch");
     {
@@ -1173,8 +1210,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
     {
       ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-      k_thin<true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
-                   ThinCfg<true>::kSmemBytes, st>>>(ta, tb, tp);
+      k_thin<true, true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
+                           ThinCfg::smem_bytes(rp), st>>>(ta, tb, tp);
     }
     QL_CHECK_LAUNCH("dB GEMM launch");
     {
