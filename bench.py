@@ -405,6 +405,115 @@ def run_reference(args, work, wl_name):
     print(json.dumps(result), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# secondary workloads (not the default line): decode-like forward and the
+# quantisation sweep, each timed kernel by kernel with L2 flushed in between
+# ---------------------------------------------------------------------------
+def _timed(fn, iters, flush, stream):
+    """Median device ms of fn() over `iters` runs; `flush` (outside the
+    events) evicts L2 before each run."""
+    import torch
+    times = []
+    for _ in range(iters):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def run_secondary(args, wl_name):
+    import torch
+
+    import bit_quantized_lora_02_b200 as Q
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    peaks, src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    flush_buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.zero_()
+
+    def dev_bits(a):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    results = []
+    iters = max(args.steps, 5)
+    if wl_name == "decode_28672x8192":
+        work = synth.WORKLOADS[wl_name]
+        r, alpha = work["r"], work["alpha"]
+        for pi, (name, d, k) in enumerate(work["proj"]):
+            W = dev_bits(synth.weight(d, k, seed=pi))
+            q = Q.nf4_quantize(W, True)
+            del W
+            A, B = dev_bits(synth.lora_a(r, k, seed=pi)), dev_bits(synth.lora_b(d, r, seed=pi))
+            for M in work["m"]:
+                X = dev_bits(synth.activations(M, k, seed=pi))
+                Y = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
+                T = torch.empty(M, Q.qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
+                ws = torch.empty(max(Q.qlora_linear_workspace_size(M, d, k, r, False), 16), dtype=torch.uint8,
+                                 device=dev)
+                fn = lambda: Q.qlora_linear_fwd(X, q, A, B, alpha, Y=Y, T_save=T, workspace=ws, stream=stream)  # noqa: E731
+                for _ in range(args.warmup):
+                    fn()
+                Q.qlora_profile_read()
+                Q.qlora_profile_enable(True)
+                ms = _timed(fn, iters, flush, stream)
+                Q.qlora_profile_enable(False)
+                kms, kn = Q.qlora_profile_read()
+                nf4 = nf4_bytes(d, k)
+                act = 2 * (M * k + M * d + r * k + d * r)
+                fl = flops_fwd(M, d, k, r)
+                main_ms = kms["fwd_gemm"] / max(kn["fwd_gemm"], 1)
+                results.append({"proj": f"{name}:{d}x{k}", "M": M, "ms": round(ms, 4),
+                                "nf4_weight_gbs": round(nf4 / (ms * 1e-3) / 1e9, 1),
+                                "nf4_weight_frac_hbm": round(nf4 / (ms * 1e-3) / 1e9 / hbm, 4),
+                                "bytes_gbs": round((nf4 + act) / (ms * 1e-3) / 1e9, 1),
+                                "tflops": round(fl / (ms * 1e-3) / 1e12, 2),
+                                "main_kernel_ms": round(main_ms, 4),
+                                "main_kernel_nf4_gbs": round(nf4 / (main_ms * 1e-3) / 1e9, 1) if main_ms else None,
+                                "launches": int(sum(kn.values())) // iters})
+        metric, unit = "QLoRA decode-like forward NF4-weight GB/s (M in 1,8,32,128)", "GB/s"
+        value = statistics.median([x["nf4_weight_gbs"] for x in results if x["M"] <= 32])
+    elif wl_name == "quant_sweep":
+        for pi, (name, d, k) in enumerate(synth.WORKLOADS[wl_name]["proj"]):
+            W = dev_bits(synth.weight(d, k, seed=pi, outliers=True))
+            n = d * k
+            nblk = -(-n // 64)
+            for dq in (True, False):
+                q = Q.nf4_alloc(d, k, dq, dev)
+                wsz = Q.qlora_nf4_sizes(d, k, 64, dq)[1]
+                qws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
+                out = torch.empty(d, k, dtype=torch.bfloat16, device=dev)
+                fq = lambda: Q.nf4_quantize(W, dq, out=q, workspace=qws, stream=stream)  # noqa: E731
+                fd = lambda: Q.nf4_dequantize(q, out=out, stream=stream)  # noqa: E731
+                for _ in range(args.warmup):
+                    fq()
+                    fd()
+                mq = _timed(fq, iters, flush, stream)
+                md = _timed(fd, iters, flush, stream)
+                consts = (nblk + 4 * (-(-nblk // 256)) + 4) if dq else 4 * nblk
+                qbytes = 2 * n + (n + 1) // 2 + consts + (2 * nblk * 2 if dq else 0)   # + bf16 scale scratch write/read
+                dbytes = (n + 1) // 2 + consts + 2 * n
+                results.append({"proj": f"{name}:{d}x{k}", "double_quant": dq,
+                                "quantize_ms": round(mq, 4), "quantize_gbs": round(qbytes / (mq * 1e-3) / 1e9, 1),
+                                "quantize_frac_hbm": round(qbytes / (mq * 1e-3) / 1e9 / hbm, 4),
+                                "dequantize_ms": round(md, 4), "dequantize_gbs": round(dbytes / (md * 1e-3) / 1e9, 1),
+                                "dequantize_frac_hbm": round(dbytes / (md * 1e-3) / 1e9 / hbm, 4)})
+        metric, unit = "NF4 quantize GB/s (4096x11008, double quant)", "GB/s"
+        value = [x for x in results if x["proj"].startswith("rect") and x["double_quant"]][0]["quantize_gbs"]
+    else:
+        raise SystemExit(f"unknown secondary workload {wl_name}")
+    print(json.dumps({"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "workload": wl_name,
+                      "hbm_peak_gbs": hbm, "peak_source": src, "l2": "flushed (512 MB write) before every run",
+                      "iters": iters, "results": results}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -412,11 +521,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b_proj_set_m4096",
-                    choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512"))
+                    choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512",
+                             "decode_28672x8192", "quant_sweep"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    if args.workload in ("decode_28672x8192", "quant_sweep"):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "secondary workloads are measured for this arm only"}))
+            return
+        run_secondary(args, args.workload)
+        return
     work = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         run_reference(args, work, args.workload)
