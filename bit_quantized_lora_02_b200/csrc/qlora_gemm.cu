@@ -216,12 +216,17 @@ template <Mode MODE, int NT>
 struct MainCfg {
   static constexpr bool kSwap = MODE == Mode::FwdSwap;
   static constexpr bool kBwd = MODE == Mode::Bwd;
+  // K width of one pipeline step: two NF4 blocks per weight row for the
+  // swapped (few-token) forward, one otherwise.  A step always holds 256 NF4
+  // blocks, one per thread of a dequant group.
+  static constexpr int kStepK = kSwap ? 128 : 64;
   static constexpr int kWRows = kSwap ? 128 : (kBwd ? 64 : 256);      // W rows per K step
-  static constexpr int kWCols = kBwd ? 256 : 64;                       // W columns per K step
+  static constexpr int kWCols = kBwd ? 256 : kStepK;                   // W columns per K step
   static constexpr int kActRows = kSwap ? NT : 256;                    // token rows per K step
   static constexpr int kAccs = kSwap ? 1 : 2;                          // M=128 accumulators per tile
   static constexpr int kMmaN = kSwap ? NT : 256;
-  static constexpr uint32_t kActBytes = kActRows * 128;
+  static constexpr uint32_t kActAtomBytes = kActRows * 128;            // one 64-wide K atom of the activations
+  static constexpr uint32_t kActBytes = kActAtomBytes * (kStepK / 64);
   static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
   static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
   static constexpr uint32_t kStageBytes = kActBytes + kWBytes + kCodeBytes;
@@ -231,6 +236,14 @@ struct MainCfg {
       kSwap ? (kMmaN <= 32 ? 32u : (kMmaN <= 64 ? 64u : 128u)) : 512u;   // two 128x256 fp32 accumulators
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr int kDeqThreads = 512;     // 16 dequant warps (warps 2..17)
+  // Few tokens (swap): two groups of 8 warps take alternate steps and every
+  // thread expands a whole block (the dequant rate is what matters there).
+  // Many tokens: all 16 warps work on every step, two threads per block, which
+  // keeps the per-step latency short enough to feed the tensor core.
+  static constexpr int kGroups = kSwap ? 2 : 1;
+  static constexpr int kGroupThreads = kDeqThreads / kGroups;
+  static constexpr int kTPB = kGroupThreads / 256;    // threads per NF4 block
+  static constexpr int kCPT = 8 / kTPB;               // 16-byte chunks per thread
   static constexpr int kThreads = 64 + kDeqThreads;
   static constexpr uint32_t kIdesc = make_idesc_bf16(128, kMmaN, false, kBwd);
 };
@@ -247,7 +260,7 @@ __global__ void __launch_bounds__(576, 1)
   uint8_t* base = smem_raw + (base_addr - raw_addr);
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
   uint64_t* full_bar = bars;            // TMA data landed (act + codes)
-  uint64_t* deq_bar = bars + S;         // dequant warps finished the W tile
+  uint64_t* deq_bar = bars + S;         // a dequant group finished the W tile
   uint64_t* empty_bar = bars + 2 * S;   // MMAs reading the stage completed
   uint64_t* tmem_full = bars + 3 * S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
@@ -273,7 +286,7 @@ __global__ void __launch_bounds__(576, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&deq_bar[i], 16);
+      mbar_init(&deq_bar[i], Cfg::kGroupThreads / 32);
       mbar_init(&empty_bar[i], 1);
     }
     mbar_init(tmem_full, 1);
@@ -308,8 +321,9 @@ __global__ void __launch_bounds__(576, 1)
           const int i = s_begin + l;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes + Cfg::kCodeBytes);
           if (Cfg::kSwap) {
-            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, 0);
-            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(n0));
+            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 128 * i, 0);
+            tma_load_2d(act_tile(st) + Cfg::kActAtomBytes, &tm_act, &full_bar[st], 128 * i + 64, 0);
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 64 * i, static_cast<int>(n0));
           } else if (Cfg::kBwd) {
             tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
             tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], static_cast<int>(n0 / 2), 64 * i);
@@ -319,7 +333,7 @@ __global__ void __launch_bounds__(576, 1)
           }
         } else {
           const int e = l - n_main;
-          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes);
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActAtomBytes);
           tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, Cfg::kSwap ? 0 : static_cast<int>(m0));
         }
         ++issued;
@@ -338,8 +352,7 @@ __global__ void __launch_bounds__(576, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      int l = 0;
-      for (; l < n_local; ++l) {
+      for (int l = 0; l < n_local; ++l) {
         const int st = l % S;
         const uint32_t ph = (l / S) & 1;
         if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
@@ -347,42 +360,43 @@ __global__ void __launch_bounds__(576, 1)
         tc_fence_after();
         const uint32_t a_act = smem_u32(act_tile(st));
         const uint32_t a_w = smem_u32(w_tile(st));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
+        const int slices = (l < n_main) ? Cfg::kStepK / 16 : 4;   // LoRA steps are 64 wide
+        for (int kk = 0; kk < slices; ++kk) {
+          const uint32_t atom = static_cast<uint32_t>(kk >> 2), kq = static_cast<uint32_t>(kk & 3);
           uint64_t da, db;
-          const uint64_t d_act = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
           if (Cfg::kSwap) {
-            da = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
-            db = d_act;
+            da = make_sdesc_sw128(a_w + 16384u * atom + 32u * kq, 16u, 1024u);
+            db = make_sdesc_sw128(a_act + Cfg::kActAtomBytes * atom + 32u * kq, 16u, 1024u);
           } else if (Cfg::kBwd) {
-            da = d_act;
+            da = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
             db = make_sdesc_sw128(a_w + 2048u * kk, 8192u, 1024u);
           } else {
-            da = d_act;
+            da = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
             db = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
           }
-          umma_bf16(tmem_base, da, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t acc = (l > 0 || kk > 0) ? 1u : 0u;
+          umma_bf16(tmem_base, da, db, Cfg::kIdesc, acc);
           if (Cfg::kAccs == 2) {
             // token rows 128..255 of the tile share the same W tile: second accumulator
             const uint64_t da1 = make_sdesc_sw128(a_act + 16384u + 32u * kk, 16u, 1024u);
-            umma_bf16(tmem_base + 256u, da1, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(tmem_base + 256u, da1, db, Cfg::kIdesc, acc);
           }
         }
         umma_commit(&empty_bar[st]);
       }
       umma_commit(tmem_full);   // also drains MMAs on the abort path
     }
-  } else if (warp >= 2) {
+  } else {
     // ------------------------------------------------------------ dequant warps
-    // 16 warps; each NF4 block of the tile is shared by kTPB threads, each
-    // expanding kCPT 16-byte chunks (8 weights each) of the block's 128-byte row.
-    constexpr int kBlocks = Cfg::kWRows * Cfg::kWCols / 64;   // blocks per K step: 256 (Fwd, Bwd), 128 (Swap)
-    constexpr int kTPB = Cfg::kDeqThreads / kBlocks;
-    constexpr int kCPT = 8 / kTPB;
-    const int t = threadIdx.x - 64;   // 0..511
-    const int blk_id = t / kTPB;
-    const int part = t % kTPB;
-    const int c_first = part * kCPT;
+    // kGroups groups take alternate K steps; a step's 256 NF4 blocks are
+    // spread over the group's threads, kTPB threads per block, each expanding
+    // kCPT 16-byte chunks (8 weights each) of the block's 128-byte row.
+    constexpr int G = Cfg::kGroups, TPB = Cfg::kTPB, CPT = Cfg::kCPT;
+    const int t = threadIdx.x - 64;            // 0..511
+    const int grp = t / Cfg::kGroupThreads;
+    const int tgt = t % Cfg::kGroupThreads;
+    const int tg = tgt / TPB;                  // block of the step
+    const int c_first = (tgt % TPB) * CPT;     // first chunk of this thread
     // the codebook as register immediates (no memory traffic)
     constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
     float C[16];
@@ -390,98 +404,104 @@ __global__ void __launch_bounds__(576, 1)
     for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
     const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
-    // this thread's block inside the tile: Fwd/Swap: row = W row; Bwd: row =
-    // W row within the 64-row K step (MN-major K row), sub = 64-column chunk
-    const int row = Cfg::kBwd ? (blk_id & 63) : blk_id;
-    const int sub = Cfg::kBwd ? (blk_id >> 6) : 0;
+    // position of this thread's block in the tile
+    //   Fwd : row = W row (0..255)
+    //   Bwd : row = W row within the 64-row K step (MN-major K row), sub = 64-column chunk
+    //   Swap: row = W row (0..127), sub = which of the step's two blocks
+    const int row = Cfg::kBwd ? (tg & 63) : (Cfg::kSwap ? (tg & 127) : tg);
+    const int sub = Cfg::kBwd ? (tg >> 6) : (Cfg::kSwap ? (tg >> 7) : 0);
+    const uint32_t w_off = Cfg::kBwd ? 8192u * sub : (Cfg::kSwap ? 16384u * sub : 0u);
+    const uint32_t c_off = (Cfg::kBwd ? (row * 128 + sub * 32) : (Cfg::kSwap ? (row * 64 + sub * 32) : (row * 32))) +
+                           4 * c_first;
     auto block_of = [&](int i, bool& valid) -> int64_t {
       int64_t wr, bc;
       if (Cfg::kBwd) {
         wr = 64ll * i + row;
         bc = n0 / 64 + sub;
-        valid = (wr < p.d) && (bc < p.kpb);
+      } else if (Cfg::kSwap) {
+        wr = n0 + row;
+        bc = 2ll * i + sub;
       } else {
         wr = n0 + row;
         bc = i;
-        valid = wr < p.d;
       }
+      valid = (wr < p.d) && (bc < p.kpb);
       return wr * p.kpb + bc;
     };
-    // block constants are fetched two K steps ahead of their use
+    // this group's steps are l = grp, grp + G, ...; block constants are
+    // fetched two of its own steps ahead
     ScaleRaw pre0{}, pre1{};
     bool pre0_valid = false, pre1_valid = false;
-    if (n_main > 0) {
-      const int64_t b0 = block_of(s_begin, pre0_valid);
+    if (grp < n_main) {
+      const int64_t b0 = block_of(s_begin + grp, pre0_valid);
       if (pre0_valid) pre0 = scale_fetch(sc, b0);
     }
-    if (n_main > 1) {
-      const int64_t b1 = block_of(s_begin + 1, pre1_valid);
+    if (grp + G < n_main) {
+      const int64_t b1 = block_of(s_begin + grp + G, pre1_valid);
       if (pre1_valid) pre1 = scale_fetch(sc, b1);
     }
-    for (int l = 0; l < n_local; ++l) {
+    for (int l = grp; l < n_local; l += G) {
       const int st = l % S;
       const uint32_t ph = (l / S) & 1;
       bool okw = mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
       okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
       if (!__all_sync(0xffffffffu, okw)) break;
-      const uint32_t wt = smem_u32(w_tile(st)) + (Cfg::kBwd ? 8192u * sub : 0u);
+      const uint32_t wt = smem_u32(w_tile(st)) + w_off;
       if (l < n_main) {
         const ScaleRaw cur = pre0;
         const bool cur_valid = pre0_valid;
         pre0 = pre1;
         pre0_valid = pre1_valid;
-        if (l + 2 < n_main) {
-          const int64_t bn = block_of(s_begin + l + 2, pre1_valid);
+        if (l + 2 * G < n_main) {
+          const int64_t bn = block_of(s_begin + l + 2 * G, pre1_valid);
           if (pre1_valid) pre1 = scale_fetch(sc, bn);
         }
-        // codes of this thread's chunks: 4 bytes per chunk
-        const uint32_t src = smem_u32(code_tile(st)) + (Cfg::kBwd ? (row * 128 + sub * 32) : (row * 32)) + 4 * c_first;
-        uint32_t w[kCPT];
-        if constexpr (kCPT == 4) {
-          const uint4 cw = lds128(src);
-          w[0] = cw.x;
-          w[1] = cw.y;
-          w[2] = cw.z;
-          w[3] = cw.w;
-        } else {
+        const uint32_t src = smem_u32(code_tile(st)) + c_off;
+        uint32_t w8[CPT];
 #pragma unroll
-          for (int c = 0; c < kCPT; ++c) w[c] = lds32(src + 4 * c);
+        for (int h = 0; h < CPT / 4; ++h) {
+          const uint4 cw = lds128(src + 16 * h);
+          w8[4 * h] = cw.x;
+          w8[4 * h + 1] = cw.y;
+          w8[4 * h + 2] = cw.z;
+          w8[4 * h + 3] = cw.w;
         }
         if (cur_valid) {
           const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
 #pragma unroll
-          for (int c = 0; c < kCPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w[c], tab));
+          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w8[c], tab));
         } else {
 #pragma unroll
-          for (int c = 0; c < kCPT; ++c) sts128(wt + sw128_offset(row, c_first + c), make_uint4(0, 0, 0, 0));
+          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), make_uint4(0, 0, 0, 0));
         }
       } else {
-        // LoRA extension step: copy 64 columns of the adapter into the W tile
+        // LoRA extension step (64 wide): copy 64 columns of the adapter into the W tile
         const int e = l - n_main;
         if (Cfg::kBwd) {
           // A (r x k): K row j = 64e + row, N columns n0 + 64 sub + [0, 64)
           const int64_t j = 64ll * e + row;
           const int64_t col = n0 + 64 * sub;
           const bool v = (j < p.r) && (col < p.k);
-          const uint16_t* src = p.lora + j * p.k + col;
+          const uint16_t* srcp = p.lora + j * p.k + col;
 #pragma unroll
-          for (int c = 0; c < kCPT; ++c) {
+          for (int c = c_first; c < c_first + CPT; ++c) {
             uint4 val = make_uint4(0, 0, 0, 0);
-            if (v) val = __ldg(reinterpret_cast<const uint4*>(src + 8 * (c_first + c)));
-            sts128(wt + sw128_offset(row, c_first + c), val);
+            if (v) val = __ldg(reinterpret_cast<const uint4*>(srcp + 8 * c));
+            sts128(wt + sw128_offset(row, c), val);
           }
-        } else {
-          // B (d x r): row n, columns 64e + 8 (c_first + c) + [0, 8)
+        } else if (!Cfg::kSwap || sub == 0) {
+          // B (d x r): row n, columns 64e + [0, 64) into the first K atom
           const int64_t n = n0 + row;
+          const uint32_t wt0 = smem_u32(w_tile(st));
 #pragma unroll
-          for (int c = 0; c < kCPT; ++c) {
+          for (int c = c_first; c < c_first + CPT; ++c) {
             uint32_t h[8];
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
-              const int64_t j = 64ll * e + 8 * (c_first + c) + q;
+              const int64_t j = 64ll * e + 8 * c + q;
               h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
             }
-            sts128(wt + sw128_offset(row, c_first + c),
+            sts128(wt0 + sw128_offset(row, c),
                    make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
           }
         }
@@ -861,6 +881,25 @@ struct Plan {
   size_t off_T, off_partT, off_Bt, off_U, off_partU, off_partA, off_partB, off_main, total;
 };
 
+// Few-token forward: the kernel streams weights, so keep every SM busy until
+// the end.  Choose the K split (1..8) with the best wave efficiency; a larger
+// split must win by 5% (its partial sums cost an extra pass).
+static int plan_swap_splits(int64_t tiles, int steps) {
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= 8; ++s) {
+    if (steps / s < 4) break;
+    const int64_t ctas = tiles * s;
+    const int64_t waves = ceil_div(ctas, kSms);
+    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kSms);
+    if (eff > best_eff + 0.05) {
+      best_eff = eff;
+      best = s;
+    }
+  }
+  return best;
+}
+
 static int swap_nt(int64_t M) {
   if (M <= 16) return 16;
   if (M <= 32) return 32;
@@ -886,7 +925,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     pl.nt = swap_nt(M);
     const int steps = static_cast<int>(k / 64);
     if (pl.nt) {
-      pl.main_splits = plan_splits(ceil_div(d, 128), steps, 8, 1);
+      pl.main_splits = plan_swap_splits(ceil_div(d, 128), static_cast<int>(ceil_div(k, 128)));
     } else {
       pl.main_splits = plan_splits(ceil_div(d, 256) * ceil_div(M, 256), steps, 8, 1);
     }
@@ -1040,7 +1079,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   mp.sc = scale_src(q);
   mp.lora = a.B;
   mp.n_out = d;
-  mp.steps_main = static_cast<int32_t>(k / 64);
+  mp.steps_main = static_cast<int32_t>(pl.nt ? ceil_div(k, 128) : k / 64);   // the swapped kernel steps 128 wide
   mp.ext_steps = rp / 64;
   mp.steps_per_split = static_cast<int32_t>(ceil_div(mp.steps_main, pl.main_splits));
   mp.splits = static_cast<int32_t>(ceil_div(mp.steps_main, mp.steps_per_split));
@@ -1051,7 +1090,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   bool ok;
   if (nt) {
     ok = map_bf16(&t_act, a.X, k, M, 64, nt) &&
-         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 128, false) &&
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 64, 128, false) &&
          map_bf16(&t_ext, T, rp, M, 64, nt);
   } else {
     ok = map_bf16(&t_act, a.X, k, M, 64, 256) &&
