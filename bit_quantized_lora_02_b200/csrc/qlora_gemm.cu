@@ -73,22 +73,22 @@ static EncodeTiledFn encode_fn() {
 // 2-D row-major tensor: `inner` elements per row (contiguous), `outer` rows,
 // `row_bytes` between rows.  Box = box_inner x box_outer.
 static bool make_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+                     uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 static bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                      uint32_t box_rows) {
-  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows, true);
+  return make_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cols, rows, cols * 2, box_cols, box_rows,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // ============================================================================
@@ -229,12 +229,16 @@ struct MainCfg {
   static constexpr uint32_t kActBytes = kActAtomBytes * (kStepK / 64);
   static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
   static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
-  static constexpr uint32_t kStageBytes = kActBytes + kWBytes + kCodeBytes;
-  static constexpr int kStagesRaw = static_cast<int>((218u * 1024u) / kStageBytes);
-  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // Two rings: TMA stages (activations + packed codes, small) and dequantized
+  // W-tile buffers (large, written by the dequant warps).  Decoupling them lets
+  // many more code tiles be in flight than W tiles.
+  static constexpr uint32_t kStageBytes = kActBytes + kCodeBytes;     // one TMA stage
+  static constexpr int kWBufs = kSwap ? 3 : 2;                         // groups in flight + one for the MMA
+  static constexpr int kStagesRaw = static_cast<int>((218u * 1024u - kWBufs * kWBytes) / kStageBytes);
+  static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   static constexpr uint32_t kTmemCols =
       kSwap ? (kMmaN <= 32 ? 32u : (kMmaN <= 64 ? 64u : 128u)) : 512u;   // two 128x256 fp32 accumulators
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kWBufs * kWBytes + 1024 /*align*/ + 512 /*barriers*/;
   static constexpr int kDeqThreads = 512;     // 16 dequant warps (warps 2..17)
   // Few tokens (swap): two groups of 8 warps take alternate steps and every
   // thread expands a whole block (the dequant rate is what matters there).
@@ -258,13 +262,16 @@ __global__ void __launch_bounds__(576, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
-  uint64_t* full_bar = bars;            // TMA data landed (act + codes)
-  uint64_t* deq_bar = bars + S;         // a dequant group finished the W tile
-  uint64_t* empty_bar = bars + 2 * S;   // MMAs reading the stage completed
-  uint64_t* tmem_full = bars + 3 * S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 2);
+  constexpr int SW = Cfg::kWBufs;
+  uint8_t* wbase = base + S * Cfg::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SW * Cfg::kWBytes);
+  uint64_t* full_bar = bars;                // TMA data landed (act + codes)
+  uint64_t* empty_bar = bars + S;           // MMAs reading the TMA stage completed
+  uint64_t* wready_bar = bars + 2 * S;      // a dequant group filled the W buffer
+  uint64_t* wfree_bar = bars + 2 * S + SW;  // MMAs reading the W buffer completed
+  uint64_t* tmem_full = bars + 2 * S + 2 * SW;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_full + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -286,8 +293,11 @@ __global__ void __launch_bounds__(576, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&deq_bar[i], Cfg::kGroupThreads / 32);
       mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < SW; ++i) {
+      mbar_init(&wready_bar[i], Cfg::kGroupThreads / 32);
+      mbar_init(&wfree_bar[i], 1);
     }
     mbar_init(tmem_full, 1);
     *abort_flag = 0;
@@ -306,8 +316,8 @@ __global__ void __launch_bounds__(576, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
-  auto w_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
-  auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes + Cfg::kWBytes; };
+  auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
+  auto w_tile = [&](int sw) { return wbase + sw * Cfg::kWBytes; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -355,11 +365,13 @@ __global__ void __launch_bounds__(576, 1)
       for (int l = 0; l < n_local; ++l) {
         const int st = l % S;
         const uint32_t ph = (l / S) & 1;
+        const int sw = l % SW;
+        const uint32_t phw = (l / SW) & 1;
         if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
-        if (!mbar_wait(&deq_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
+        if (!mbar_wait(&wready_bar[sw], phw, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
         tc_fence_after();
         const uint32_t a_act = smem_u32(act_tile(st));
-        const uint32_t a_w = smem_u32(w_tile(st));
+        const uint32_t a_w = smem_u32(w_tile(sw));
         const int slices = (l < n_main) ? Cfg::kStepK / 16 : 4;   // LoRA steps are 64 wide
         for (int kk = 0; kk < slices; ++kk) {
           const uint32_t atom = static_cast<uint32_t>(kk >> 2), kq = static_cast<uint32_t>(kk & 3);
@@ -383,6 +395,7 @@ __global__ void __launch_bounds__(576, 1)
           }
         }
         umma_commit(&empty_bar[st]);
+        umma_commit(&wfree_bar[sw]);
       }
       umma_commit(tmem_full);   // also drains MMAs on the abort path
     }
@@ -411,8 +424,13 @@ __global__ void __launch_bounds__(576, 1)
     const int row = Cfg::kBwd ? (tg & 63) : (Cfg::kSwap ? (tg & 127) : tg);
     const int sub = Cfg::kBwd ? (tg >> 6) : (Cfg::kSwap ? (tg >> 7) : 0);
     const uint32_t w_off = Cfg::kBwd ? 8192u * sub : (Cfg::kSwap ? 16384u * sub : 0u);
-    const uint32_t c_off = (Cfg::kBwd ? (row * 128 + sub * 32) : (Cfg::kSwap ? (row * 64 + sub * 32) : (row * 32))) +
-                           4 * c_first;
+    // Code tile rows: 32 B (Fwd, plain), 64 B (Swap, TMA 64-byte swizzle: 16-byte
+    // chunk j of row r sits at j ^ ((r >> 1) & 3)), 128 B (Bwd, 128-byte swizzle:
+    // j ^ (r & 7)).  The swizzles spread a quarter-warp's reads over all banks.
+    constexpr uint32_t kCodeRow = Cfg::kBwd ? 128u : (Cfg::kSwap ? 64u : 32u);
+    const uint32_t c_row = row * kCodeRow;
+    const uint32_t lc0 = (Cfg::kBwd || Cfg::kSwap ? 2u * sub : 0u) + static_cast<uint32_t>(c_first / 4);
+    const uint32_t c_xor = Cfg::kBwd ? (row & 7u) : (Cfg::kSwap ? ((row >> 1) & 3u) : 0u);
     auto block_of = [&](int i, bool& valid) -> int64_t {
       int64_t wr, bc;
       if (Cfg::kBwd) {
@@ -443,10 +461,12 @@ __global__ void __launch_bounds__(576, 1)
     for (int l = grp; l < n_local; l += G) {
       const int st = l % S;
       const uint32_t ph = (l / S) & 1;
-      bool okw = mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
+      const int sw = l % SW;
+      const uint32_t phw = (l / SW) & 1;
+      bool okw = mbar_wait(&wfree_bar[sw], phw ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
       okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
       if (!__all_sync(0xffffffffu, okw)) break;
-      const uint32_t wt = smem_u32(w_tile(st)) + w_off;
+      const uint32_t wt = smem_u32(w_tile(sw)) + w_off;
       if (l < n_main) {
         const ScaleRaw cur = pre0;
         const bool cur_valid = pre0_valid;
@@ -456,11 +476,11 @@ __global__ void __launch_bounds__(576, 1)
           const int64_t bn = block_of(s_begin + l + 2 * G, pre1_valid);
           if (pre1_valid) pre1 = scale_fetch(sc, bn);
         }
-        const uint32_t src = smem_u32(code_tile(st)) + c_off;
+        const uint32_t ctile = smem_u32(code_tile(st)) + c_row;
         uint32_t w8[CPT];
 #pragma unroll
         for (int h = 0; h < CPT / 4; ++h) {
-          const uint4 cw = lds128(src + 16 * h);
+          const uint4 cw = lds128(ctile + 16u * ((lc0 + h) ^ c_xor));
           w8[4 * h] = cw.x;
           w8[4 * h + 1] = cw.y;
           w8[4 * h + 2] = cw.z;
@@ -492,7 +512,7 @@ __global__ void __launch_bounds__(576, 1)
         } else if (!Cfg::kSwap || sub == 0) {
           // B (d x r): row n, columns 64e + [0, 64) into the first K atom
           const int64_t n = n0 + row;
-          const uint32_t wt0 = smem_u32(w_tile(st));
+          const uint32_t wt0 = smem_u32(w_tile(sw));
 #pragma unroll
           for (int c = c_first; c < c_first + CPT; ++c) {
             uint32_t h[8];
@@ -508,7 +528,7 @@ __global__ void __launch_bounds__(576, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&deq_bar[st]);
+      if (lane == 0) mbar_arrive(&wready_bar[sw]);
     }
 
     // ------------------------------------------------------------ epilogue
@@ -1090,11 +1110,13 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   bool ok;
   if (nt) {
     ok = map_bf16(&t_act, a.X, k, M, 64, nt) &&
-         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 64, 128, false) &&
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 64, 128,
+                  CU_TENSOR_MAP_SWIZZLE_64B) &&
          map_bf16(&t_ext, T, rp, M, 64, nt);
   } else {
     ok = map_bf16(&t_act, a.X, k, M, 64, 256) &&
-         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 256, false) &&
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 256,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
          map_bf16(&t_ext, T, rp, M, 64, 256);
   }
   if (!ok) {
@@ -1184,7 +1206,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     mp.partial = reinterpret_cast<float*>(ws + pl.off_main);
     CUtensorMap t_act, t_codes, t_ext;
     if (!map_bf16(&t_act, a.dY, d, M, 64, 256) ||
-        !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 64, false) ||
+        !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 64,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map_bf16(&t_ext, U, rp, M, 64, 256)) {
       *why = "tensor map encoding failed (backward)";
       return QLORA_ERR_CUDA;
