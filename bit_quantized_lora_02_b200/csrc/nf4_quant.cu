@@ -143,14 +143,6 @@ void quant_thresholds(float out[15]) {
 // ----------------------------------------------------------------------------
 // Quantisation kernel
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-
 // xn = RN32(w / s).  For a block scale in [2^-60, 2^60] this uses the
 // correctly rounded reciprocal r = RN32(1/s) and one residual correction
 // (Markstein's final division step: y = RN(w r); e = fma(-s, y, w);

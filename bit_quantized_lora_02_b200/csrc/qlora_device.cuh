@@ -24,6 +24,7 @@ enum DeviceError : int {
   DEV_WAIT_TIMEOUT_MMA = 3,      // MMA completion never signalled
   DEV_WAIT_TIMEOUT_EPILOGUE = 4,
   DEV_WAIT_TIMEOUT_DRAIN = 5,
+  DEV_SMEM_LAYOUT = 6,           // the shared-memory window could not hold a kernel's layout
 };
 
 extern __device__ int g_status;
@@ -203,6 +204,15 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 // ----------------------------------------------------------------------------
 // Small helpers
 // ----------------------------------------------------------------------------
+// 16-byte read-only global load (non-coherent path; data the kernel never writes)
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));

@@ -42,6 +42,7 @@
 #include <mutex>
 #include <utility>
 
+#include "nf4_scale.cuh"
 #include "nf4_table.h"
 #include "qlora_device.cuh"
 #include "qlora_internal.h"
@@ -161,37 +162,6 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
-// Block scale s^ for NF4 block `blk`.
-struct ScaleSrc {
-  const float* absmax;   // DQ off
-  const int8_t* c2;      // DQ on
-  const float* c1;
-  const float* mean;     // device scalar, DQ on
-  int dq;
-};
-
-struct ScaleRaw {
-  float a;   // absmax (DQ off) or c1 (DQ on)
-  int b;     // c2
-};
-
-__device__ __forceinline__ ScaleRaw scale_fetch(const ScaleSrc& s, int64_t blk) {
-  ScaleRaw r;
-  if (s.dq) {
-    r.b = __ldg(s.c2 + blk);
-    r.a = __ldg(s.c1 + (blk >> 8));
-  } else {
-    r.a = __ldg(s.absmax + blk);
-    r.b = 0;
-  }
-  return r;
-}
-
-// s^ = RN32(RN32(c2 / c1) + mean) with DQ, else the stored absmax.
-__device__ __forceinline__ float scale_value(int dq, float mean, ScaleRaw r) {
-  return dq ? __fadd_rn(__fdiv_rn(static_cast<float>(r.b), r.a), mean) : r.a;
-}
-
 // ============================================================================
 // Main fused kernel
 // ============================================================================
@@ -233,7 +203,7 @@ struct MainCfg {
   // W-tile buffers (large, written by the dequant warps).  Decoupling them lets
   // many more code tiles be in flight than W tiles.
   static constexpr uint32_t kStageBytes = kActBytes + kCodeBytes;     // one TMA stage
-  static constexpr int kWBufs = kSwap ? 3 : 2;                         // groups in flight + one for the MMA
+  static constexpr int kWBufs = 3;   // W tiles being written or waiting + one the MMAs read
   static constexpr int kStagesRaw = static_cast<int>((218u * 1024u - kWBufs * kWBytes) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
   static constexpr uint32_t kTmemCols =
@@ -449,6 +419,7 @@ __global__ void __launch_bounds__(576, 1)
     // this group's steps are l = grp, grp + G, ...; block constants are
     // fetched two of its own steps ahead
     ScaleRaw pre0{}, pre1{};
+    ScaleRecip recip;
     bool pre0_valid = false, pre1_valid = false;
     if (grp < n_main) {
       const int64_t b0 = block_of(s_begin + grp, pre0_valid);
@@ -487,7 +458,7 @@ __global__ void __launch_bounds__(576, 1)
           w8[4 * h + 3] = cw.w;
         }
         if (cur_valid) {
-          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur), C);
+          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur, recip), C);
 #pragma unroll
           for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w8[c], tab));
         } else {
@@ -897,6 +868,7 @@ struct Plan {
   // main
   int main_splits;
   int nt;   // swap token tile (0 = non-swap)
+  bool fewtok;   // forward through the few-token kernels
   // workspace offsets (bytes)
   size_t off_T, off_partT, off_Bt, off_U, off_partU, off_partA, off_partB, off_main, total;
 };
@@ -941,7 +913,10 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
   };
   pl.off_T = need_T ? take(static_cast<size_t>(M) * rp * 2) : 0;
   pl.off_partT = need_T ? take(static_cast<size_t>(pl.splits_T) * M * rp * 4) : 0;
-  if (!bwd) {
+  if (!bwd && fewtok_eligible(M, d, k)) {
+    pl.fewtok = true;
+    pl.off_main = take(fewtok_workspace_bytes(M, d, k));
+  } else if (!bwd) {
     pl.nt = swap_nt(M);
     const int steps = static_cast<int>(k / 64);
     if (pl.nt) {
@@ -975,25 +950,6 @@ size_t fwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
 }
 size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
   return make_plan(M, d, k, r, true, true).total;
-}
-
-// Raise a kernel's dynamic shared-memory limit once per device (the attribute
-// call costs host time on every launch otherwise).
-// The cache is keyed by the kernel's address: instantiations of one kernel
-// template share a function type but each needs its own attribute.
-template <typename K>
-static cudaError_t set_smem(K kernel, uint32_t bytes) {
-  static std::mutex mu;
-  static std::map<std::pair<const void*, int>, uint32_t> done;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
-  std::lock_guard<std::mutex> lk(mu);
-  auto it = done.find(key);
-  if (it != done.end() && it->second >= bytes) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
-  if (e == cudaSuccess) done[key] = bytes;
-  return e;
 }
 
 static int grid1d(int64_t work, int per_block) {
@@ -1088,6 +1044,15 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   Plan pl = make_plan(M, d, k, a.r, false, true);
   char* ws = static_cast<char*>(a.ws);
   uint16_t* T = own_T ? reinterpret_cast<uint16_t*>(ws + pl.off_T) : a.T;
+  if (pl.fewtok) {
+    CUtensorMap tm;
+    if (!make_map(&tm, a.q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 256,
+                  CU_TENSOR_MAP_SWIZZLE_128B)) {
+      *why = "tensor map encoding failed (few-token forward)";
+      return QLORA_ERR_CUDA;
+    }
+    return launch_fewtok_fwd(a, T, ws + pl.off_main, &tm, st, why);
+  }
   float* partT = reinterpret_cast<float*>(ws + pl.off_partT);
   int rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, a.s, pl.splits_T, partT, T, st, why);
   if (rc) return rc;

@@ -3,7 +3,11 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/qlora.h"
@@ -52,6 +56,33 @@ size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r);
 // Returns 0 on success, a negative qlora_status otherwise; `why` names the failure.
 int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why);
 int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why);
+
+// few-token forward (qlora_fewtok.cu): M <= kFewTokMax tokens, weights streamed
+// once with register-resident dequantisation.  `tm_codes` maps the packed codes
+// as (k/2 bytes) x d rows, box 128 x 256, 128-byte swizzle.
+constexpr int kFewTokMax = 16;
+bool fewtok_eligible(int64_t M, int64_t d, int64_t k);
+size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k);
+int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensorMap* tm_codes, cudaStream_t st,
+                      const char** why);
+
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device); the
+// attribute call costs host time on every launch otherwise.  Instantiations of
+// one kernel template share a function type, so the key is the address.
+template <typename K>
+cudaError_t set_smem(K kernel, uint32_t bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, uint32_t> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const std::pair<const void*, int> key(reinterpret_cast<const void*>(kernel), dev);
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) done[key] = bytes;
+  return e;
+}
 
 // tracing (qlora_prof.cu): construct around each kernel launch
 struct ProfScope {
