@@ -510,7 +510,7 @@ def run_secondary(args, wl_name):
     else:
         raise SystemExit(f"unknown secondary workload {wl_name}")
     print(json.dumps({"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "workload": wl_name,
-                      "hbm_peak_gbs": hbm, "peak_source": src, "l2": "flushed (512 MB write) before every run",
+                      "hbm_peak_gbs": hbm, "peak_source": src, "l2": f"flushed ({2 * L2_BYTES >> 20} MiB write) before every run",
                       "iters": iters, "results": results}), flush=True)
 
 

@@ -7,34 +7,42 @@
 //
 // With a handful of tokens each 4-bit weight takes part in at most 16
 // products, so the layer is bound by streaming the packed codes from HBM
-// (half a byte per weight) and by the work of expanding them.  This path keeps
-// the expanded weights in registers:
+// (half a byte per weight).  This path keeps the expanded weights in registers
+// and is organised around keeping enough bytes in flight:
 //
-//   * TMA streams code tiles of 256 weight rows x 256 columns (32 KB) through a
-//     ring in shared memory, issued by one lane of warp 0 a few items ahead of
-//     the 16 warps that consume them; one CTA per SM and an even static split
-//     of the (row block, K chunk) items over the CTAs, so every SM streams the
-//     same number of bytes.
+//   * Work items are 256 weight rows x 256 columns (32 KB of codes), split
+//     evenly over one CTA per SM.  TMA brings each item's code tile and the
+//     matching 256 columns of X (one 3-D box) through a ring of up to five
+//     stages; the refill of the stage of item i with item i + S is issued by
+//     warp i mod 16, so issuing costs no single warp more than its share.  The
+//     8-bit block constants c2 come with the first item of each group of four
+//     (16 blocks x 256 rows, two slots); the group constants c1 (or, without
+//     double quantisation, the absmax) are loaded three items ahead.
 //   * A code byte (two weights) is expanded with one shared-memory lookup: a
-//     256-entry table holds the bf16 pair (C[low nibble], C[high nibble]).  It
-//     is replicated per lane (no bank conflicts) with 256 bytes per entry at a
-//     64 KB-aligned base, so one byte permute forms each lookup address.
+//     256-entry table holds the bf16 pair (C[low nibble], C[high nibble]),
+//     replicated per lane (a lane always reads its own bank).  Entries are
+//     256 bytes apart from a 64 KB-aligned base, so a single byte permute
+//     turns a code byte into its lookup address.
 //   * Products run on mma.sync m16n8k16 (bf16 operands, fp32 accumulation):
 //     the weights are the register-resident A operand and 8 tokens the N side.
 //     Inside a 64-weight block the K order is permuted so that each lane's own
 //     code bytes fill its fragment slots; X is read with the same permutation.
+//     Tensor-core instructions that take their operands from shared memory
+//     would need every expanded weight written to and read back from shared
+//     memory, which at this arithmetic intensity costs more than the HBM
+//     stream itself.
 //   * The codebook enters the products unscaled; each block's partial sum is
 //     multiplied by its scale s^ in fp32.  C[q] in bf16 times s^ carries the
 //     same bound, 2^-9 relative, as the bf16 weight BF16(C[q] s^) that the
 //     dequantisation produces.
-//   * Partial sums of a row block that several CTAs share are added, in CTA
-//     order, by the CTA that finishes the block last (one ticket per row
-//     block).  It also adds the LoRA term T_s B^T (mma.sync) and writes Y.
+//   * When a CTA leaves a row block it writes its partial sums.  A third
+//     kernel, k_fewtok_finish, adds each row block's partial sums in CTA
+//     order, adds the LoRA term T_s B^T (mma.sync) and writes Y.
 //
-// T_s = BF16(s X A^T) comes from k_lora_down_fewtok, a cluster kernel launched
-// just before; the main kernel is its programmatic dependent, streams weights
-// while it runs, and waits for it (griddepcontrol.wait) only before the
-// tickets.  The down kernel also clears the tickets.
+// The three kernels are chained by programmatic dependent launch:
+// k_lora_down_fewtok computes T_s = BF16(s X A^T) (a cluster kernel), the main
+// kernel streams the weights while it runs and waits for it only before
+// exiting, and the finish kernel launches while the main kernel drains.
 #include <cstdio>
 
 #include "nf4_scale.cuh"
@@ -50,86 +58,102 @@ constexpr int kFtWarps = 16;                                // 4 per SM sub-part
 constexpr int kFtThreads = kFtWarps * 32;
 constexpr int kFtRows = 256;                                // weight rows per item
 constexpr int kFtK = 256;                                   // weights per row per item
-constexpr uint32_t kFtStageBytes = kFtRows * kFtK / 2;      // 32 KB of codes
-constexpr int kFtMaxStages = 4;
+constexpr uint32_t kFtCodeBytes = kFtRows * kFtK / 2;       // 32 KB of codes per item
+constexpr int kFtMaxStages = 5;
 constexpr uint32_t kFtTableBytes = 65536;
 constexpr uint32_t kFtSmemBytes = 227u * 1024u;             // the whole window; placed in the kernel
 constexpr int kFtCluster = 8;                               // CTAs of one down-projection cluster
+constexpr int kFtScaleAhead = 3;                            // items of block constants in flight
+constexpr uint32_t kFtC2Box = 16u * kFtRows;                // c2 of 16 blocks x 256 rows (four items)
+constexpr int kFtC2Slots = 2;
+
+template <int NTOK>
+struct FtCfg {
+  static constexpr int kTG = NTOK / 8;                            // token groups of 8 (MMA N)
+  static constexpr uint32_t kXBox = NTOK * 128u;                   // 64 columns of X for NTOK tokens
+  static constexpr uint32_t kStageBytes = kFtCodeBytes + 4u * kXBox;
+  static constexpr uint32_t kScratch = 4u * 32u * 16u * kTG * 4u;  // [row set][lane][16 TG floats]
+  static constexpr uint32_t kMisc = 128;                           // barriers and flags
+};
 
 struct FtParams {
   int64_t M, d, k;
   int32_t kpb;          // NF4 blocks per weight row
   int32_t r, rp;
   ScaleSrc sc;
-  const uint16_t* X;    // M x k
   const uint16_t* B;    // d x r
   const uint16_t* T;    // M x rp, T_s (written by the down kernel)
   uint16_t* Y;          // M x d
   float* partial;       // [G][segmax][NTOK][256]
-  unsigned* tickets;    // [RB]
   int32_t items, KC, G, segmax;
+  int32_t c2_tma;       // c2 arrives through the TMA ring (double quantisation, kpb % 16 == 0)
 };
 
-// Shared-memory placement.  The lookup table needs a 64 KB-aligned base; the
-// ring stages (1 KB-aligned for the 128-byte swizzle), the barriers and the
-// reduction scratch fill the space before and after it.
+// Shared-memory placement.  The lookup table needs a 64 KB-aligned base.  For
+// each possible table position the ring stages (1 KB-aligned for the 128-byte
+// swizzle) fill the space below and above it, then the small pieces (c2 ring,
+// scratch, barriers) take the first gap that holds them; the position that
+// leaves room for the most stages wins.  Stages below the table are numbered
+// first: stage i < nlo sits at lo0 + i * stage bytes, the rest at hi0 + ...
 struct FtLayout {
-  uint32_t table, misc, scratch;
-  uint32_t stage0, stage1, stage2, stage3;
-  int nst;
+  uint32_t table, misc, scratch, c2, lo0, hi0;
+  int nlo, nst;
   bool ok;
 };
 
-template <int TG>
+template <int NTOK>
 __device__ __forceinline__ FtLayout ft_layout(uint32_t raw) {
-  constexpr uint32_t kMisc = 128;
-  constexpr uint32_t kScratch = 4u * 32u * 16u * TG * 4u;     // [row set][lane][16 TG floats]
-  FtLayout L{};
+  using Cfg = FtCfg<NTOK>;
+  constexpr uint32_t SB = Cfg::kStageBytes;
+  FtLayout best{};
+  best.ok = false;
   const uint32_t end = raw + kFtSmemBytes;
-  L.table = (raw + 65535u) & ~65535u;
-  L.ok = L.table + kFtTableBytes <= end;
-  uint32_t a0 = raw, a1 = L.table, b0 = L.table + kFtTableBytes, b1 = end;
-  auto take = [&](uint32_t bytes, uint32_t align, uint32_t& out) -> bool {
-    uint32_t x = (a0 + align - 1u) & ~(align - 1u);
-    if (x + bytes <= a1) {
-      out = x;
-      a0 = x + bytes;
-      return true;
+  for (uint32_t T = (raw + kFtTableBytes - 1u) & ~(kFtTableBytes - 1u); T + kFtTableBytes <= end; T += kFtTableBytes) {
+    const uint32_t lo0 = (raw + 1023u) & ~1023u, hi0 = T + kFtTableBytes;
+    const int maxlo = lo0 <= T ? static_cast<int>((T - lo0) / SB) : 0;
+    const int maxhi = static_cast<int>((end - hi0) / SB);
+    for (int nlo = maxlo; nlo >= 0; --nlo) {
+      int nhi = maxhi;
+      if (nlo + nhi > kFtMaxStages) nhi = kFtMaxStages - nlo;
+      if (nhi < 0) continue;
+      for (; nhi >= 0; --nhi) {
+        if (best.ok && nlo + nhi <= best.nst) break;
+        uint32_t a = lo0 + nlo * SB, b = hi0 + nhi * SB;
+        auto take = [&](uint32_t bytes, uint32_t align, uint32_t& out) -> bool {
+          uint32_t x = (a + align - 1u) & ~(align - 1u);
+          if (x + bytes <= T) {
+            out = x;
+            a = x + bytes;
+            return true;
+          }
+          x = (b + align - 1u) & ~(align - 1u);
+          if (x + bytes <= end) {
+            out = x;
+            b = x + bytes;
+            return true;
+          }
+          return false;
+        };
+        FtLayout L{};
+        if (take(kFtC2Slots * kFtC2Box, 128u, L.c2) && take(Cfg::kScratch, 16u, L.scratch) &&
+            take(Cfg::kMisc, 16u, L.misc)) {
+          L.table = T;
+          L.lo0 = lo0;
+          L.hi0 = hi0;
+          L.nlo = nlo;
+          L.nst = nlo + nhi;
+          L.ok = L.nst >= 3;
+          if (L.ok) best = L;
+          break;
+        }
+      }
     }
-    x = (b0 + align - 1u) & ~(align - 1u);
-    if (x + bytes <= b1) {
-      out = x;
-      b0 = x + bytes;
-      return true;
-    }
-    return false;
-  };
-  L.ok = L.ok && take(kMisc + kScratch, 16u, L.misc);
-  L.scratch = L.misc + kMisc;
-  uint32_t s[kFtMaxStages] = {0, 0, 0, 0};
-  L.nst = 0;
-#pragma unroll
-  for (int i = 0; i < kFtMaxStages; ++i)
-    if (take(kFtStageBytes, 1024u, s[i])) ++L.nst;
-  L.stage0 = s[0];
-  L.stage1 = s[1];
-  L.stage2 = s[2];
-  L.stage3 = s[3];
-  L.ok = L.ok && L.nst >= 2;
-  return L;
-}
-
-__device__ __forceinline__ uint32_t ft_stage(const FtLayout& L, int st) {
-  return st == 0 ? L.stage0 : (st == 1 ? L.stage1 : (st == 2 ? L.stage2 : L.stage3));
+  }
+  return best;
 }
 
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
 }
 // Lookup in the constant code-byte table (written once before a CTA-wide
 // barrier): no ordering constraints, so the compiler may batch them.
@@ -143,6 +167,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
   return v;
 }
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
 
 // D += A B: 16 x 8 x 16, bf16 inputs, fp32 accumulators (register fragments).
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -153,6 +183,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// D = A B (no accumulator input).
+__device__ __forceinline__ void mma16816_first(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
+}
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -183,87 +221,88 @@ __device__ __forceinline__ int first_item(int c, int items, int G) {
   return static_cast<int>(static_cast<int64_t>(c) * items / G);
 }
 
+// Two bf16 at an even element offset as one 32-bit word (4-byte aligned).
+__device__ __forceinline__ uint32_t ld_pair(const uint16_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
 }  // namespace
 
 // ============================================================================
-// T_s = BF16(s X A^T) for M <= NTOK tokens.  One cluster of 8 CTAs per group
-// of 8 ranks: CTA q of the cluster sums over the q-th eighth of K (warp w =
-// rank 8 g + w, lanes strided over 8-column chunks), and CTA 0 adds the eight
-// partial sums in order through distributed shared memory.
+// T_s = BF16(s X A^T) for M <= 16 tokens on mma.sync: tokens are the M side
+// (16 rows), 8 ranks the N side.  One cluster of 8 CTAs per group of 8 ranks;
+// CTA q of the cluster covers the q-th eighth of K, its 8 warps take every
+// 8th 16-column step of it, the warps' fragments are added in warp order and
+// CTA 0 adds the eight CTAs' sums in order through distributed shared memory.
 // ============================================================================
-template <int NTOK>
 __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
     k_lora_down_fewtok(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int M, int64_t k, int r,
-                       int rp, float s, uint16_t* __restrict__ T, unsigned* __restrict__ tickets, int n_tickets) {
+                       int rp, float s, uint16_t* __restrict__ T) {
   griddep_launch_dependents();
-  __shared__ float part[8][NTOK];
+  __shared__ float4 red[8][32];
   const uint32_t q = cluster_rank();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int j = static_cast<int>(blockIdx.x / kFtCluster) * 8 + warp;
-  const int64_t nch = k >> 3;
-  const int64_t c0 = nch * q / kFtCluster, c1 = nch * (q + 1) / kFtCluster;
-  float acc[NTOK];
-#pragma unroll
-  for (int m = 0; m < NTOK; ++m) acc[m] = 0.0f;
-  if (j < r) {
-    for (int64_t ch = c0 + lane; ch < c1; ch += 32) {
-      const uint4 av = ldg_nc_v4(A + static_cast<int64_t>(j) * k + ch * 8);
-      const float a[8] = {bf16_lo(av.x), bf16_hi(av.x), bf16_lo(av.y), bf16_hi(av.y),
-                          bf16_lo(av.z), bf16_hi(av.z), bf16_lo(av.w), bf16_hi(av.w)};
-#pragma unroll
-      for (int m = 0; m < NTOK; ++m) {
-        if (m < M) {
-          const uint4 xv = ldg_nc_v4(X + static_cast<int64_t>(m) * k + ch * 8);
-          float v = acc[m];
-          v = fmaf(bf16_lo(xv.x), a[0], v);
-          v = fmaf(bf16_hi(xv.x), a[1], v);
-          v = fmaf(bf16_lo(xv.y), a[2], v);
-          v = fmaf(bf16_hi(xv.y), a[3], v);
-          v = fmaf(bf16_lo(xv.z), a[4], v);
-          v = fmaf(bf16_hi(xv.z), a[5], v);
-          v = fmaf(bf16_lo(xv.w), a[6], v);
-          v = fmaf(bf16_hi(xv.w), a[7], v);
-          acc[m] = v;
-        }
-      }
+  const int g = lane >> 2, c = lane & 3;
+  const int j0 = static_cast<int>(blockIdx.x / kFtCluster) * 8;
+  const int64_t n16 = k >> 4;
+  const int64_t s0 = n16 * q / kFtCluster, s1 = n16 * (q + 1) / kFtCluster;
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (j0 < r) {
+    const bool ta = g < M, tb = g + 8 < M, jv = j0 + g < r;
+    const uint16_t* xa = X + static_cast<int64_t>(g) * k + 2 * c;
+    const uint16_t* xb = X + static_cast<int64_t>(g + 8) * k + 2 * c;
+    const uint16_t* ar = A + static_cast<int64_t>(j0 + g) * k + 2 * c;
+#pragma unroll 4
+    for (int64_t st = s0 + warp; st < s1; st += 8) {
+      const int64_t k0 = 16 * st;
+      const uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
+      const uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
+      const uint32_t b0 = jv ? ld_pair(ar + k0) : 0u, b1 = jv ? ld_pair(ar + k0 + 8) : 0u;
+      mma16816(acc, a0, a1, a2, a3, b0, b1);
     }
   }
-#pragma unroll
-  for (int m = 0; m < NTOK; ++m) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int m = 0; m < NTOK; ++m) part[warp][m] = acc[m];
+  red[warp][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  __syncthreads();
+  if (warp == 0) {
+    float4 t = red[0][lane];
+    for (int w = 1; w < 8; ++w) {
+      const float4 v = red[w][lane];
+      t.x += v.x;
+      t.y += v.y;
+      t.z += v.z;
+      t.w += v.w;
+    }
+    red[0][lane] = t;
   }
   cluster_sync_all();
-  if (q == 0 && threadIdx.x < 8 * NTOK) {
-    const int w = threadIdx.x / NTOK, m = threadIdx.x % NTOK;
-    float sum = 0.0f;
-    for (uint32_t p = 0; p < kFtCluster; ++p) sum += ld_cluster_f32(&part[w][m], p);
-    const int jj = static_cast<int>(blockIdx.x / kFtCluster) * 8 + w;
-    if (m < M && jj < rp) {
-      const uint32_t b = pack_bf16x2(jj < r ? s * sum : 0.0f, 0.0f);
-      T[static_cast<int64_t>(m) * rp + jj] = static_cast<uint16_t>(b & 0xFFFFu);
+  if (q == 0 && warp == 0) {
+    float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    for (uint32_t p = 0; p < kFtCluster; ++p)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) tot[e] += ld_cluster_f32(reinterpret_cast<const float*>(&red[0][lane]) + e, p);
+    // fragment element e: token g + 8 (e >> 1), rank j0 + 2 c + (e & 1)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int tok = g + 8 * (e >> 1), j = j0 + 2 * c + (e & 1);
+      if (tok < M && j < rp)
+        T[static_cast<int64_t>(tok) * rp + j] =
+            static_cast<uint16_t>(pack_bf16x2(j < r ? s * tot[e] : 0.0f, 0.0f) & 0xFFFFu);
     }
   }
   cluster_sync_all();   // peers keep their shared memory until CTA 0 has read it
-  if (blockIdx.x == 0)
-    for (int i = threadIdx.x; i < n_tickets; i += blockDim.x) tickets[i] = 0u;
 }
 
 // ============================================================================
 // Main kernel
 // ============================================================================
 // Combine the four warps that share a 64-row set (one per 64-column block of
-// the item) and write the CTA's partial sums of the finished row block.
+// the item) and write the CTA's partial sums of the row block it leaves: in
+// three rounds the warps of block b = 1, 2, 3 park their sums in shared memory
+// (one slot per row set and lane) and the block-0 warp adds them in order.
 template <int TG>
 __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch, float* part, int rs, int bk,
                                          int lane) {
   float* scr = scratch + (rs * 32 + lane) * 16 * TG;
-  __syncthreads();
   for (int b = 1; b < 4; ++b) {
+    __syncthreads();   // the slot is free (block-0 warps have read the previous round)
     if (bk == b) {
 #pragma unroll
       for (int rg = 0; rg < 4; ++rg)
@@ -285,7 +324,6 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
           acc[rg][t][3] += v.w;
         }
     }
-    __syncthreads();
   }
   if (bk == 0) {
     const int g = lane >> 2, c = lane & 3;
@@ -309,11 +347,15 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
       for (int e = 0; e < 4; ++e) acc[rg][t][e] = 0.0f;
 }
 
-// Last CTA of row block rb: Y = BF16(sum of the CTAs' partial sums + T_s B^T).
-// Warp w takes rows 16 w .. 16 w + 15 of the block.
+// Row block rb: Y = BF16(sum of the CTAs' partial sums + T_s B^T); warp w
+// takes rows 16 w .. 16 w + 15 of the block.  All global loads of a batch are
+// issued before any is used (a row block has a few contributors and r / 16
+// LoRA steps).
 template <int NTOK>
 __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, int lane) {
   constexpr int TG = NTOK / 8;
+  constexpr int kC = 4;    // contributors per batch
+  constexpr int kS = 4;    // LoRA K steps (16 ranks each) per batch
   const int g = lane >> 2, c = lane & 3;
   const int64_t na = static_cast<int64_t>(rb) * kFtRows + 16 * warp + g, nb = na + 8;
   const int ra = 16 * warp + g;
@@ -324,42 +366,61 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
     for (int e = 0; e < 4; ++e) v[t][e] = 0.0f;
   const int64_t i0 = static_cast<int64_t>(rb) * p.KC;
   const int cf = cta_of_item(i0, p.items, p.G), cl = cta_of_item(i0 + p.KC - 1, p.items, p.G);
-  for (int cc = cf; cc <= cl; ++cc) {
-    const int seg = rb - first_item(cc, p.items, p.G) / p.KC;
-    const float* part = p.partial + (static_cast<int64_t>(cc) * p.segmax + seg) * NTOK * kFtRows;
+  for (int c0 = cf; c0 <= cl; c0 += kC) {
+    float pv[kC][TG][4];
 #pragma unroll
-    for (int t = 0; t < TG; ++t) {
-      const int tok = 8 * t + 2 * c;
-      v[t][0] += part[tok * kFtRows + ra];
-      v[t][1] += part[(tok + 1) * kFtRows + ra];
-      v[t][2] += part[tok * kFtRows + ra + 8];
-      v[t][3] += part[(tok + 1) * kFtRows + ra + 8];
+    for (int u = 0; u < kC; ++u) {
+      const int cc = c0 + u;
+      const bool ok = cc <= cl;
+      const int seg = ok ? rb - first_item(cc, p.items, p.G) / p.KC : 0;
+      const float* part = p.partial + (static_cast<int64_t>(ok ? cc : cf) * p.segmax + seg) * NTOK * kFtRows;
+#pragma unroll
+      for (int t = 0; t < TG; ++t) {
+        const int tok = 8 * t + 2 * c;
+        pv[u][t][0] = ok ? part[tok * kFtRows + ra] : 0.0f;
+        pv[u][t][1] = ok ? part[(tok + 1) * kFtRows + ra] : 0.0f;
+        pv[u][t][2] = ok ? part[tok * kFtRows + ra + 8] : 0.0f;
+        pv[u][t][3] = ok ? part[(tok + 1) * kFtRows + ra + 8] : 0.0f;
+      }
     }
+#pragma unroll
+    for (int u = 0; u < kC; ++u)
+#pragma unroll
+      for (int t = 0; t < TG; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[t][e] += pv[u][t][e];
   }
   // LoRA term: rows of B are the A operand, T_s^T the B operand.
+  const bool even = (p.r & 1) == 0;
   auto bpair = [&](int64_t n, int j) -> uint32_t {
-    uint32_t lo = 0, hi = 0;
-    if (n < p.d) {
-      if (j < p.r) lo = p.B[n * p.r + j];
-      if (j + 1 < p.r) hi = p.B[n * p.r + j + 1];
-    }
+    if (n >= p.d || j >= p.r) return 0u;
+    const uint16_t* src = p.B + n * p.r + j;
+    if (even) return ld_pair(src);
+    const uint32_t lo = src[0], hi = (j + 1 < p.r) ? src[1] : 0u;
     return lo | (hi << 16);
   };
-  for (int ks = 0; ks < p.rp / 16; ++ks) {
-    const int j0 = 16 * ks + 2 * c;
-    if (16 * ks >= p.r) break;
-    const uint32_t a0 = bpair(na, j0), a1 = bpair(nb, j0), a2 = bpair(na, j0 + 8), a3 = bpair(nb, j0 + 8);
+  for (int k0 = 0; 16 * k0 < p.r; k0 += kS) {
+    uint32_t af[kS][4], bf[kS][TG][2];
 #pragma unroll
-    for (int t = 0; t < TG; ++t) {
-      const int tok = 8 * t + g;
-      uint32_t b0 = 0, b1 = 0;
-      if (tok < p.M) {
-        const uint32_t* trow = reinterpret_cast<const uint32_t*>(p.T + static_cast<int64_t>(tok) * p.rp);
-        b0 = trow[j0 >> 1];
-        b1 = trow[(j0 + 8) >> 1];
+    for (int u = 0; u < kS; ++u) {
+      const int j0 = 16 * (k0 + u) + 2 * c;
+      const bool ok = 16 * (k0 + u) < p.r;
+      af[u][0] = ok ? bpair(na, j0) : 0u;
+      af[u][1] = ok ? bpair(nb, j0) : 0u;
+      af[u][2] = ok ? bpair(na, j0 + 8) : 0u;
+      af[u][3] = ok ? bpair(nb, j0 + 8) : 0u;
+#pragma unroll
+      for (int t = 0; t < TG; ++t) {
+        const int tok = 8 * t + g;
+        const uint16_t* trow = p.T + static_cast<int64_t>(tok) * p.rp;
+        bf[u][t][0] = (ok && tok < p.M) ? ld_pair(trow + j0) : 0u;
+        bf[u][t][1] = (ok && tok < p.M) ? ld_pair(trow + j0 + 8) : 0u;
       }
-      mma16816(v[t], a0, a1, a2, a3, b0, b1);
     }
+#pragma unroll
+    for (int u = 0; u < kS; ++u)
+#pragma unroll
+      for (int t = 0; t < TG; ++t) mma16816(v[t], af[u][0], af[u][1], af[u][2], af[u][3], bf[u][t][0], bf[u][t][1]);
   }
 #pragma unroll
   for (int t = 0; t < TG; ++t) {
@@ -374,13 +435,30 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
   }
 }
 
+// One CTA per row block, 16 warps; launched as the programmatic dependent of
+// the main kernel.
+template <int NTOK>
+__global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) {
+  griddep_wait();   // the main kernel's partial sums (and, through it, T_s)
+  ft_finish<NTOK>(p, blockIdx.x, threadIdx.x >> 5, threadIdx.x & 31);
+}
+
+// Block constants of one item for this lane's two rows, loaded ahead of use:
+// c2 bytes (DQ) and validity bits in `w`, c1 (DQ) or absmax in a and b.
+struct FtScaleQ {
+  uint32_t w;
+  float a, b;
+};
+
 template <int NTOK>
 __global__ void __launch_bounds__(kFtThreads, 1)
-    k_qlora_fewtok(const __grid_constant__ CUtensorMap tm_codes, const FtParams p) {
-  constexpr int TG = NTOK / 8;
+    k_qlora_fewtok(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_c2, const FtParams p) {
+  using Cfg = FtCfg<NTOK>;
+  constexpr int TG = Cfg::kTG;
   extern __shared__ __align__(1024) uint8_t ft_smem[];
   const uint32_t raw = smem_u32(ft_smem);
-  const FtLayout L = ft_layout<TG>(raw);
+  const FtLayout L = ft_layout<NTOK>(raw);
   if (!L.ok) {
     if (threadIdx.x == 0) report(DEV_SMEM_LAYOUT);
     return;
@@ -388,27 +466,36 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   auto gptr = [&](uint32_t a) { return ft_smem + (a - raw); };
   uint64_t* full = reinterpret_cast<uint64_t*>(gptr(L.misc));
   uint64_t* empty = full + kFtMaxStages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + 2 * kFtMaxStages);
-  volatile int* last_flag = abort_flag + 1;
+  volatile int* last_item = reinterpret_cast<volatile int*>(full + 2 * kFtMaxStages);   // per stage, for draining
+  volatile int* abort_flag = last_item + kFtMaxStages;
   const int S = L.nst;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int it0 = first_item(blockIdx.x, p.items, p.G);
   const int it1 = first_item(blockIdx.x + 1, p.items, p.G);
   const int n_items = it1 - it0;
+  auto stage = [&](int st) {
+    return st < L.nlo ? L.lo0 + static_cast<uint32_t>(st) * Cfg::kStageBytes
+                      : L.hi0 + static_cast<uint32_t>(st - L.nlo) * Cfg::kStageBytes;
+  };
 
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], kFtWarps);
     }
+    for (int i = 0; i < kFtMaxStages; ++i) last_item[i] = -1;
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_x);
+    if (p.c2_tma) tma_prefetch_desc(&tm_c2);
   }
   {
-    // code-byte table: entry e = (C[e & 15], C[e >> 4]) in bf16, one copy per lane
+    // code-byte table: entry e = (C[e & 15], C[e >> 4]) in bf16; lane l's copy
+    // of entry e at e * 256 + 4 l
     constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
-    for (int i = threadIdx.x; i < 256 * 32; i += kFtWarps * 32) {
+    for (int i = threadIdx.x; i < 256 * 32; i += kFtThreads) {
       const int e = i >> 5;
       const uint32_t v = pack_bf16x2(__uint_as_float(kCB[e & 15]), __uint_as_float(kCB[e >> 4]));
       sts32(L.table + static_cast<uint32_t>(e) * 256u + static_cast<uint32_t>(i & 31) * 4u, v);
@@ -416,196 +503,213 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   }
   __syncthreads();
 
-  {
-    // ------------------------------------------------------------ consumers
-    // warp = (row set rs: 64 rows) x (block bk: 64 columns of the item)
-    const int rs = warp & 3, bk = warp >> 2;
-    const int g = lane >> 2, c = lane & 3;
-    const uint32_t lanebase = L.table + static_cast<uint32_t>(lane) * 4u;
-    // this lane's 8 code bytes of row 64 rs + g in the 128-byte-swizzled tile
-    const uint32_t lane_off = static_cast<uint32_t>(64 * rs + g) * 128u +
-                              16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ g) + 8u * static_cast<uint32_t>(c & 1);
-    float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
-    float acc[4][TG][4];
+  // warp = (row set rs: 64 rows) x (block bk: 64 columns of the item)
+  const int rs = warp & 3, bk = warp >> 2;
+  const int g = lane >> 2, c = lane & 3;
+  const uint32_t lanebase = L.table + static_cast<uint32_t>(lane) * 4u;
+  // this lane's 8 code bytes of row 64 rs + g in the 128-byte-swizzled tile
+  const uint32_t code_off = static_cast<uint32_t>(64 * rs + g) * 128u +
+                            16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ g) + 8u * static_cast<uint32_t>(c & 1);
+  // this lane's 16 columns of X (token 8 t + g) in the 128-byte-swizzled X chunk of block bk
+  const uint32_t x_off = kFtCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
+  const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
+  float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
+  const float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;
+  ScaleRecip rec0, rec1;
+
+  // ---- TMA issue of item j into stage sj: the code tile, the item's 256
+  // columns of X and, at the first item of a group of four, the group's c2
+  // (slot = group index mod 2; a slot is refilled only after the item that
+  // read it has been released, at least five items later).
+  auto issue_item = [&](int j, int sj) {
+    const int gi = it0 + j, irb = gi / p.KC, ikc = gi - irb * p.KC;
+    const bool c2n = p.c2_tma && (j == 0 || (ikc & 3) == 0);
+    mbar_arrive_expect_tx(&full[sj], Cfg::kStageBytes + (c2n ? kFtC2Box : 0u));
+    uint8_t* dst = gptr(stage(sj));
+    tma_load_2d(dst, &tm_codes, &full[sj], ikc * (kFtK / 2), irb * kFtRows);
+    tma_load_3d(dst + kFtCodeBytes, &tm_x, &full[sj], 0, 0, 4 * ikc);
+    if (c2n)
+      tma_load_2d(gptr(L.c2 + ((gi >> 2) & 1) * kFtC2Box), &tm_c2, &full[sj], 4 * (ikc & ~3), irb * kFtRows);
+    last_item[sj] = j;
+  };
+  if (threadIdx.x == 0)
+    for (int j = 0; j < n_items && j < S; ++j) issue_item(j, j);
+
+  // ---- block constants, kFtScaleAhead items ahead
+  int frb = it0 / p.KC, fkc = it0 - frb * p.KC, fetched = 0;
+  auto fetch = [&]() -> FtScaleQ {
+    FtScaleQ qv{0u, 0.0f, 0.0f};
+    if (fetched < n_items) {
+      const int64_t blk = 4ll * fkc + bk;
+      const int64_t n0 = static_cast<int64_t>(frb) * kFtRows + 64 * rs + 16 * c + g;
+      const bool bv = blk < p.kpb;
+      const bool v0 = bv && (n0 < p.d), v1 = bv && (n0 + 8 < p.d);
+      if (p.sc.dq) {
+        uint32_t c2a = 0, c2b = 0;
+        if (v0) {
+          if (!p.c2_tma) c2a = static_cast<uint8_t>(__ldg(p.sc.c2 + n0 * p.kpb + blk));
+          qv.a = __ldg(p.sc.c1 + ((n0 * p.kpb + blk) >> 8));
+        }
+        if (v1) {
+          if (!p.c2_tma) c2b = static_cast<uint8_t>(__ldg(p.sc.c2 + (n0 + 8) * p.kpb + blk));
+          qv.b = __ldg(p.sc.c1 + (((n0 + 8) * p.kpb + blk) >> 8));
+        }
+        qv.w = c2a | (c2b << 8);
+      } else {
+        if (v0) qv.a = __ldg(p.sc.absmax + n0 * p.kpb + blk);
+        if (v1) qv.b = __ldg(p.sc.absmax + (n0 + 8) * p.kpb + blk);
+      }
+      qv.w |= (v0 ? 1u << 16 : 0u) | (v1 ? 1u << 17 : 0u);
+      if (++fkc == p.KC) {
+        fkc = 0;
+        ++frb;
+      }
+    }
+    ++fetched;
+    return qv;
+  };
+  FtScaleQ sq[kFtScaleAhead];
+#pragma unroll
+  for (int i = 0; i < kFtScaleAhead; ++i) sq[i] = fetch();
+
+  float acc[4][TG][4];
+#pragma unroll
+  for (int rg = 0; rg < 4; ++rg)
+#pragma unroll
+    for (int t = 0; t < TG; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[rg][t][e] = 0.0f;
+
+  // ---- leaving a row block: the CTA's partial sums out
+  int seg = 0;
+  auto leave_block = [&](int) {
+    ft_flush<TG>(acc, scratch, p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * kFtRows, rs,
+                 bk, lane);
+    ++seg;
+  };
+
+  int st = 0, rb = it0 / p.KC, kc = it0 - rb * p.KC;
+  uint32_t ph = 0;
+  int pst = 0;        // stage and parity of the previous item
+  uint32_t pph = 0;
+  uint32_t c2w0 = 0, c2w1 = 0;   // c2 of this lane's two rows for the four items of the group
+  for (int i = 0; i < n_items; ++i) {
+    FtScaleQ cur = sq[0];
+#pragma unroll
+    for (int qi = 0; qi < kFtScaleAhead - 1; ++qi) sq[qi] = sq[qi + 1];
+    sq[kFtScaleAhead - 1] = fetch();
+
+    mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
+    const uint32_t sb = stage(st);
+    if (p.c2_tma && (i == 0 || (kc & 3) == 0)) {
+      // first item of a group of four: the group's c2, row 16 c + g (+8) of the
+      // row set; byte 4 t + bk is block bk of item t of the group
+      const uint32_t cb = L.c2 + (((it0 + i) >> 2) & 1) * kFtC2Box + static_cast<uint32_t>(64 * rs + 16 * c + g) * 16u;
+      const uint4 ra = lds128(cb), rb8 = lds128(cb + 8u * 16u);
+      const uint32_t sel = 0x40u + 0x11u * static_cast<uint32_t>(bk);   // byte bk of each word
+      c2w0 = prmt(prmt(ra.x, ra.y, sel), prmt(ra.z, ra.w, sel), 0x5410u);
+      c2w1 = prmt(prmt(rb8.x, rb8.y, sel), prmt(rb8.z, rb8.w, sel), 0x5410u);
+    }
+    if (p.c2_tma) cur.w |= ((c2w0 >> (8 * (kc & 3))) & 0xFFu) | (((c2w1 >> (8 * (kc & 3))) & 0xFFu) << 8);
+    uint2 cw[4][2];
 #pragma unroll
     for (int rg = 0; rg < 4; ++rg)
 #pragma unroll
-      for (int t = 0; t < TG; ++t)
+      for (int h = 0; h < 2; ++h) cw[rg][h] = lds64(sb + code_off + static_cast<uint32_t>(16 * rg + 8 * h) * 128u);
+    uint4 xv[TG][2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[rg][t][e] = 0.0f;
-    const float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;
-    ScaleRecip rec0, rec1;
+    for (int t = 0; t < TG; ++t) {
+      xv[t][0] = lds128(sb + x_off + static_cast<uint32_t>(8 * t) * 128u + x_c0);
+      xv[t][1] = lds128(sb + x_off + static_cast<uint32_t>(8 * t) * 128u + x_c1);
+    }
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&empty[st]);
+      // this warp's turn: refill the stage of item i - 1 (released by every
+      // warp one item ago) with item i - 1 + S
+      if (i > 0 && (i & (kFtWarps - 1)) == warp && i - 1 + S < n_items && !*abort_flag &&
+          mbar_wait(&empty[pst], pph, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT))
+        issue_item(i - 1 + S, pst);
+    }
+    pst = st;
+    pph = ph;
+    if (++st == S) {
+      st = 0;
+      ph ^= 1u;
+    }
 
-    // inputs of item gi that do not come through the ring: the block scales of
-    // this lane's two rows (16 c + g and +8 of the row set) and the lane's 16
-    // columns of X for each token group
-    auto fetch = [&](int rb, int kc, ScaleRaw& r0, ScaleRaw& r1, bool& v0, bool& v1, uint4 (&xv)[TG][2]) {
-      const int64_t blk = 4ll * kc + bk;
-      const int64_t n0 = static_cast<int64_t>(rb) * kFtRows + 64 * rs + 16 * c + g;
-      const bool bv = blk < p.kpb;
-      v0 = bv && (n0 < p.d);
-      v1 = bv && (n0 + 8 < p.d);
-      if (v0) r0 = scale_fetch(p.sc, n0 * p.kpb + blk);
-      if (v1) r1 = scale_fetch(p.sc, (n0 + 8) * p.kpb + blk);
-      const int64_t kb = 64ll * blk + 16 * c;
+    float sm0 = 0.0f, sm1 = 0.0f;
+    if (cur.w & (1u << 16)) {
+      ScaleRaw r0;
+      r0.a = cur.a;
+      r0.b = static_cast<int>(static_cast<int8_t>(cur.w & 0xFFu));
+      sm0 = scale_value(p.sc.dq, mean, r0, rec0);
+    }
+    if (cur.w & (1u << 17)) {
+      ScaleRaw r1;
+      r1.a = cur.b;
+      r1.b = static_cast<int>(static_cast<int8_t>((cur.w >> 8) & 0xFFu));
+      sm1 = scale_value(p.sc.dq, mean, r1, rec1);
+    }
+    // four independent accumulation chains (one per 16-row group)
+    float tmp[4][TG][4];
 #pragma unroll
-      for (int t = 0; t < TG; ++t) {
-        const int tok = 8 * t + g;
-        if (bv && tok < p.M) {
-          const uint16_t* src = p.X + static_cast<int64_t>(tok) * p.k + kb;
-          xv[t][0] = ldg_nc_v4(src);
-          xv[t][1] = ldg_nc_v4(src + 8);
-        } else {
-          xv[t][0] = make_uint4(0, 0, 0, 0);
-          xv[t][1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-    };
-
-    // lane 0 of warp 0 keeps S - 1 items in flight ahead of its own position
-    const bool producer = (threadIdx.x == 0);
-    int pst = 0, issued = 0;
-    uint32_t pph = 0;
-    auto issue = [&]() {
-      if (!mbar_wait(&empty[pst], pph ^ 1u, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) return;
-      const int gi = it0 + issued, rb = gi / p.KC, kc = gi - rb * p.KC;
-      mbar_arrive_expect_tx(&full[pst], kFtStageBytes);
-      tma_load_2d(gptr(ft_stage(L, pst)), &tm_codes, &full[pst], kc * (kFtK / 2), rb * kFtRows);
-      ++issued;
-      if (++pst == S) {
-        pst = 0;
-        pph ^= 1u;
-      }
-    };
-    if (producer)
-      while (issued < n_items && issued < S - 1 && !*abort_flag) issue();
-
-    int st = 0, cur_rb = -1, seg = -1;
-    uint32_t ph = 0;
-    ScaleRaw nr0{}, nr1{};
-    bool nv0 = false, nv1 = false;
-    uint4 nx[TG][2];
-    // (row block, K chunk) of the current item
-    int crb = it0 / p.KC, ckc = it0 - crb * p.KC;
-    if (n_items > 0) fetch(crb, ckc, nr0, nr1, nv0, nv1, nx);
-    for (int i = 0; i < n_items; ++i) {
-      const int rb = crb;
-      const bool wrap = (ckc + 1 == p.KC);
-      const int nrb = wrap ? crb + 1 : crb, nkc = wrap ? 0 : ckc + 1;   // the next item
-      crb = nrb;
-      ckc = nkc;
-      if (rb != cur_rb) {
-        if (cur_rb >= 0)
-          ft_flush<TG>(acc, scratch, p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * kFtRows,
-                       rs, bk, lane);
-        cur_rb = rb;
-        ++seg;
-      }
-      const ScaleRaw r0 = nr0, r1 = nr1;
-      const bool v0 = nv0, v1 = nv1;
-      uint4 xv[TG][2];
-#pragma unroll
-      for (int t = 0; t < TG; ++t) {
-        xv[t][0] = nx[t][0];
-        xv[t][1] = nx[t][1];
-      }
-      if (i + 1 < n_items) fetch(nrb, nkc, nr0, nr1, nv0, nv1, nx);
-
-      mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
-      const uint32_t sbase = ft_stage(L, st) + lane_off;
-      uint2 cw[4][2];
-#pragma unroll
-      for (int rg = 0; rg < 4; ++rg)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) cw[rg][h] = lds64(sbase + static_cast<uint32_t>(16 * rg + 8 * h) * 128u);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-      if (++st == S) {
-        st = 0;
-        ph ^= 1u;
-      }
-      // refill the stage every warp released one item ago
-      if (producer && issued < n_items && !*abort_flag) issue();
-
-      const float sm0 = v0 ? scale_value(p.sc.dq, mean, r0, rec0) : 0.0f;
-      const float sm1 = v1 ? scale_value(p.sc.dq, mean, r1, rec1) : 0.0f;
-      // four independent accumulation chains (one per 16-row group), stepped
-      // together so consecutive tensor-core ops never wait on each other
-      float tmp[4][TG][4];
-#pragma unroll
-      for (int rg = 0; rg < 4; ++rg)
-#pragma unroll
-        for (int t = 0; t < TG; ++t)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) tmp[rg][t][e] = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // MMA step j takes this lane's weights 4j .. 4j+3 (bytes 2j, 2j+1)
-        const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
-        const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
-#pragma unroll
-        for (int rg = 0; rg < 4; ++rg) {
-          const uint32_t w0 = (j < 2) ? cw[rg][0].x : cw[rg][0].y;
-          const uint32_t w1 = (j < 2) ? cw[rg][1].x : cw[rg][1].y;
-          const uint32_t a0 = lds32_const(prmt(w0, lanebase, sa));
-          const uint32_t a2 = lds32_const(prmt(w0, lanebase, sb));
-          const uint32_t a1 = lds32_const(prmt(w1, lanebase, sa));
-          const uint32_t a3 = lds32_const(prmt(w1, lanebase, sb));
-#pragma unroll
-          for (int t = 0; t < TG; ++t) {
-            const uint4 xq = xv[t][j >> 1];
-            const uint32_t b0 = (j & 1) ? xq.z : xq.x;
-            const uint32_t b1 = (j & 1) ? xq.w : xq.y;
-            mma16816(tmp[rg][t], a0, a1, a2, a3, b0, b1);
-          }
-        }
-      }
+    for (int j = 0; j < 4; ++j) {
+      // MMA step j takes this lane's weights 4j .. 4j+3: code bytes 2j and
+      // 2j + 1, i.e. bytes b = 2 (j & 1) and b + 1 of word j >> 1.  The byte
+      // permute puts the code byte into bits 8-15 of the lane's table address.
+      const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
+      const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
 #pragma unroll
       for (int rg = 0; rg < 4; ++rg) {
-        const float s0 = __shfl_sync(0xffffffffu, sm0, 4 * g + rg);
-        const float s1 = __shfl_sync(0xffffffffu, sm1, 4 * g + rg);
+        const uint32_t w0 = (j < 2) ? cw[rg][0].x : cw[rg][0].y;
+        const uint32_t w1 = (j < 2) ? cw[rg][1].x : cw[rg][1].y;
+        const uint32_t a0 = lds32_const(prmt(w0, lanebase, sa));
+        const uint32_t a2 = lds32_const(prmt(w0, lanebase, sb));
+        const uint32_t a1 = lds32_const(prmt(w1, lanebase, sa));
+        const uint32_t a3 = lds32_const(prmt(w1, lanebase, sb));
 #pragma unroll
         for (int t = 0; t < TG; ++t) {
-          acc[rg][t][0] = fmaf(tmp[rg][t][0], s0, acc[rg][t][0]);
-          acc[rg][t][1] = fmaf(tmp[rg][t][1], s0, acc[rg][t][1]);
-          acc[rg][t][2] = fmaf(tmp[rg][t][2], s1, acc[rg][t][2]);
-          acc[rg][t][3] = fmaf(tmp[rg][t][3], s1, acc[rg][t][3]);
+          const uint4 xq = xv[t][j >> 1];
+          const uint32_t b0 = (j & 1) ? xq.z : xq.x;
+          const uint32_t b1 = (j & 1) ? xq.w : xq.y;
+          if (j == 0)
+            mma16816_first(tmp[rg][t], a0, a1, a2, a3, b0, b1);
+          else
+            mma16816(tmp[rg][t], a0, a1, a2, a3, b0, b1);
         }
       }
     }
-    if (cur_rb >= 0)
-      ft_flush<TG>(acc, scratch, p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * kFtRows,
-                   rs, bk, lane);
-    if (producer && *abort_flag) {
-      // let the copies still in flight land before the CTA exits
-      const int first = issued > S ? issued - S : 0;
-      for (int l = first; l < issued; ++l) {
-        const uint32_t a = smem_u32(&full[l % S]);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(a, (l / S) & 1) && globaltimer_ns() - t0 < 100000000ull) {
-        }
+#pragma unroll
+    for (int rg = 0; rg < 4; ++rg) {
+      const float s0 = __shfl_sync(0xffffffffu, sm0, 4 * g + rg);
+      const float s1 = __shfl_sync(0xffffffffu, sm1, 4 * g + rg);
+#pragma unroll
+      for (int t = 0; t < TG; ++t) {
+        acc[rg][t][0] = fmaf(tmp[rg][t][0], s0, acc[rg][t][0]);
+        acc[rg][t][1] = fmaf(tmp[rg][t][1], s0, acc[rg][t][1]);
+        acc[rg][t][2] = fmaf(tmp[rg][t][2], s1, acc[rg][t][2]);
+        acc[rg][t][3] = fmaf(tmp[rg][t][3], s1, acc[rg][t][3]);
       }
+    }
+    // leaving the row block (the next item starts another one, or the range ends)
+    if (++kc == p.KC || i + 1 == n_items) {
+      leave_block(rb);
+      kc = 0;
+      ++rb;
     }
   }
-
-  // ------------------------------------------------------------ row-block tickets
+  griddep_wait();   // this grid completes after the down kernel, which the finish kernel relies on
   __syncthreads();
-  griddep_wait();   // T_s and the cleared tickets of the down kernel
-  if (*abort_flag || n_items == 0) return;
-  const int rb_first = it0 / p.KC, rb_last = (it1 - 1) / p.KC;
-  for (int rb = rb_first; rb <= rb_last; ++rb) {
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      const int64_t i0 = static_cast<int64_t>(rb) * p.KC;
-      const int ncontrib = cta_of_item(i0 + p.KC - 1, p.items, p.G) - cta_of_item(i0, p.items, p.G) + 1;
-      const unsigned t = atomicAdd(&p.tickets[rb], 1u);
-      *last_flag = (t == static_cast<unsigned>(ncontrib - 1)) ? 1 : 0;
-    }
-    __syncthreads();
-    if (*last_flag) {
-      __threadfence();
-      ft_finish<NTOK>(p, rb, warp, lane);
+  if (threadIdx.x == 0 && *abort_flag) {
+    // let the copies still in flight land before the CTA exits
+    for (int sj = 0; sj < S; ++sj) {
+      const int j = last_item[sj];
+      if (j < 0) continue;
+      const uint32_t a = smem_u32(&full[sj]);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, (j / S) & 1) && globaltimer_ns() - t0 < 100000000ull) {
+      }
     }
   }
 }
@@ -617,7 +721,7 @@ namespace {
 
 struct FtPlan {
   int ntok, KC, RB, items, G, segmax;
-  size_t part_bytes, ticket_bytes;
+  size_t part_bytes;
 };
 
 FtPlan ft_plan(int64_t M, int64_t d, int64_t k) {
@@ -630,18 +734,47 @@ FtPlan ft_plan(int64_t M, int64_t d, int64_t k) {
   const int per = static_cast<int>(ceil_div(f.items, f.G));
   f.segmax = static_cast<int>(ceil_div(per, f.KC)) + 1;
   f.part_bytes = static_cast<size_t>(f.G) * f.segmax * f.ntok * kFtRows * 4;
-  f.ticket_bytes = static_cast<size_t>(f.RB) * 4;
   return f;
 }
 
-cudaError_t ft_set_smem(const void* fn) {
-  static bool done[2] = {false, false};
-  // one attribute per instantiation; the call is cheap but not free
-  const int idx = fn == reinterpret_cast<const void*>(k_qlora_fewtok<8>) ? 0 : 1;
-  if (done[idx]) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kFtSmemBytes));
-  if (e == cudaSuccess) done[idx] = true;
-  return e;
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// X (M x k bf16) as a 3-D tensor (64 columns, M rows, k / 64 chunks) in boxes
+// of 64 columns x ntok rows x 4 chunks: one item's 256 columns in one copy,
+// stored chunk by chunk (rows >= M read as zero)
+bool map_x(CUtensorMap* m, const uint16_t* X, int64_t M, int64_t k, int ntok) {
+  void* fp = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fp == nullptr)
+    return false;
+  cuuint64_t dims[3] = {64u, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(k / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(k) * 2, 128u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(ntok), 4u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return reinterpret_cast<EncodeTiledFn>(fp)(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(X), dims,
+                                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// c2 (d x kpb int8) in boxes of 16 blocks x 256 rows
+bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d) {
+  void* fp = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fp == nullptr)
+    return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(kpb), static_cast<cuuint64_t>(d)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(kpb)};
+  cuuint32_t box[2] = {16u, static_cast<cuuint32_t>(kFtRows)};
+  cuuint32_t estr[2] = {1, 1};
+  return reinterpret_cast<EncodeTiledFn>(fp)(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(c2), dims,
+                                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -652,22 +785,32 @@ bool fewtok_eligible(int64_t M, int64_t d, int64_t k) {
 
 size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k) {
   const FtPlan f = ft_plan(M, d, k);
-  return align_up(f.part_bytes, 256) + align_up(f.ticket_bytes, 256);
+  return align_up(f.part_bytes, 256);
 }
 
 template <int NTOK>
 static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm, uint16_t* T, float* part,
-                     unsigned* tickets, cudaStream_t st, const char** why) {
+                     cudaStream_t st, const char** why) {
+  CUtensorMap tx, tc2;
+  if (!map_x(&tx, a.X, a.M, a.k, NTOK)) {
+    *why = "tensor map encoding failed (few-token X)";
+    return QLORA_ERR_CUDA;
+  }
+  // c2 through TMA when its rows are 16-byte multiples and its base is 16-byte aligned
+  const int64_t kpb = a.k / 64;
+  const bool c2_tma = a.q->double_quant && kpb % 16 == 0 && (reinterpret_cast<uintptr_t>(a.q->c2) & 15u) == 0 &&
+                      map_c2(&tc2, a.q->c2, kpb, a.d);
+  if (!c2_tma) tc2 = tx;   // unused
   {
     ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    k_lora_down_fewtok<NTOK><<<static_cast<unsigned>(kFtCluster * (a.rp / 8)), 256, 0, st>>>(
-        a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, a.s, T, tickets, f.RB);
+    k_lora_down_fewtok<<<static_cast<unsigned>(kFtCluster * (a.rp / 8)), 256, 0, st>>>(
+        a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, a.s, T);
   }
   if (cudaGetLastError() != cudaSuccess) {
     *why = "few-token down-projection launch";
     return QLORA_ERR_CUDA;
   }
-  if (ft_set_smem(reinterpret_cast<const void*>(k_qlora_fewtok<NTOK>)) != cudaSuccess) {
+  if (set_smem(k_qlora_fewtok<NTOK>, kFtSmemBytes) != cudaSuccess) {
     *why = "smem attribute (few-token)";
     return QLORA_ERR_CUDA;
   }
@@ -683,16 +826,15 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   p.sc.c2 = a.q->c2;
   p.sc.c1 = a.q->c1;
   p.sc.mean = a.q->mean;
-  p.X = a.X;
   p.B = a.B;
   p.T = T;
   p.Y = a.Y;
   p.partial = part;
-  p.tickets = tickets;
   p.items = f.items;
   p.KC = f.KC;
   p.G = f.G;
   p.segmax = f.segmax;
+  p.c2_tma = c2_tma ? 1 : 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(f.G));
   cfg.blockDim = dim3(kFtThreads);
@@ -706,10 +848,20 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   cudaError_t e;
   {
     ProfScope ps_(QLORA_KC_FWD_GEMM, st);
-    e = cudaLaunchKernelEx(&cfg, k_qlora_fewtok<NTOK>, tm, p);
+    e = cudaLaunchKernelEx(&cfg, k_qlora_fewtok<NTOK>, tm, tx, tc2, p);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     *why = "few-token forward launch";
+    return QLORA_ERR_CUDA;
+  }
+  cfg.gridDim = dim3(static_cast<unsigned>(f.RB));
+  cfg.dynamicSmemBytes = 0;
+  {
+    ProfScope ps_(QLORA_KC_AUX, st);
+    e = cudaLaunchKernelEx(&cfg, k_fewtok_finish<NTOK>, p);
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
+    *why = "few-token finish launch";
     return QLORA_ERR_CUDA;
   }
   return 0;
@@ -720,9 +872,8 @@ int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensor
   const FtPlan f = ft_plan(a.M, a.d, a.k);
   char* w = static_cast<char*>(ws);
   float* part = reinterpret_cast<float*>(w);
-  unsigned* tickets = reinterpret_cast<unsigned*>(w + align_up(f.part_bytes, 256));
-  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, tickets, st, why)
-                     : ft_launch<16>(a, f, *tm_codes, T, part, tickets, st, why);
+  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, st, why)
+                     : ft_launch<16>(a, f, *tm_codes, T, part, st, why);
 }
 
 }  // namespace qlora
