@@ -16,8 +16,10 @@
 //     stages; the refill of the stage of item i with item i + S is issued by
 //     warp i mod 16, so issuing costs no single warp more than its share.  The
 //     8-bit block constants c2 come with the first item of each group of four
-//     (16 blocks x 256 rows, two slots); the group constants c1 (or, without
-//     double quantisation, the absmax) are loaded three items ahead.
+//     (16 blocks x 256 rows, two slots).  A row's group constant c1 changes
+//     at most every 256 blocks and is reloaded only when it does.  (Without
+//     TMA-able c2 rows, or without double quantisation, the per-block
+//     constants are loaded one item ahead.)
 //   * A code byte (two weights) is expanded with one shared-memory lookup: a
 //     256-entry table holds the bf16 pair (C[low nibble], C[high nibble]),
 //     replicated per lane (a lane always reads its own bank).  Entries are
@@ -63,7 +65,6 @@ constexpr int kFtMaxStages = 5;
 constexpr uint32_t kFtTableBytes = 65536;
 constexpr uint32_t kFtSmemBytes = 227u * 1024u;             // the whole window; placed in the kernel
 constexpr int kFtCluster = 8;                               // CTAs of one down-projection cluster
-constexpr int kFtScaleAhead = 3;                            // items of block constants in flight
 constexpr uint32_t kFtC2Box = 16u * kFtRows;                // c2 of 16 blocks x 256 rows (four items)
 constexpr int kFtC2Slots = 2;
 
@@ -228,10 +229,11 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p) { return *reinter
 
 // ============================================================================
 // T_s = BF16(s X A^T) for M <= 16 tokens on mma.sync: tokens are the M side
-// (16 rows), 8 ranks the N side.  One cluster of 8 CTAs per group of 8 ranks;
-// CTA q of the cluster covers the q-th eighth of K, its 8 warps take every
-// 8th 16-column step of it, the warps' fragments are added in warp order and
-// CTA 0 adds the eight CTAs' sums in order through distributed shared memory.
+// (16 rows), 8 ranks the N side.  One cluster of 8 CTAs per group of 8 ranks
+// below r; CTA q of the cluster covers the q-th eighth of K, its 8 warps take
+// every 8th 16-column step of it, the warps' fragments are added in warp order
+// and CTA 0 adds the eight CTAs' sums in order through distributed shared
+// memory.  The last cluster also writes the zero columns r .. rp - 1.
 // ============================================================================
 __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
     k_lora_down_fewtok(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int M, int64_t k, int r,
@@ -285,6 +287,12 @@ __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
       if (tok < M && j < rp)
         T[static_cast<int64_t>(tok) * rp + j] =
             static_cast<uint16_t>(pack_bf16x2(j < r ? s * tot[e] : 0.0f, 0.0f) & 0xFFFFu);
+    }
+  }
+  if (q == 0 && blockIdx.x / kFtCluster == gridDim.x / kFtCluster - 1) {
+    for (int i = threadIdx.x; i < M * rp; i += blockDim.x) {
+      const int tok = i / rp, j = i - tok * rp;
+      if (j >= j0 + 8) T[static_cast<int64_t>(tok) * rp + j] = 0;
     }
   }
   cluster_sync_all();   // peers keep their shared memory until CTA 0 has read it
@@ -443,13 +451,6 @@ __global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) 
   ft_finish<NTOK>(p, blockIdx.x, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
-// Block constants of one item for this lane's two rows, loaded ahead of use:
-// c2 bytes (DQ) and validity bits in `w`, c1 (DQ) or absmax in a and b.
-struct FtScaleQ {
-  uint32_t w;
-  float a, b;
-};
-
 template <int NTOK>
 __global__ void __launch_bounds__(kFtThreads, 1)
     k_qlora_fewtok(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
@@ -515,7 +516,6 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
   float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
   const float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;
-  ScaleRecip rec0, rec1;
 
   // ---- TMA issue of item j into stage sj: the code tile, the item's 256
   // columns of X and, at the first item of a group of four, the group's c2
@@ -535,42 +535,65 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   if (threadIdx.x == 0)
     for (int j = 0; j < n_items && j < S; ++j) issue_item(j, j);
 
-  // ---- block constants, kFtScaleAhead items ahead
-  int frb = it0 / p.KC, fkc = it0 - frb * p.KC, fetched = 0;
-  auto fetch = [&]() -> FtScaleQ {
-    FtScaleQ qv{0u, 0.0f, 0.0f};
-    if (fetched < n_items) {
-      const int64_t blk = 4ll * fkc + bk;
-      const int64_t n0 = static_cast<int64_t>(frb) * kFtRows + 64 * rs + 16 * c + g;
-      const bool bv = blk < p.kpb;
-      const bool v0 = bv && (n0 < p.d), v1 = bv && (n0 + 8 < p.d);
-      if (p.sc.dq) {
-        uint32_t c2a = 0, c2b = 0;
-        if (v0) {
-          if (!p.c2_tma) c2a = static_cast<uint8_t>(__ldg(p.sc.c2 + n0 * p.kpb + blk));
-          qv.a = __ldg(p.sc.c1 + ((n0 * p.kpb + blk) >> 8));
-        }
-        if (v1) {
-          if (!p.c2_tma) c2b = static_cast<uint8_t>(__ldg(p.sc.c2 + (n0 + 8) * p.kpb + blk));
-          qv.b = __ldg(p.sc.c1 + (((n0 + 8) * p.kpb + blk) >> 8));
-        }
-        qv.w = c2a | (c2b << 8);
-      } else {
-        if (v0) qv.a = __ldg(p.sc.absmax + n0 * p.kpb + blk);
-        if (v1) qv.b = __ldg(p.sc.absmax + (n0 + 8) * p.kpb + blk);
-      }
-      qv.w |= (v0 ? 1u << 16 : 0u) | (v1 ? 1u << 17 : 0u);
-      if (++fkc == p.KC) {
-        fkc = 0;
-        ++frb;
-      }
-    }
-    ++fetched;
-    return qv;
+  // ---- block constants.  This lane computes s^ for rows 16 c + g and +8 of its
+  // row set and block bk of each item.
+  const bool dq = p.sc.dq != 0, c2_tma = p.c2_tma != 0;
+  // Per row: flat index of block 0 of the row, the current group of 256
+  // blocks and its constant c1 with the correctly rounded reciprocal (s^ =
+  // RN(RN(c2 / c1) + mean) through one residual correction; see nf4_scale.cuh).
+  struct RowConst {
+    int64_t base, grp;
+    float c1, rc;
+    bool fast, valid;
   };
-  FtScaleQ sq[kFtScaleAhead];
+  RowConst rw[2];
+  auto set_rows = [&](int rbx) {
+    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
 #pragma unroll
-  for (int i = 0; i < kFtScaleAhead; ++i) sq[i] = fetch();
+    for (int h = 0; h < 2; ++h) {
+      rw[h].valid = r0 + 8 * h < p.d;
+      rw[h].base = (r0 + 8 * h) * p.kpb;
+      rw[h].grp = -1;
+    }
+  };
+  auto row_scale = [&](RowConst& R, int64_t blk, int c2v) -> float {
+    const int64_t gq = (R.base + blk) >> 8;
+    if (gq != R.grp) {
+      R.grp = gq;
+      R.c1 = __ldg(p.sc.c1 + gq);
+      R.rc = __frcp_rn(R.c1);
+      R.fast = (R.c1 >= 0x1p-60f) && (R.c1 <= 0x1p60f);
+    }
+    const float w = static_cast<float>(c2v);
+    float q;
+    if (R.fast) {
+      const float y = __fmul_rn(w, R.rc);
+      const float e = __fmaf_rn(-R.c1, y, w);
+      q = __fmaf_rn(e, R.rc, y);
+    } else {
+      q = __fdiv_rn(w, R.c1);
+    }
+    return __fadd_rn(q, mean);
+  };
+  // c2 (loaded path) or absmax of the next item
+  uint32_t nc2 = 0;
+  float nab0 = 0.0f, nab1 = 0.0f;
+  auto prefetch = [&](int rbx, int kcx) {
+    if (dq && c2_tma) return;
+    const int64_t blk = 4ll * kcx + bk;
+    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
+    const bool bv = blk < p.kpb;
+    if (dq) {
+      const uint32_t a = (bv && r0 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + r0 * p.kpb + blk)) : 0u;
+      const uint32_t b = (bv && r0 + 8 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + (r0 + 8) * p.kpb + blk)) : 0u;
+      nc2 = a | (b << 8);
+    } else {
+      nab0 = (bv && r0 < p.d) ? __ldg(p.sc.absmax + r0 * p.kpb + blk) : 0.0f;
+      nab1 = (bv && r0 + 8 < p.d) ? __ldg(p.sc.absmax + (r0 + 8) * p.kpb + blk) : 0.0f;
+    }
+  };
+  set_rows(it0 / p.KC);
+  if (n_items > 0) prefetch(it0 / p.KC, it0 - (it0 / p.KC) * p.KC);
 
   float acc[4][TG][4];
 #pragma unroll
@@ -593,11 +616,11 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   int pst = 0;        // stage and parity of the previous item
   uint32_t pph = 0;
   uint32_t c2w0 = 0, c2w1 = 0;   // c2 of this lane's two rows for the four items of the group
+  const bool loaded_consts = !(dq && c2_tma);
   for (int i = 0; i < n_items; ++i) {
-    FtScaleQ cur = sq[0];
-#pragma unroll
-    for (int qi = 0; qi < kFtScaleAhead - 1; ++qi) sq[qi] = sq[qi + 1];
-    sq[kFtScaleAhead - 1] = fetch();
+    const uint32_t cur_c2 = nc2;
+    const float cur_ab0 = nab0, cur_ab1 = nab1;
+    if (loaded_consts && i + 1 < n_items) prefetch(kc + 1 == p.KC ? rb + 1 : rb, kc + 1 == p.KC ? 0 : kc + 1);
 
     mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
     const uint32_t sb = stage(st);
@@ -610,7 +633,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
       c2w0 = prmt(prmt(ra.x, ra.y, sel), prmt(ra.z, ra.w, sel), 0x5410u);
       c2w1 = prmt(prmt(rb8.x, rb8.y, sel), prmt(rb8.z, rb8.w, sel), 0x5410u);
     }
-    if (p.c2_tma) cur.w |= ((c2w0 >> (8 * (kc & 3))) & 0xFFu) | (((c2w1 >> (8 * (kc & 3))) & 0xFFu) << 8);
+
     uint2 cw[4][2];
 #pragma unroll
     for (int rg = 0; rg < 4; ++rg)
@@ -627,7 +650,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
       mbar_arrive(&empty[st]);
       // this warp's turn: refill the stage of item i - 1 (released by every
       // warp one item ago) with item i - 1 + S
-      if (i > 0 && (i & (kFtWarps - 1)) == warp && i - 1 + S < n_items && !*abort_flag &&
+      if (i > 0 && (i & (kFtWarps - 1)) == warp && i - 1 + S < n_items &&
           mbar_wait(&empty[pst], pph, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT))
         issue_item(i - 1 + S, pst);
     }
@@ -639,17 +662,18 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     }
 
     float sm0 = 0.0f, sm1 = 0.0f;
-    if (cur.w & (1u << 16)) {
-      ScaleRaw r0;
-      r0.a = cur.a;
-      r0.b = static_cast<int>(static_cast<int8_t>(cur.w & 0xFFu));
-      sm0 = scale_value(p.sc.dq, mean, r0, rec0);
-    }
-    if (cur.w & (1u << 17)) {
-      ScaleRaw r1;
-      r1.a = cur.b;
-      r1.b = static_cast<int>(static_cast<int8_t>((cur.w >> 8) & 0xFFu));
-      sm1 = scale_value(p.sc.dq, mean, r1, rec1);
+    {
+      const int64_t blk = 4ll * kc + bk;
+      const bool bv = blk < p.kpb;
+      if (dq) {
+        const uint32_t c2p = c2_tma ? (((c2w0 >> (8 * (kc & 3))) & 0xFFu) | (((c2w1 >> (8 * (kc & 3))) & 0xFFu) << 8))
+                                    : cur_c2;
+        if (bv && rw[0].valid) sm0 = row_scale(rw[0], blk, static_cast<int>(static_cast<int8_t>(c2p & 0xFFu)));
+        if (bv && rw[1].valid) sm1 = row_scale(rw[1], blk, static_cast<int>(static_cast<int8_t>(c2p >> 8)));
+      } else {
+        sm0 = bv && rw[0].valid ? cur_ab0 : 0.0f;
+        sm1 = bv && rw[1].valid ? cur_ab1 : 0.0f;
+      }
     }
     // four independent accumulation chains (one per 16-row group)
     float tmp[4][TG][4];
@@ -697,6 +721,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
       leave_block(rb);
       kc = 0;
       ++rb;
+      set_rows(rb);
     }
   }
   griddep_wait();   // this grid completes after the down kernel, which the finish kernel relies on
@@ -803,7 +828,7 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   if (!c2_tma) tc2 = tx;   // unused
   {
     ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    k_lora_down_fewtok<<<static_cast<unsigned>(kFtCluster * (a.rp / 8)), 256, 0, st>>>(
+    k_lora_down_fewtok<<<static_cast<unsigned>(kFtCluster * ceil_div(a.r, 8)), 256, 0, st>>>(
         a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, a.s, T);
   }
   if (cudaGetLastError() != cudaSuccess) {
