@@ -31,11 +31,12 @@
 //   k_qlora_main<FwdSwap> few tokens (M <= 128): W rows are the MMA's M side
 //                         (128 per tile), the tokens its N side, so the tensor
 //                         core is not padded to 128 tokens; split over K.
-//   k_thin<false,*>       T_s and U_s partial sums (K-major activations; A read
-//                         K-major, B read MN-major straight from its storage).
-//   k_thin<true,true>     dA^T and dB partial sums (MN-major operands, the
-//                         reduction runs over tokens).
-//   k_reduce_*            deterministic sums of split-K partials.
+//   k_thin<false,*>       T_s and U_s (K-major activations; A read K-major, B
+//                         read MN-major straight from its storage).
+//   k_thin<true,true>     dA and dB (MN-major operands, the reduction runs over
+//                         tokens).  The K splits of a tile form a cluster and are
+//                         added in shared memory.
+//   k_reduce_bf16         deterministic sum of the main GEMM's split-K partials.
 #include <cstdio>
 #include <cstring>
 #include <map>
@@ -50,6 +51,24 @@
 namespace qlora {
 
 
+
+// ============================================================================
+// Cluster helpers
+// ============================================================================
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// 16 bytes at the same shared-memory offset in CTA `rank` of the cluster
+__device__ __forceinline__ float4 ld_cluster_f4(uint32_t local_addr, uint32_t rank) {
+  uint32_t remote;
+  float4 v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(remote)
+               : "memory");
+  return v;
+}
 
 // ============================================================================
 // Tensor maps
@@ -587,17 +606,33 @@ __global__ void __launch_bounds__(576, 1)
 }
 
 // ============================================================================
-// Thin GEMM: D[128 x rp] += A_tile * B_tile^T over a K range, fp32 partials.
+// Thin GEMM: D[128 x rp] = A_tile * B_tile^T over K.
 //   kMN = false: A, B K-major (T_s: X and A; U_s: dY and B^T).
 //   kMN = true : A, B MN-major, reduction over tokens (dA^T: X^T and U_s;
 //                dB: dY^T and T_s).
+// K is split over the CTAs of one thread-block cluster (blockIdx.y = rank,
+// at most 8).  Each CTA parks its fp32 tile in its own shared memory; after a
+// cluster barrier CTA q adds rows [q 128 / S, (q + 1) 128 / S) of the S tiles
+// in rank order through distributed shared memory and writes the result, so
+// no partial sums go through HBM and the sum order is fixed.
 // ============================================================================
+enum ThinOut : int {
+  THIN_BF16 = 0,   // out16[row][j] = BF16(scale * D)       (T_s, U_s; rp columns)
+  THIN_DA = 1,     // outf[j][row]  = D for j < r           (dA from dA^T; row stride `ld`)
+  THIN_DB = 2,     // outf[row][j]  = D for j < r           (dB; row stride r)
+};
+
 struct ThinParams {
   int64_t rows;          // output rows in total (M, k or d)
   int32_t rp;            // output columns (multiple of 64)
   int32_t steps;         // K steps in total
   int32_t steps_per_split;
-  float* partial;        // [splits][rows][rp]
+  int32_t mode;          // ThinOut
+  int32_t r;
+  int64_t ld;            // THIN_DA: row stride of dA (= k)
+  float scale;
+  uint16_t* out16;
+  float* outf;
 };
 
 struct ThinCfg {
@@ -712,29 +747,76 @@ __global__ void __launch_bounds__(128, 2)
   }
   __syncwarp();
 
-  // epilogue: all four warps (warp w owns TMEM lanes 32w..32w+31)
+  // epilogue, 1: every warp moves its 32 TMEM lanes (rows) into this CTA's
+  // fp32 tile in shared memory, over the now idle stages (rows padded by 4
+  // floats so that a quarter-warp's 16-byte stores hit distinct banks)
   const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
+  __syncthreads();   // the producer has drained any copy still in flight into the stages
   tc_fence_after();
-  if (ok) {
-    const int64_t row = row0 + 32 * warp + lane;
+  const uint32_t ldr = static_cast<uint32_t>(rp + 4);   // floats per tile row
+  float* red = reinterpret_cast<float*>(base);
+  {
+    const int trow = 32 * warp + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
     for (int cb = 0; cb < rp / 32; ++cb) {
       uint32_t v[32];
       tmem_ld32(lane_base + 32 * cb, v);
       tmem_ld_wait();
-      if (row < p.rows) {
-        float* dst = p.partial + (static_cast<int64_t>(split) * p.rows + row) * rp + 32 * cb;
-        if (n_local == 0) {
+      float* dst = red + trow * ldr + 32 * cb;
+      const bool zero = !ok || n_local == 0;
 #pragma unroll
-          for (int g = 0; g < 8; ++g) *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(0, 0, 0, 0);
-        } else {
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<uint4*>(dst + 4 * g) =
+            zero ? make_uint4(0, 0, 0, 0) : make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    }
+  }
+  // 2: every CTA of the cluster has parked its tile (all CTAs always take both
+  // cluster barriers, also on the abort path)
+  cluster_sync_all();
+  // 3: this CTA adds its row slice of the cluster's tiles in rank order
+  {
+    const int S2 = static_cast<int>(gridDim.y);
+    const int q = static_cast<int>(blockIdx.y);
+    const int r0 = q * 128 / S2, r1 = (q + 1) * 128 / S2, nr = r1 - r0;
+    const int c4n = rp / 4;
+    const uint32_t red_addr = smem_u32(red);
+    for (int idx = threadIdx.x; idx < nr * c4n; idx += blockDim.x) {
+      // dA writes transposed rows: consecutive threads take consecutive rows
+      const int rr = (p.mode == THIN_DA) ? r0 + idx % nr : r0 + idx / c4n;
+      const int c4 = (p.mode == THIN_DA) ? idx / nr : idx % c4n;
+      const uint32_t off = (static_cast<uint32_t>(rr) * ldr + 4u * static_cast<uint32_t>(c4)) * 4u;
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int pr = 0; pr < S2; ++pr) {
+        const float4 v = ld_cluster_f4(red_addr + off, static_cast<uint32_t>(pr));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      const int64_t row = row0 + rr;
+      if (row >= p.rows) continue;
+      const int j0 = 4 * c4;
+      if (p.mode == THIN_BF16) {
+        uint2 o;
+        o.x = pack_bf16x2(acc.x * p.scale, acc.y * p.scale);
+        o.y = pack_bf16x2(acc.z * p.scale, acc.w * p.scale);
+        *reinterpret_cast<uint2*>(p.out16 + row * rp + j0) = o;
+      } else {
+        const float e[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+        for (int u = 0; u < 4; ++u) {
+          if (j0 + u < p.r) {
+            if (p.mode == THIN_DA)
+              p.outf[static_cast<int64_t>(j0 + u) * p.ld + row] = e[u];
+            else
+              p.outf[row * p.r + j0 + u] = e[u];
+          }
         }
       }
     }
   }
+  // 4: peers keep their tiles until every CTA of the cluster has read them
+  cluster_sync_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -762,43 +844,6 @@ __global__ void k_reduce_bf16(const float* __restrict__ partial, int splits, int
     o.x = pack_bf16x2(acc.x * scale, acc.y * scale);
     o.y = pack_bf16x2(acc.z * scale, acc.w * scale);
     reinterpret_cast<uint2*>(out)[i] = o;
-  }
-}
-
-// dB[n][j] = sum_s partial[s][n][j] for j < r   (partial rows are rp wide)
-__global__ void k_reduce_dB(const float* __restrict__ partial, int splits, int64_t d, int rp, int r,
-                            float* __restrict__ dB) {
-  const int64_t count = d * r;
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = i / r;
-    const int j = static_cast<int>(i - n * r);
-    float acc = 0.0f;
-    for (int s = 0; s < splits; ++s) acc += partial[(s * d + n) * rp + j];
-    dB[i] = acc;
-  }
-}
-
-// dA[j][c] = sum_s partial[s][c][j]  (partial holds dA^T, rows = k columns)
-__global__ void k_reduce_dA(const float* __restrict__ partial, int splits, int64_t k, int rp, int r,
-                            float* __restrict__ dA) {
-  __shared__ float tile[32][33];
-  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * 32;
-  const int j0 = blockIdx.y * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-  for (int yy = ty; yy < 32; yy += 8) {
-    const int64_t c = c0 + yy;
-    const int j = j0 + tx;
-    float acc = 0.0f;
-    if (c < k && j < rp)
-      for (int s = 0; s < splits; ++s) acc += partial[(s * k + c) * rp + j];
-    tile[yy][tx] = acc;
-  }
-  __syncthreads();
-  for (int yy = ty; yy < 32; yy += 8) {
-    const int j = j0 + yy;
-    const int64_t c = c0 + tx;
-    if (j < r && c < k) dA[static_cast<int64_t>(j) * k + c] = tile[tx][yy];
   }
 }
 
@@ -859,6 +904,7 @@ static int plan_thin_splits(int64_t tiles, int steps, int rp) {
   if (s < 1) s = 1;
   const int64_t cap = steps / 8 > 1 ? steps / 8 : 1;
   if (s > cap) s = cap;
+  if (s > 8) s = 8;   // the splits form one thread-block cluster (portable size)
   return static_cast<int>(s);
 }
 
@@ -870,7 +916,7 @@ struct Plan {
   int nt;   // swap token tile (0 = non-swap)
   bool fewtok;   // forward through the few-token kernels
   // workspace offsets (bytes)
-  size_t off_T, off_partT, off_Bt, off_U, off_partU, off_partA, off_partB, off_main, total;
+  size_t off_T, off_Bt, off_U, off_main, total;
 };
 
 // Few-token forward: the kernel streams weights, so keep every SM busy until
@@ -912,7 +958,6 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     return o;
   };
   pl.off_T = need_T ? take(static_cast<size_t>(M) * rp * 2) : 0;
-  pl.off_partT = need_T ? take(static_cast<size_t>(pl.splits_T) * M * rp * 4) : 0;
   if (!bwd && fewtok_eligible(M, d, k)) {
     pl.fewtok = true;
     pl.off_main = take(fewtok_workspace_bytes(M, d, k));
@@ -931,12 +976,9 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     pl.splits_U = plan_thin_splits(mt, dsteps, rp);
     pl.off_Bt = take(static_cast<size_t>(rp) * d * 2);
     pl.off_U = take(static_cast<size_t>(M) * rp * 2);
-    pl.off_partU = take(static_cast<size_t>(pl.splits_U) * M * rp * 4);
     const int msteps = static_cast<int>(ceil_div(M, 64));
     pl.splits_dA = plan_thin_splits(ceil_div(k, 128), msteps, rp);
     pl.splits_dB = plan_thin_splits(ceil_div(d, 128), msteps, rp);
-    pl.off_partA = take(static_cast<size_t>(pl.splits_dA) * k * rp * 4);
-    pl.off_partB = take(static_cast<size_t>(pl.splits_dB) * d * rp * 4);
     pl.main_splits = plan_splits(ceil_div(k, 256) * ceil_div(M, 256), dsteps, 8, 1);
     pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * k * 4) : 0;
   }
@@ -972,9 +1014,48 @@ static int grid1d(int64_t work, int per_block) {
 // b_mn = false: bmat is (brows x K) row-major, read K-major (A of the layer).
 // b_mn = true : bmat is (K x brows) row-major, read MN-major (B of the layer,
 //               K = d, N = r), which needs brows * 2 bytes to be a multiple of 16.
+// One low-rank GEMM: grid (row tiles, K splits), the splits of a row tile
+// forming one cluster that reduces in shared memory.
+template <bool kAMN, bool kBMN>
+static int launch_thin(const CUtensorMap& ta, const CUtensorMap& tb, ThinParams tp, int64_t tiles, int splits,
+                       cudaStream_t st, const char** why) {
+  tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, splits));
+  const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
+  const uint32_t smem = ThinCfg::smem_bytes(tp.rp);
+  if (set_smem(k_thin<kAMN, kBMN>, smem) != cudaSuccess) {
+    *why = "smem attribute (thin GEMM)";
+    return QLORA_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(real));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(real);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  {
+    ProfScope ps_(QLORA_KC_LORA_GEMM, st);
+    e = cudaLaunchKernelEx(&cfg, k_thin<kAMN, kBMN>, ta, tb, tp);
+  }
+  if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
+    *why = "thin GEMM launch";
+    return QLORA_ERR_CUDA;
+  }
+  return 0;
+}
+
+// T_s = BF16(s X A^T) (or U_s = BF16(s dY B) with `act` = dY and `bmat` = B^T)
+// b_mn = false: bmat is (brows x K) row-major, read K-major (A of the layer).
+// b_mn = true : bmat is (K x brows) row-major, read MN-major (B of the layer,
+//               K = d, N = r), which needs brows * 2 bytes to be a multiple of 16.
 static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uint16_t* bmat, int64_t brows,
-                            bool b_mn, int rp, float s, int splits, float* partial, uint16_t* out, cudaStream_t st,
-                            const char** why) {
+                            bool b_mn, int rp, float s, int splits, uint16_t* out, cudaStream_t st, const char** why) {
   CUtensorMap ta, tb;
   const bool okb = b_mn ? map_bf16(&tb, bmat, brows, K, 64, 64) : map_bf16(&tb, bmat, K, brows, 64, rp);
   if (!map_bf16(&ta, act, K, M, 64, 128) || !okb) {
@@ -985,30 +1066,11 @@ static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uin
   tp.rows = M;
   tp.rp = rp;
   tp.steps = static_cast<int>(ceil_div(K, 64));
-  tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, splits));
-  tp.partial = partial;
-  const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-  const uint32_t smem = ThinCfg::smem_bytes(rp);
-  if ((b_mn ? set_smem(k_thin<false, true>, smem) : set_smem(k_thin<false, false>, smem)) != cudaSuccess) {
-    *why = "smem attribute";
-    return QLORA_ERR_CUDA;
-  }
-  dim3 grid(static_cast<unsigned>(ceil_div(M, 128)), static_cast<unsigned>(real));
-  {
-    ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    if (b_mn)
-      k_thin<false, true><<<grid, 128, smem, st>>>(ta, tb, tp);
-    else
-      k_thin<false, false><<<grid, 128, smem, st>>>(ta, tb, tp);
-  }
-  QL_CHECK_LAUNCH("thin GEMM launch");
-  const int64_t count = M * rp;
-  {
-    ProfScope ps_(QLORA_KC_AUX, st);
-    k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(partial, real, count, s, out);
-  }
-  QL_CHECK_LAUNCH("reduce launch");
-  return 0;
+  tp.mode = THIN_BF16;
+  tp.scale = s;
+  tp.out16 = out;
+  return b_mn ? launch_thin<false, true>(ta, tb, tp, ceil_div(M, 128), splits, st, why)
+              : launch_thin<false, false>(ta, tb, tp, ceil_div(M, 128), splits, st, why);
 }
 
 template <Mode MODE, int NT>
@@ -1053,8 +1115,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     }
     return launch_fewtok_fwd(a, T, ws + pl.off_main, &tm, st, why);
   }
-  float* partT = reinterpret_cast<float*>(ws + pl.off_partT);
-  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, a.s, pl.splits_T, partT, T, st, why);
+  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, a.s, pl.splits_T, T, st, why);
   if (rc) return rc;
 
   const qlora_nf4_t& q = *a.q;
@@ -1130,8 +1191,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   const uint16_t* T = a.Tin;
   if (!T) {
     uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + pl.off_T);
-    rc = run_lowrank_down(a.X, M, k, a.A, r, false, rp, a.s, pl.splits_T, reinterpret_cast<float*>(ws + pl.off_partT),
-                          Tw, st, why);
+    rc = run_lowrank_down(a.X, M, k, a.A, r, false, rp, a.s, pl.splits_T, Tw, st, why);
     if (rc) return rc;
     T = Tw;
   }
@@ -1140,8 +1200,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   // K-major copy B^T (rp x d) is made first.
   uint16_t* U = reinterpret_cast<uint16_t*>(ws + pl.off_U);
   if (r % 8 == 0) {
-    rc = run_lowrank_down(a.dY, M, d, a.B, r, true, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU),
-                          U, st, why);
+    rc = run_lowrank_down(a.dY, M, d, a.B, r, true, rp, a.s, pl.splits_U, U, st, why);
   } else {
     uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
     {
@@ -1150,8 +1209,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
           a.B, d, r, rp, Bt);
     }
     QL_CHECK_LAUNCH("transpose launch");
-    rc = run_lowrank_down(a.dY, M, d, Bt, rp, false, rp, a.s, pl.splits_U, reinterpret_cast<float*>(ws + pl.off_partU),
-                          U, st, why);
+    rc = run_lowrank_down(a.dY, M, d, Bt, rp, false, rp, a.s, pl.splits_U, U, st, why);
   }
   if (rc) return rc;
 
@@ -1202,25 +1260,12 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.rows = k;
     tp.rp = rp;
     tp.steps = static_cast<int>(ceil_div(M, 64));
-    tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dA));
-    tp.partial = reinterpret_cast<float*>(ws + pl.off_partA);
-    const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-    if (set_smem(k_thin<true, true>, ThinCfg::smem_bytes(rp)) != cudaSuccess) {
-      *why = "smem attribute (thin MN)";
-      return QLORA_ERR_CUDA;
-    }
-    {
-      ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-      k_thin<true, true><<<dim3(static_cast<unsigned>(ceil_div(k, 128)), static_cast<unsigned>(real)), 128,
-                           ThinCfg::smem_bytes(rp), st>>>(ta, tb, tp);
-    }
-    QL_CHECK_LAUNCH("dA GEMM launch");
-    {
-      ProfScope ps_(QLORA_KC_AUX, st);
-      k_reduce_dA<<<dim3(static_cast<unsigned>(ceil_div(k, 32)), static_cast<unsigned>(ceil_div(r, 32))), 256, 0, st>>>(
-        tp.partial, real, k, rp, r, a.dA);
-    }
-    QL_CHECK_LAUNCH("dA reduce launch");
+    tp.mode = THIN_DA;
+    tp.r = r;
+    tp.ld = k;
+    tp.outf = a.dA;
+    rc = launch_thin<true, true>(ta, tb, tp, ceil_div(k, 128), pl.splits_dA, st, why);
+    if (rc) return rc;
   }
   {
     CUtensorMap ta, tb;
@@ -1232,20 +1277,11 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.rows = d;
     tp.rp = rp;
     tp.steps = static_cast<int>(ceil_div(M, 64));
-    tp.steps_per_split = static_cast<int>(ceil_div(tp.steps, pl.splits_dB));
-    tp.partial = reinterpret_cast<float*>(ws + pl.off_partB);
-    const int real = static_cast<int>(ceil_div(tp.steps, tp.steps_per_split));
-    {
-      ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-      k_thin<true, true><<<dim3(static_cast<unsigned>(ceil_div(d, 128)), static_cast<unsigned>(real)), 128,
-                           ThinCfg::smem_bytes(rp), st>>>(ta, tb, tp);
-    }
-    QL_CHECK_LAUNCH("dB GEMM launch");
-    {
-      ProfScope ps_(QLORA_KC_AUX, st);
-      k_reduce_dB<<<grid1d(d * r, 256), 256, 0, st>>>(tp.partial, real, d, rp, r, a.dB);
-    }
-    QL_CHECK_LAUNCH("dB reduce launch");
+    tp.mode = THIN_DB;
+    tp.r = r;
+    tp.outf = a.dB;
+    rc = launch_thin<true, true>(ta, tb, tp, ceil_div(d, 128), pl.splits_dB, st, why);
+    if (rc) return rc;
   }
   return 0;
 }
