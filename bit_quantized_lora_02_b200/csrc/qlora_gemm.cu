@@ -606,6 +606,430 @@ __global__ void __launch_bounds__(576, 1)
 }
 
 // ============================================================================
+// Paired fused kernel: tcgen05.mma.cta_group::2.
+//
+// Two CTAs of a cluster (ranks 0 and 1, adjacent 256-token tiles) share one
+// MMA of M = 256 (128 token rows from each CTA) and N = 256 weight rows
+// (forward) or input columns (backward), of which each CTA holds and
+// dequantises one half.  With two accumulators per CTA a pair covers 512 tokens
+// x 256 columns, so every dequantised weight feeds 512 tokens and each CTA
+// expands half the weights per K step of the single-CTA kernel for the same
+// tensor work.
+//
+//   * Each CTA loads its own activation tile and its half of the codes (TMA,
+//     local barriers) and dequantises its half of W into its own shared memory.
+//   * Two dequant groups of 8 warps take alternate K steps; when a group's W
+//     half is written it arrives on the rank-0 CTA's wready barrier (remotely
+//     from rank 1), after having waited for its own TMA stage, so the barrier
+//     completing means both halves of W and both activation tiles are there.
+//   * One thread of rank 0 issues the MMAs for both CTAs; its commits arrive on
+//     the stage / W-buffer / accumulator barriers of both CTAs (multicast).
+//   * TMEM is allocated and freed by warp 1 of both CTAs together.
+// ============================================================================
+template <bool BWD>
+struct PairCfg {
+  static constexpr int kWRows = BWD ? 64 : 128;          // this CTA's half of the W tile per K step
+  static constexpr int kWCols = BWD ? 128 : 64;
+  static constexpr uint32_t kActBytes = 256u * 128u;     // 256 tokens x 64 K, bf16
+  static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
+  static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
+  static constexpr uint32_t kStageBytes = kActBytes + kCodeBytes;
+  static constexpr int kWBufs = 4;                       // two groups writing, one waiting, one read
+  static constexpr uint32_t kFixedBytes = kWBufs * kWBytes + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int kStagesRaw = static_cast<int>((227u * 1024u - kFixedBytes) / kStageBytes);
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static_assert(kStages >= 3, "shared memory for at least three TMA stages");
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kFixedBytes;
+  static constexpr int kGroups = 2, kGroupThreads = 256, kTPB = 2, kCPT = 4;
+  static constexpr int kThreads = 576;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kIdesc = make_idesc_bf16(256, 256, false, BWD);
+};
+
+__device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive (once) on the mbarrier at this offset in both CTAs of the pair when
+// every MMA issued so far by this thread has completed.
+__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
+  const uint16_t mask = 3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+// Arrive on the mbarrier at this offset in cluster CTA `rank`.
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// mbar_wait for barriers that another CTA of the cluster arrives on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int code) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait_cluster(a, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cluster(a, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        report(code);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+template <bool BWD>
+__global__ void __launch_bounds__(576, 1)
+    k_qlora_pair(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+                 const __grid_constant__ CUtensorMap tm_ext, const MainParams p) {
+  using Cfg = PairCfg<BWD>;
+  constexpr int S = Cfg::kStages;
+  constexpr int SW = Cfg::kWBufs;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  uint8_t* wbase = base + S * Cfg::kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SW * Cfg::kWBytes);
+  uint64_t* full_bar = bars;                // this CTA's TMA stage landed (act + codes)
+  uint64_t* empty_bar = bars + S;           // the MMAs reading the stage completed (both CTAs)
+  uint64_t* wready_bar = bars + 2 * S;      // rank 0 only: both halves of W written
+  uint64_t* wfree_bar = bars + 2 * S + SW;  // the MMAs reading the W buffer completed (both CTAs)
+  uint64_t* tmem_full = bars + 2 * S + 2 * SW;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tmem_full + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_full + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  // the two CTAs of a pair are neighbours along x (peer CTAs of cta_group::2)
+  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 256;   // output columns of the pair
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 256;   // this CTA's tokens
+  const int64_t h0 = n0 + 128 * static_cast<int64_t>(rank);     // this CTA's half of the columns
+  const int split = blockIdx.z;
+  const int s_begin = split * p.steps_per_split;
+  const int s_end = min(p.steps_main, s_begin + p.steps_per_split);
+  const int n_main = max(0, s_end - s_begin);
+  const int n_local = n_main + (split == 0 ? p.ext_steps : 0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < SW; ++i) {
+      mbar_init(&wready_bar[i], 2 * (Cfg::kGroupThreads / 32));   // one group's warps of both CTAs
+      mbar_init(&wfree_bar[i], 1);
+    }
+    mbar_init(tmem_full, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_act);
+    tma_prefetch_desc(&tm_codes);
+    tma_prefetch_desc(&tm_ext);
+  }
+  // both CTAs' barriers exist before either CTA arrives on the other's
+  __syncthreads();
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (warp == 1) {
+    tmem_alloc2(tmem_slot, Cfg::kTmemCols);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
+  auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
+  auto w_tile = [&](int sw) { return wbase + sw * Cfg::kWBytes; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int issued = 0;
+      for (int l = 0; l < n_local; ++l) {
+        const int st = l % S;
+        const uint32_t ph = (l / S) & 1;
+        if (!mbar_wait_cluster(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
+        if (l < n_main) {
+          const int i = s_begin + l;
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes + Cfg::kCodeBytes);
+          tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
+          if (BWD)
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], static_cast<int>(h0 / 2), 64 * i);
+          else
+            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(h0));
+        } else {
+          const int e = l - n_main;
+          mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes);
+          tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, static_cast<int>(m0));
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        const int first = issued > S ? issued - S : 0;
+        for (int l = first; l < issued; ++l) {
+          const uint32_t a = smem_u32(&full_bar[l % S]);
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(a, (l / S) & 1) && globaltimer_ns() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (rank 0 only)
+    if (lane == 0 && rank == 0) {
+      for (int l = 0; l < n_local; ++l) {
+        const int st = l % S;
+        const uint32_t ph = (l / S) & 1;
+        const int sw = l % SW;
+        const uint32_t phw = (l / SW) & 1;
+        if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
+        if (!mbar_wait_cluster(&wready_bar[sw], phw, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
+        tc_fence_after();
+        const uint32_t a_act = smem_u32(act_tile(st));
+        const uint32_t a_w = smem_u32(w_tile(sw));
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t da = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
+          const uint64_t db = BWD ? make_sdesc_sw128(a_w + 2048u * kk, 8192u, 1024u)
+                                  : make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
+          const uint32_t acc = (l > 0 || kk > 0) ? 1u : 0u;
+          umma2_bf16(tmem_base, da, db, Cfg::kIdesc, acc);
+          // token rows 128..255 of each CTA: second accumulator, same W
+          const uint64_t da1 = make_sdesc_sw128(a_act + 16384u + 32u * kk, 16u, 1024u);
+          umma2_bf16(tmem_base + 256u, da1, db, Cfg::kIdesc, acc);
+        }
+        umma2_commit_both(&empty_bar[st]);
+        umma2_commit_both(&wfree_bar[sw]);
+      }
+      umma2_commit_both(tmem_full);   // also drains MMAs on the abort path
+    }
+  } else {
+    // ------------------------------------------------------------ dequant warps (both CTAs)
+    constexpr int G = Cfg::kGroups, TPB = Cfg::kTPB, CPT = Cfg::kCPT;
+    const int t = threadIdx.x - 64;            // 0..511
+    const int grp = t / Cfg::kGroupThreads;
+    const int tgt = t % Cfg::kGroupThreads;
+    const int tg = tgt / TPB;                  // block of the step (0..127)
+    const int c_first = (tgt % TPB) * CPT;     // first 16-byte chunk of this thread
+    constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
+    float C[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
+    const ScaleSrc sc = p.sc;
+    const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
+    //   Fwd: row = W row of this CTA's half (0..127)
+    //   Bwd: row = W row within the 64-row K step, sub = 64-column chunk of this CTA's half
+    const int row = BWD ? (tg & 63) : tg;
+    const int sub = BWD ? (tg >> 6) : 0;
+    const uint32_t w_off = BWD ? 8192u * sub : 0u;
+    // code rows: 32 B (Fwd, plain), 64 B (Bwd, TMA 64-byte swizzle: 16-byte
+    // chunk j of row r sits at j ^ ((r >> 1) & 3))
+    constexpr uint32_t kCodeRow = BWD ? 64u : 32u;
+    const uint32_t c_row = row * kCodeRow;
+    const uint32_t lc0 = (BWD ? 2u * sub : 0u) + static_cast<uint32_t>(c_first / 4);
+    const uint32_t c_xor = BWD ? ((row >> 1) & 3u) : 0u;
+    auto block_of = [&](int i, bool& valid) -> int64_t {
+      int64_t wr, bc;
+      if (BWD) {
+        wr = 64ll * i + row;
+        bc = h0 / 64 + sub;
+      } else {
+        wr = h0 + row;
+        bc = i;
+      }
+      valid = (wr < p.d) && (bc < p.kpb);
+      return wr * p.kpb + bc;
+    };
+    ScaleRaw pre0{}, pre1{};
+    ScaleRecip recip;
+    bool pre0_valid = false, pre1_valid = false;
+    if (grp < n_main) {
+      const int64_t b0 = block_of(s_begin + grp, pre0_valid);
+      if (pre0_valid) pre0 = scale_fetch(sc, b0);
+    }
+    if (grp + G < n_main) {
+      const int64_t b1 = block_of(s_begin + grp + G, pre1_valid);
+      if (pre1_valid) pre1 = scale_fetch(sc, b1);
+    }
+    for (int l = grp; l < n_local; l += G) {
+      const int st = l % S;
+      const uint32_t ph = (l / S) & 1;
+      const int sw = l % SW;
+      const uint32_t phw = (l / SW) & 1;
+      bool okw = mbar_wait_cluster(&wfree_bar[sw], phw ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
+      okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      const uint32_t wt = smem_u32(w_tile(sw)) + w_off;
+      if (l < n_main) {
+        const ScaleRaw cur = pre0;
+        const bool cur_valid = pre0_valid;
+        pre0 = pre1;
+        pre0_valid = pre1_valid;
+        if (l + 2 * G < n_main) {
+          const int64_t bn = block_of(s_begin + l + 2 * G, pre1_valid);
+          if (pre1_valid) pre1 = scale_fetch(sc, bn);
+        }
+        const uint32_t ctile = smem_u32(code_tile(st)) + c_row;
+        uint32_t w8[CPT];
+#pragma unroll
+        for (int h = 0; h < CPT / 4; ++h) {
+          const uint4 cw = lds128(ctile + 16u * ((lc0 + h) ^ c_xor));
+          w8[4 * h] = cw.x;
+          w8[4 * h + 1] = cw.y;
+          w8[4 * h + 2] = cw.z;
+          w8[4 * h + 3] = cw.w;
+        }
+        if (cur_valid) {
+          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur, recip), C);
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w8[c], tab));
+        } else {
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), make_uint4(0, 0, 0, 0));
+        }
+      } else {
+        // LoRA extension step (64 wide): this CTA's half of the adapter into the W tile
+        const int e = l - n_main;
+        if (BWD) {
+          // A (r x k): K row j = 64e + row, N columns h0 + 64 sub + [0, 64)
+          const int64_t j = 64ll * e + row;
+          const int64_t col = h0 + 64 * sub;
+          const bool v = (j < p.r) && (col < p.k);
+          const uint16_t* srcp = p.lora + j * p.k + col;
+#pragma unroll
+          for (int c = c_first; c < c_first + CPT; ++c) {
+            uint4 val = make_uint4(0, 0, 0, 0);
+            if (v) val = __ldg(reinterpret_cast<const uint4*>(srcp + 8 * c));
+            sts128(wt + sw128_offset(row, c), val);
+          }
+        } else {
+          // B (d x r): row n, columns 64e + [0, 64)
+          const int64_t n = h0 + row;
+#pragma unroll
+          for (int c = c_first; c < c_first + CPT; ++c) {
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int64_t j = 64ll * e + 8 * c + q;
+              h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
+            }
+            sts128(wt + sw128_offset(row, c),
+                   make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&wready_bar[sw]);
+        else
+          mbar_arrive_cluster(&wready_bar[sw], 0);
+      }
+    }
+
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_cluster(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
+    tc_fence_after();
+    if (ok) {
+      const int q = warp & 3;
+      const int idx = (warp - 2) >> 2;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
+      const int acc = idx >> 1;                       // which 128-token half of this CTA's tile
+      const int64_t m = m0 + 128 * acc + 32 * q + lane;
+      for (int cb = 0; cb < 4; ++cb) {
+        const int col0 = 128 * (idx & 1) + 32 * cb;
+        uint32_t v[32];
+        tmem_ld32(lane_base + 256u * acc + col0, v);
+        tmem_ld_wait();
+        if (m < p.M) {
+          const int64_t n = n0 + col0;
+          if (p.splits == 1) {
+            uint16_t* dst = p.out + m * p.n_out + n;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              if (n + 8 * g + 8 <= p.n_out) {
+                uint4 o;
+                o.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
+                o.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
+                o.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
+                o.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
+                *reinterpret_cast<uint4*>(dst + 8 * g) = o;
+              }
+            }
+          } else {
+            float* dst = p.partial + (static_cast<int64_t>(split) * p.M + m) * p.n_out + n;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+              if (n + 4 * g + 4 <= p.n_out)
+                *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  if (warp == 1 && lane == 0) {
+    // this CTA's accumulator must be idle before the pair's columns are released
+    const uint32_t a = smem_u32(tmem_full);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait_cluster(a, 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  // neither CTA leaves while the other's MMAs or remote arrivals may still
+  // touch its shared memory
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// ============================================================================
 // Thin GEMM: D[128 x rp] = A_tile * B_tile^T over K.
 //   kMN = false: A, B K-major (T_s: X and A; U_s: dY and B^T).
 //   kMN = true : A, B MN-major, reduction over tokens (dA^T: X^T and U_s;
@@ -967,7 +1391,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     if (pl.nt) {
       pl.main_splits = plan_swap_splits(ceil_div(d, 128), static_cast<int>(ceil_div(k, 128)));
     } else {
-      pl.main_splits = plan_splits(ceil_div(d, 256) * ceil_div(M, 256), steps, 8, 1);
+      pl.main_splits = plan_splits(ceil_div(d, 256) * 2 * ceil_div(M, 512), steps, 8, 1);
     }
     pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * d * 4) : 0;
   } else {
@@ -979,7 +1403,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
     const int msteps = static_cast<int>(ceil_div(M, 64));
     pl.splits_dA = plan_thin_splits(ceil_div(k, 128), msteps, rp);
     pl.splits_dB = plan_thin_splits(ceil_div(d, 128), msteps, rp);
-    pl.main_splits = plan_splits(ceil_div(k, 256) * ceil_div(M, 256), dsteps, 8, 1);
+    pl.main_splits = plan_splits(ceil_div(k, 256) * 2 * ceil_div(M, 512), dsteps, 8, 1);
     pl.off_main = pl.main_splits > 1 ? take(static_cast<size_t>(pl.main_splits) * M * k * 4) : 0;
   }
   pl.total = off;
@@ -1089,6 +1513,42 @@ static int launch_main(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
   return 0;
 }
 
+// The paired kernel: clusters of two CTAs along the token tiles (grid x).
+template <bool BWD>
+static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tc, const CUtensorMap& te, const MainParams& mp,
+                       dim3 grid, cudaStream_t st, const char** why) {
+  using Cfg = PairCfg<BWD>;
+  if (set_smem(k_qlora_pair<BWD>, Cfg::kSmemBytes) != cudaSuccess) {
+    *why = "smem attribute (paired GEMM)";
+    return QLORA_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(Cfg::kThreads);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  {
+    ProfScope ps_(BWD ? QLORA_KC_BWD_GEMM : QLORA_KC_FWD_GEMM, st);
+    e = cudaLaunchKernelEx(&cfg, k_qlora_pair<BWD>, ta, tc, te, mp);
+  }
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    static thread_local char msg[160];
+    snprintf(msg, sizeof msg, "paired GEMM launch: %s (%s)", cudaGetErrorName(e), cudaGetErrorString(e));
+    *why = msg;
+    return QLORA_ERR_CUDA;
+  }
+  return 0;
+}
+
 static ScaleSrc scale_src(const qlora_nf4_t& q) {
   ScaleSrc s{};
   s.dq = q.double_quant;
@@ -1140,8 +1600,9 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
          map_bf16(&t_ext, T, rp, M, 64, nt);
   } else {
+    // paired kernel: each CTA loads the codes of its 128-row half
     ok = map_bf16(&t_act, a.X, k, M, 64, 256) &&
-         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 256,
+         make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 32, 128,
                   CU_TENSOR_MAP_SWIZZLE_NONE) &&
          map_bf16(&t_ext, T, rp, M, 64, 256);
   }
@@ -1153,7 +1614,8 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   if (nt) {
     grid = dim3(static_cast<unsigned>(ceil_div(d, 128)), 1, static_cast<unsigned>(mp.splits));
   } else {
-    grid = dim3(static_cast<unsigned>(ceil_div(d, 256)), static_cast<unsigned>(ceil_div(M, 256)),
+    // token tiles rounded up to whole pairs (a CTA past M still dequantises its half)
+    grid = dim3(static_cast<unsigned>(2 * ceil_div(M, 512)), static_cast<unsigned>(ceil_div(d, 256)),
                 static_cast<unsigned>(mp.splits));
   }
   switch (nt) {
@@ -1161,7 +1623,7 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     case 32: rc = launch_main<Mode::FwdSwap, 32>(t_act, t_codes, t_ext, mp, grid, st, why); break;
     case 64: rc = launch_main<Mode::FwdSwap, 64>(t_act, t_codes, t_ext, mp, grid, st, why); break;
     case 128: rc = launch_main<Mode::FwdSwap, 128>(t_act, t_codes, t_ext, mp, grid, st, why); break;
-    default: rc = launch_main<Mode::Fwd, 0>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    default: rc = launch_pair<false>(t_act, t_codes, t_ext, mp, grid, st, why); break;
   }
   if (rc) return rc;
   if (mp.splits > 1) {
@@ -1229,15 +1691,15 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     mp.partial = reinterpret_cast<float*>(ws + pl.off_main);
     CUtensorMap t_act, t_codes, t_ext;
     if (!map_bf16(&t_act, a.dY, d, M, 64, 256) ||
-        !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 64,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&t_codes, q.codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 64, 64,
+                  CU_TENSOR_MAP_SWIZZLE_64B) ||
         !map_bf16(&t_ext, U, rp, M, 64, 256)) {
       *why = "tensor map encoding failed (backward)";
       return QLORA_ERR_CUDA;
     }
-    dim3 grid(static_cast<unsigned>(ceil_div(k, 256)), static_cast<unsigned>(ceil_div(M, 256)),
+    dim3 grid(static_cast<unsigned>(2 * ceil_div(M, 512)), static_cast<unsigned>(ceil_div(k, 256)),
               static_cast<unsigned>(mp.splits));
-    rc = launch_main<Mode::Bwd, 0>(t_act, t_codes, t_ext, mp, grid, st, why);
+    rc = launch_pair<true>(t_act, t_codes, t_ext, mp, grid, st, why);
     if (rc) return rc;
     if (mp.splits > 1) {
       const int64_t count = M * k;
