@@ -19,18 +19,22 @@
 // never written to device memory.
 //
 // Kernels
-//   k_qlora_main<Fwd>     Y tile 256 tokens x 256 weight rows.  TMA stages X
-//                         and the packed codes; 16 dequant warps expand the codes
-//                         to bf16 in the 128-byte-swizzled K-major layout the
-//                         tensor core reads; one thread issues tcgen05.mma into
-//                         two 128 x 256 fp32 TMEM accumulators; the LoRA term is
-//                         one (or more) extra 64-wide K steps.
-//   k_qlora_main<Bwd>     dX tile 256 tokens x 256 input columns; the dequant
-//                         warps write W in the MN-major swizzled layout (the
-//                         reduction runs over W's rows).
-//   k_qlora_main<FwdSwap> few tokens (M <= 128): W rows are the MMA's M side
-//                         (128 per tile), the tokens its N side, so the tensor
-//                         core is not padded to 128 tokens; split over K.
+//   k_qlora_pair<false> forward, more than 128 tokens.  A cluster of two CTAs
+//                         (tcgen05.mma.cta_group::2) computes 512 tokens x 256
+//                         weight rows: each CTA stages its 256 token rows of X
+//                         and the packed codes of its 128 weight rows by TMA,
+//                         16 dequant warps expand the codes to bf16 in the
+//                         128-byte-swizzled K-major layout the tensor core
+//                         reads, and one thread of the first CTA issues the
+//                         MMAs into two 128 x 256 fp32 TMEM accumulators per
+//                         CTA; the LoRA term is one (or more) extra 64-wide K
+//                         steps.
+//   k_qlora_pair<true>    dX, 512 tokens x 256 input columns per pair; the
+//                         dequant warps write W in the MN-major swizzled layout
+//                         (the reduction runs over W's rows).
+//   k_qlora_swap<NT>      17..128 tokens: W rows are the MMA's M side (128 per
+//                         tile), the tokens its N side, so the tensor core is
+//                         not padded to 128 tokens; split over K.
 //   k_thin<false,*>       T_s and U_s (K-major activations; A read K-major, B
 //                         read MN-major straight from its storage).
 //   k_thin<true,true>     dA and dB (MN-major operands, the reduction runs over
@@ -182,42 +186,36 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 }
 
 // ============================================================================
-// Main fused kernel
+// Parameters shared by the fused kernels
 // ============================================================================
-enum class Mode : int { Fwd = 0, Bwd = 1, FwdSwap = 2 };
-
 struct MainParams {
   int64_t M, d, k;
   int32_t r, rp;
   int32_t kpb;              // NF4 blocks per weight row (k / 64)
   ScaleSrc sc;
-  const uint16_t* lora;     // Fwd/FwdSwap: B (d x r); Bwd: A (r x k)
+  const uint16_t* lora;     // forward: B (d x r); backward: A (r x k)
   uint16_t* out;            // bf16 output (splits == 1)
   float* partial;           // fp32 [splits][M][n_out] (splits > 1)
-  int64_t n_out;            // output columns: d (Fwd/FwdSwap) or k (Bwd)
+  int64_t n_out;            // output columns: d (forward) or k (backward)
   int32_t steps_main;       // main K steps in total
   int32_t steps_per_split;
   int32_t ext_steps;        // rp / 64
   int32_t splits;
 };
 
-template <Mode MODE, int NT>
-struct MainCfg {
-  static constexpr bool kSwap = MODE == Mode::FwdSwap;
-  static constexpr bool kBwd = MODE == Mode::Bwd;
-  // K width of one pipeline step: two NF4 blocks per weight row for the
-  // swapped (few-token) forward, one otherwise.  A step always holds 256 NF4
-  // blocks, one per thread of a dequant group.
-  static constexpr int kStepK = kSwap ? 128 : 64;
-  static constexpr int kWRows = kSwap ? 128 : (kBwd ? 64 : 256);      // W rows per K step
-  static constexpr int kWCols = kBwd ? 256 : kStepK;                   // W columns per K step
-  static constexpr int kActRows = kSwap ? NT : 256;                    // token rows per K step
-  static constexpr int kAccs = kSwap ? 1 : 2;                          // M=128 accumulators per tile
-  static constexpr int kMmaN = kSwap ? NT : 256;
-  static constexpr uint32_t kActAtomBytes = kActRows * 128;            // one 64-wide K atom of the activations
+// ============================================================================
+// Swapped forward (17..128 tokens): the weight rows are the MMA's M side (128
+// per CTA), the NT tokens its N side.  K step 128 (two NF4 blocks per weight
+// row); the LoRA extension steps are 64 wide.
+// ============================================================================
+template <int NT>
+struct SwapCfg {
+  static constexpr int kStepK = 128;
+  static constexpr int kWRows = 128;                                   // W rows per K step
+  static constexpr uint32_t kActAtomBytes = NT * 128;                  // one 64-wide K atom of the activations
   static constexpr uint32_t kActBytes = kActAtomBytes * (kStepK / 64);
-  static constexpr uint32_t kWBytes = kWRows * kWCols * 2;
-  static constexpr uint32_t kCodeBytes = kWRows * kWCols / 2;
+  static constexpr uint32_t kWBytes = kWRows * kStepK * 2;
+  static constexpr uint32_t kCodeBytes = kWRows * kStepK / 2;
   // Two rings: TMA stages (activations + packed codes, small) and dequantized
   // W-tile buffers (large, written by the dequant warps).  Decoupling them lets
   // many more code tiles be in flight than W tiles.
@@ -225,27 +223,21 @@ struct MainCfg {
   static constexpr int kWBufs = 3;   // W tiles being written or waiting + one the MMAs read
   static constexpr int kStagesRaw = static_cast<int>((218u * 1024u - kWBufs * kWBytes) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr uint32_t kTmemCols =
-      kSwap ? (kMmaN <= 32 ? 32u : (kMmaN <= 64 ? 64u : 128u)) : 512u;   // two 128x256 fp32 accumulators
+  static constexpr uint32_t kTmemCols = NT <= 32 ? 32u : (NT <= 64 ? 64u : 128u);
   static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kWBufs * kWBytes + 1024 /*align*/ + 512 /*barriers*/;
-  static constexpr int kDeqThreads = 512;     // 16 dequant warps (warps 2..17)
-  // Few tokens (swap): two groups of 8 warps take alternate steps and every
-  // thread expands a whole block (the dequant rate is what matters there).
-  // Many tokens: all 16 warps work on every step, two threads per block, which
-  // keeps the per-step latency short enough to feed the tensor core.
-  static constexpr int kGroups = kSwap ? 2 : 1;
-  static constexpr int kGroupThreads = kDeqThreads / kGroups;
-  static constexpr int kTPB = kGroupThreads / 256;    // threads per NF4 block
-  static constexpr int kCPT = 8 / kTPB;               // 16-byte chunks per thread
-  static constexpr int kThreads = 64 + kDeqThreads;
-  static constexpr uint32_t kIdesc = make_idesc_bf16(128, kMmaN, false, kBwd);
+  // two groups of 8 dequant warps take alternate steps; every thread expands
+  // one whole block (the dequant rate is what matters with few tokens)
+  static constexpr int kGroups = 2;
+  static constexpr int kGroupThreads = 256;
+  static constexpr int kThreads = 64 + kGroups * kGroupThreads;
+  static constexpr uint32_t kIdesc = make_idesc_bf16(128, NT, false, false);
 };
 
-template <Mode MODE, int NT>
+template <int NT>
 __global__ void __launch_bounds__(576, 1)
-    k_qlora_main(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
+    k_qlora_swap(const __grid_constant__ CUtensorMap tm_act, const __grid_constant__ CUtensorMap tm_codes,
                  const __grid_constant__ CUtensorMap tm_ext, const MainParams p) {
-  using Cfg = MainCfg<MODE, NT>;
+  using Cfg = SwapCfg<NT>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -265,14 +257,7 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // tile coordinates
-  int64_t m0 = 0, n0 = 0;   // token row / output column of the tile (non-swap); W row (swap)
-  if (Cfg::kSwap) {
-    n0 = static_cast<int64_t>(blockIdx.x) * 128;
-  } else {
-    n0 = static_cast<int64_t>(blockIdx.x) * 256;
-    m0 = static_cast<int64_t>(blockIdx.y) * 256;
-  }
+  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 128;   // first W row of the tile
   const int split = blockIdx.z;
   const int s_begin = split * p.steps_per_split;
   const int s_end = min(p.steps_main, s_begin + p.steps_per_split);
@@ -319,21 +304,13 @@ __global__ void __launch_bounds__(576, 1)
         if (l < n_main) {
           const int i = s_begin + l;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes + Cfg::kCodeBytes);
-          if (Cfg::kSwap) {
-            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 128 * i, 0);
-            tma_load_2d(act_tile(st) + Cfg::kActAtomBytes, &tm_act, &full_bar[st], 128 * i + 64, 0);
-            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 64 * i, static_cast<int>(n0));
-          } else if (Cfg::kBwd) {
-            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
-            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], static_cast<int>(n0 / 2), 64 * i);
-          } else {
-            tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 64 * i, static_cast<int>(m0));
-            tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(n0));
-          }
+          tma_load_2d(act_tile(st), &tm_act, &full_bar[st], 128 * i, 0);
+          tma_load_2d(act_tile(st) + Cfg::kActAtomBytes, &tm_act, &full_bar[st], 128 * i + 64, 0);
+          tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 64 * i, static_cast<int>(n0));
         } else {
           const int e = l - n_main;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActAtomBytes);
-          tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, Cfg::kSwap ? 0 : static_cast<int>(m0));
+          tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, 0);
         }
         ++issued;
       }
@@ -364,24 +341,9 @@ __global__ void __launch_bounds__(576, 1)
         const int slices = (l < n_main) ? Cfg::kStepK / 16 : 4;   // LoRA steps are 64 wide
         for (int kk = 0; kk < slices; ++kk) {
           const uint32_t atom = static_cast<uint32_t>(kk >> 2), kq = static_cast<uint32_t>(kk & 3);
-          uint64_t da, db;
-          if (Cfg::kSwap) {
-            da = make_sdesc_sw128(a_w + 16384u * atom + 32u * kq, 16u, 1024u);
-            db = make_sdesc_sw128(a_act + Cfg::kActAtomBytes * atom + 32u * kq, 16u, 1024u);
-          } else if (Cfg::kBwd) {
-            da = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
-            db = make_sdesc_sw128(a_w + 2048u * kk, 8192u, 1024u);
-          } else {
-            da = make_sdesc_sw128(a_act + 32u * kk, 16u, 1024u);
-            db = make_sdesc_sw128(a_w + 32u * kk, 16u, 1024u);
-          }
-          const uint32_t acc = (l > 0 || kk > 0) ? 1u : 0u;
-          umma_bf16(tmem_base, da, db, Cfg::kIdesc, acc);
-          if (Cfg::kAccs == 2) {
-            // token rows 128..255 of the tile share the same W tile: second accumulator
-            const uint64_t da1 = make_sdesc_sw128(a_act + 16384u + 32u * kk, 16u, 1024u);
-            umma_bf16(tmem_base + 256u, da1, db, Cfg::kIdesc, acc);
-          }
+          const uint64_t da = make_sdesc_sw128(a_w + 16384u * atom + 32u * kq, 16u, 1024u);
+          const uint64_t db = make_sdesc_sw128(a_act + Cfg::kActAtomBytes * atom + 32u * kq, 16u, 1024u);
+          umma_bf16(tmem_base, da, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[st]);
         umma_commit(&wfree_bar[sw]);
@@ -390,15 +352,12 @@ __global__ void __launch_bounds__(576, 1)
     }
   } else {
     // ------------------------------------------------------------ dequant warps
-    // kGroups groups take alternate K steps; a step's 256 NF4 blocks are
-    // spread over the group's threads, kTPB threads per block, each expanding
-    // kCPT 16-byte chunks (8 weights each) of the block's 128-byte row.
-    constexpr int G = Cfg::kGroups, TPB = Cfg::kTPB, CPT = Cfg::kCPT;
+    // Two groups take alternate K steps; a step's 256 NF4 blocks (two per W
+    // row) go one to a thread, each expanding the block's eight 16-byte chunks.
+    constexpr int G = Cfg::kGroups;
     const int t = threadIdx.x - 64;            // 0..511
     const int grp = t / Cfg::kGroupThreads;
-    const int tgt = t % Cfg::kGroupThreads;
-    const int tg = tgt / TPB;                  // block of the step
-    const int c_first = (tgt % TPB) * CPT;     // first chunk of this thread
+    const int tg = t % Cfg::kGroupThreads;     // block of the step
     // the codebook as register immediates (no memory traffic)
     constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
     float C[16];
@@ -406,32 +365,19 @@ __global__ void __launch_bounds__(576, 1)
     for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
     const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
-    // position of this thread's block in the tile
-    //   Fwd : row = W row (0..255)
-    //   Bwd : row = W row within the 64-row K step (MN-major K row), sub = 64-column chunk
-    //   Swap: row = W row (0..127), sub = which of the step's two blocks
-    const int row = Cfg::kBwd ? (tg & 63) : (Cfg::kSwap ? (tg & 127) : tg);
-    const int sub = Cfg::kBwd ? (tg >> 6) : (Cfg::kSwap ? (tg >> 7) : 0);
-    const uint32_t w_off = Cfg::kBwd ? 8192u * sub : (Cfg::kSwap ? 16384u * sub : 0u);
-    // Code tile rows: 32 B (Fwd, plain), 64 B (Swap, TMA 64-byte swizzle: 16-byte
-    // chunk j of row r sits at j ^ ((r >> 1) & 3)), 128 B (Bwd, 128-byte swizzle:
-    // j ^ (r & 7)).  The swizzles spread a quarter-warp's reads over all banks.
-    constexpr uint32_t kCodeRow = Cfg::kBwd ? 128u : (Cfg::kSwap ? 64u : 32u);
-    const uint32_t c_row = row * kCodeRow;
-    const uint32_t lc0 = (Cfg::kBwd || Cfg::kSwap ? 2u * sub : 0u) + static_cast<uint32_t>(c_first / 4);
-    const uint32_t c_xor = Cfg::kBwd ? (row & 7u) : (Cfg::kSwap ? ((row >> 1) & 3u) : 0u);
+    // row = W row (0..127), sub = which of the step's two blocks
+    const int row = tg & 127;
+    const int sub = tg >> 7;
+    const uint32_t w_off = 16384u * sub;
+    // Code tile rows are 64 B with the TMA 64-byte swizzle: 16-byte chunk j of
+    // row r sits at j ^ ((r >> 1) & 3), which spreads a quarter-warp's reads
+    // over all banks.
+    const uint32_t c_row = row * 64u;
+    const uint32_t lc0 = 2u * sub;
+    const uint32_t c_xor = (row >> 1) & 3u;
     auto block_of = [&](int i, bool& valid) -> int64_t {
-      int64_t wr, bc;
-      if (Cfg::kBwd) {
-        wr = 64ll * i + row;
-        bc = n0 / 64 + sub;
-      } else if (Cfg::kSwap) {
-        wr = n0 + row;
-        bc = 2ll * i + sub;
-      } else {
-        wr = n0 + row;
-        bc = i;
-      }
+      const int64_t wr = n0 + row;
+      const int64_t bc = 2ll * i + sub;
       valid = (wr < p.d) && (bc < p.kpb);
       return wr * p.kpb + bc;
     };
@@ -467,9 +413,9 @@ __global__ void __launch_bounds__(576, 1)
           if (pre1_valid) pre1 = scale_fetch(sc, bn);
         }
         const uint32_t ctile = smem_u32(code_tile(st)) + c_row;
-        uint32_t w8[CPT];
+        uint32_t w8[8];
 #pragma unroll
-        for (int h = 0; h < CPT / 4; ++h) {
+        for (int h = 0; h < 2; ++h) {
           const uint4 cw = lds128(ctile + 16u * ((lc0 + h) ^ c_xor));
           w8[4 * h] = cw.x;
           w8[4 * h + 1] = cw.y;
@@ -479,41 +425,27 @@ __global__ void __launch_bounds__(576, 1)
         if (cur_valid) {
           const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur, recip), C);
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w8[c], tab));
+          for (int c = 0; c < 8; ++c) sts128(wt + sw128_offset(row, c), dq8(w8[c], tab));
         } else {
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), make_uint4(0, 0, 0, 0));
+          for (int c = 0; c < 8; ++c) sts128(wt + sw128_offset(row, c), make_uint4(0, 0, 0, 0));
         }
-      } else {
-        // LoRA extension step (64 wide): copy 64 columns of the adapter into the W tile
+      } else if (sub == 0) {
+        // LoRA extension step (64 wide): B (d x r) row n, columns 64e + [0, 64)
+        // into the first K atom
         const int e = l - n_main;
-        if (Cfg::kBwd) {
-          // A (r x k): K row j = 64e + row, N columns n0 + 64 sub + [0, 64)
-          const int64_t j = 64ll * e + row;
-          const int64_t col = n0 + 64 * sub;
-          const bool v = (j < p.r) && (col < p.k);
-          const uint16_t* srcp = p.lora + j * p.k + col;
+        const int64_t n = n0 + row;
+        const uint32_t wt0 = smem_u32(w_tile(sw));
 #pragma unroll
-          for (int c = c_first; c < c_first + CPT; ++c) {
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (v) val = __ldg(reinterpret_cast<const uint4*>(srcp + 8 * c));
-            sts128(wt + sw128_offset(row, c), val);
+        for (int c = 0; c < 8; ++c) {
+          uint32_t h[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int64_t j = 64ll * e + 8 * c + q;
+            h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
           }
-        } else if (!Cfg::kSwap || sub == 0) {
-          // B (d x r): row n, columns 64e + [0, 64) into the first K atom
-          const int64_t n = n0 + row;
-          const uint32_t wt0 = smem_u32(w_tile(sw));
-#pragma unroll
-          for (int c = c_first; c < c_first + CPT; ++c) {
-            uint32_t h[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int64_t j = 64ll * e + 8 * c + q;
-              h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
-            }
-            sts128(wt0 + sw128_offset(row, c),
-                   make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
-          }
+          sts128(wt0 + sw128_offset(row, c),
+                 make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
         }
       }
       fence_proxy_async_smem();
@@ -523,63 +455,28 @@ __global__ void __launch_bounds__(576, 1)
 
     // ------------------------------------------------------------ epilogue
     // warp w may read TMEM lanes 32 (w % 4) ..; the four warps sharing a lane
-    // quarter split the columns (idx = 0..3)
+    // quarter split the token columns (idx = 0..3).  Lanes = W rows n.
     const bool ok = __all_sync(0xffffffffu, mbar_wait(tmem_full, 0, abort_flag, DEV_WAIT_TIMEOUT_EPILOGUE));
     tc_fence_after();
     if (ok) {
       const int q = warp & 3;
       const int idx = (warp - 2) >> 2;
       const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * q) << 16);
-      if (!Cfg::kSwap) {
-        const int acc = idx >> 1;                       // which 128-token half of the tile
-        const int64_t m = m0 + 128 * acc + 32 * q + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 128 * (idx & 1) + 32 * cb;
-          uint32_t v[32];
-          tmem_ld32(lane_base + 256u * acc + col0, v);
-          tmem_ld_wait();
-          if (m < p.M) {
-            const int64_t n = n0 + col0;
-            if (p.splits == 1) {
-              uint16_t* dst = p.out + m * p.n_out + n;
+      const int64_t n = n0 + 32 * q + lane;
+      for (int cb = idx; cb < NT / 16; cb += 4) {
+        uint32_t v[16];
+        tmem_ld16(lane_base + 16 * cb, v);
+        tmem_ld_wait();
+        if (n < p.d) {
 #pragma unroll
-              for (int g = 0; g < 4; ++g) {
-                if (n + 8 * g + 8 <= p.n_out) {
-                  uint4 o;
-                  o.x = pack_bf16x2(__uint_as_float(v[8 * g + 0]), __uint_as_float(v[8 * g + 1]));
-                  o.y = pack_bf16x2(__uint_as_float(v[8 * g + 2]), __uint_as_float(v[8 * g + 3]));
-                  o.z = pack_bf16x2(__uint_as_float(v[8 * g + 4]), __uint_as_float(v[8 * g + 5]));
-                  o.w = pack_bf16x2(__uint_as_float(v[8 * g + 6]), __uint_as_float(v[8 * g + 7]));
-                  *reinterpret_cast<uint4*>(dst + 8 * g) = o;
-                }
-              }
-            } else {
-              float* dst = p.partial + (static_cast<int64_t>(split) * p.M + m) * p.n_out + n;
-#pragma unroll
-              for (int g = 0; g < 8; ++g)
-                if (n + 4 * g + 4 <= p.n_out)
-                  *reinterpret_cast<uint4*>(dst + 4 * g) = make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-            }
-          }
-        }
-      } else {
-        // lanes = W rows n, columns = tokens
-        const int64_t n = n0 + 32 * q + lane;
-        for (int cb = idx; cb < NT / 16; cb += 4) {
-          uint32_t v[16];
-          tmem_ld16(lane_base + 16 * cb, v);
-          tmem_ld_wait();
-          if (n < p.d) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int64_t tok = 16 * cb + j;
-              if (tok < p.M) {
-                if (p.splits == 1) {
-                  const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f);
-                  p.out[tok * p.n_out + n] = static_cast<uint16_t>(b & 0xFFFFu);
-                } else {
-                  p.partial[(static_cast<int64_t>(split) * p.M + tok) * p.n_out + n] = __uint_as_float(v[j]);
-                }
+          for (int j = 0; j < 16; ++j) {
+            const int64_t tok = 16 * cb + j;
+            if (tok < p.M) {
+              if (p.splits == 1) {
+                const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f);
+                p.out[tok * p.n_out + n] = static_cast<uint16_t>(b & 0xFFFFu);
+              } else {
+                p.partial[(static_cast<int64_t>(split) * p.M + tok) * p.n_out + n] = __uint_as_float(v[j]);
               }
             }
           }
@@ -619,9 +516,12 @@ __global__ void __launch_bounds__(576, 1)
 //   * Each CTA loads its own activation tile and its half of the codes (TMA,
 //     local barriers) and dequantises its half of W into its own shared memory.
 //   * Two dequant groups of 8 warps take alternate K steps; when a group's W
-//     half is written it arrives on the rank-0 CTA's wready barrier (remotely
-//     from rank 1), after having waited for its own TMA stage, so the barrier
-//     completing means both halves of W and both activation tiles are there.
+//     half is written (after its own TMA stage landed) its warps arrive on
+//     their CTA's wready barrier.  In rank 1 the otherwise idle MMA thread
+//     waits for that barrier and forwards it to rank 0's wready barrier with
+//     one cluster-scope release, so rank 0's barrier completing means both
+//     halves of W and both activation tiles are there, and the dequant warps
+//     never pay for a cluster-scope fence.
 //   * One thread of rank 0 issues the MMAs for both CTAs; its commits arrive on
 //     the stage / W-buffer / accumulator barriers of both CTAs (multicast).
 //   * TMEM is allocated and freed by warp 1 of both CTAs together.
@@ -756,7 +656,8 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < SW; ++i) {
-      mbar_init(&wready_bar[i], 2 * (Cfg::kGroupThreads / 32));   // one group's warps of both CTAs
+      // rank 0: its own group's warps + the relay of rank 1; rank 1: its own warps
+      mbar_init(&wready_bar[i], Cfg::kGroupThreads / 32 + (rank == 0 ? 1 : 0));
       mbar_init(&wfree_bar[i], 1);
     }
     mbar_init(tmem_full, 1);
@@ -789,7 +690,7 @@ __global__ void __launch_bounds__(576, 1)
       for (int l = 0; l < n_local; ++l) {
         const int st = l % S;
         const uint32_t ph = (l / S) & 1;
-        if (!mbar_wait_cluster(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
+        if (!mbar_wait(&empty_bar[st], ph ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA)) break;
         if (l < n_main) {
           const int i = s_begin + l;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes + Cfg::kCodeBytes);
@@ -842,6 +743,15 @@ __global__ void __launch_bounds__(576, 1)
         umma2_commit_both(&wfree_bar[sw]);
       }
       umma2_commit_both(tmem_full);   // also drains MMAs on the abort path
+    } else if (lane == 0) {
+      // relay (rank 1): once this CTA's group has written its W half and seen
+      // its TMA stage land, pass that on to rank 0 with one cluster-scope
+      // release, so the dequant warps themselves only arrive locally
+      for (int l = 0; l < n_local; ++l) {
+        const int sw = l % SW;
+        if (!mbar_wait(&wready_bar[sw], (l / SW) & 1, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
+        mbar_arrive_cluster(&wready_bar[sw], 0);
+      }
     }
   } else {
     // ------------------------------------------------------------ dequant warps (both CTAs)
@@ -896,7 +806,7 @@ __global__ void __launch_bounds__(576, 1)
       const uint32_t ph = (l / S) & 1;
       const int sw = l % SW;
       const uint32_t phw = (l / SW) & 1;
-      bool okw = mbar_wait_cluster(&wfree_bar[sw], phw ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
+      bool okw = mbar_wait(&wfree_bar[sw], phw ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
       okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
       if (!__all_sync(0xffffffffu, okw)) break;
       const uint32_t wt = smem_u32(w_tile(sw)) + w_off;
@@ -960,12 +870,7 @@ __global__ void __launch_bounds__(576, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        if (rank == 0)
-          mbar_arrive(&wready_bar[sw]);
-        else
-          mbar_arrive_cluster(&wready_bar[sw], 0);
-      }
+      if (lane == 0) mbar_arrive(&wready_bar[sw]);
     }
 
     // ------------------------------------------------------------ epilogue (both CTAs)
@@ -1497,19 +1402,19 @@ static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uin
               : launch_thin<false, false>(ta, tb, tp, ceil_div(M, 128), splits, st, why);
 }
 
-template <Mode MODE, int NT>
-static int launch_main(const CUtensorMap& ta, const CUtensorMap& tc, const CUtensorMap& te, const MainParams& mp,
+template <int NT>
+static int launch_swap(const CUtensorMap& ta, const CUtensorMap& tc, const CUtensorMap& te, const MainParams& mp,
                        dim3 grid, cudaStream_t st, const char** why) {
-  using Cfg = MainCfg<MODE, NT>;
-  if (set_smem(k_qlora_main<MODE, NT>, Cfg::kSmemBytes) != cudaSuccess) {
-    *why = "smem attribute (main)";
+  using Cfg = SwapCfg<NT>;
+  if (set_smem(k_qlora_swap<NT>, Cfg::kSmemBytes) != cudaSuccess) {
+    *why = "smem attribute (swapped GEMM)";
     return QLORA_ERR_CUDA;
   }
   {
-    ProfScope ps_((MODE == Mode::Bwd ? QLORA_KC_BWD_GEMM : QLORA_KC_FWD_GEMM), st);
-    k_qlora_main<MODE, NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
+    ProfScope ps_(QLORA_KC_FWD_GEMM, st);
+    k_qlora_swap<NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
   }
-  QL_CHECK_LAUNCH("main GEMM launch");
+  QL_CHECK_LAUNCH("swapped GEMM launch");
   return 0;
 }
 
@@ -1619,10 +1524,10 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
                 static_cast<unsigned>(mp.splits));
   }
   switch (nt) {
-    case 16: rc = launch_main<Mode::FwdSwap, 16>(t_act, t_codes, t_ext, mp, grid, st, why); break;
-    case 32: rc = launch_main<Mode::FwdSwap, 32>(t_act, t_codes, t_ext, mp, grid, st, why); break;
-    case 64: rc = launch_main<Mode::FwdSwap, 64>(t_act, t_codes, t_ext, mp, grid, st, why); break;
-    case 128: rc = launch_main<Mode::FwdSwap, 128>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 16: rc = launch_swap<16>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 32: rc = launch_swap<32>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 64: rc = launch_swap<64>(t_act, t_codes, t_ext, mp, grid, st, why); break;
+    case 128: rc = launch_swap<128>(t_act, t_codes, t_ext, mp, grid, st, why); break;
     default: rc = launch_pair<false>(t_act, t_codes, t_ext, mp, grid, st, why); break;
   }
   if (rc) return rc;
