@@ -516,12 +516,12 @@ __global__ void __launch_bounds__(576, 1)
 //   * Each CTA loads its own activation tile and its half of the codes (TMA,
 //     local barriers) and dequantises its half of W into its own shared memory.
 //   * Two dequant groups of 8 warps take alternate K steps; when a group's W
-//     half is written (after its own TMA stage landed) its warps arrive on
-//     their CTA's wready barrier.  In rank 1 the otherwise idle MMA thread
-//     waits for that barrier and forwards it to rank 0's wready barrier with
-//     one cluster-scope release, so rank 0's barrier completing means both
-//     halves of W and both activation tiles are there, and the dequant warps
-//     never pay for a cluster-scope fence.
+//     half is written (after its own TMA stage landed) each of its warps
+//     fences its stores to the async proxy and arrives on rank 0's wready
+//     barrier (remotely from rank 1, with the default arrive semantics, as
+//     transform warps feeding a 2-SM MMA do), so the barrier completing means
+//     both halves of W and both activation tiles are there.  (A cluster-scope
+//     release on that arrive costs about a microsecond per step.)
 //   * One thread of rank 0 issues the MMAs for both CTAs; its commits arrive on
 //     the stage / W-buffer / accumulator barriers of both CTAs (multicast).
 //   * TMEM is allocated and freed by warp 1 of both CTAs together.
@@ -576,11 +576,13 @@ __device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
       "h"(mask)
       : "memory");
 }
-// Arrive on the mbarrier at this offset in cluster CTA `rank`.
-__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t rank) {
+// Arrive on the mbarrier at this offset in cluster CTA `rank` (default
+// semantics, as the peer CTA of a 2-SM MMA signals its leader that operands it
+// wrote are ready; the writer fences its stores to the async proxy first).
+__device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(bar)), "r"(rank));
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
   uint32_t ok;
@@ -656,8 +658,7 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&empty_bar[i], 1);
     }
     for (int i = 0; i < SW; ++i) {
-      // rank 0: its own group's warps + the relay of rank 1; rank 1: its own warps
-      mbar_init(&wready_bar[i], Cfg::kGroupThreads / 32 + (rank == 0 ? 1 : 0));
+      mbar_init(&wready_bar[i], 2 * (Cfg::kGroupThreads / 32));   // one group's warps of both CTAs (rank 0 only)
       mbar_init(&wfree_bar[i], 1);
     }
     mbar_init(tmem_full, 1);
@@ -725,7 +726,7 @@ __global__ void __launch_bounds__(576, 1)
         const int sw = l % SW;
         const uint32_t phw = (l / SW) & 1;
         if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
-        if (!mbar_wait_cluster(&wready_bar[sw], phw, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
+        if (!mbar_wait(&wready_bar[sw], phw, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
         tc_fence_after();
         const uint32_t a_act = smem_u32(act_tile(st));
         const uint32_t a_w = smem_u32(w_tile(sw));
@@ -743,15 +744,6 @@ __global__ void __launch_bounds__(576, 1)
         umma2_commit_both(&wfree_bar[sw]);
       }
       umma2_commit_both(tmem_full);   // also drains MMAs on the abort path
-    } else if (lane == 0) {
-      // relay (rank 1): once this CTA's group has written its W half and seen
-      // its TMA stage land, pass that on to rank 0 with one cluster-scope
-      // release, so the dequant warps themselves only arrive locally
-      for (int l = 0; l < n_local; ++l) {
-        const int sw = l % SW;
-        if (!mbar_wait(&wready_bar[sw], (l / SW) & 1, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
-        mbar_arrive_cluster(&wready_bar[sw], 0);
-      }
     }
   } else {
     // ------------------------------------------------------------ dequant warps (both CTAs)
@@ -870,7 +862,12 @@ __global__ void __launch_bounds__(576, 1)
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&wready_bar[sw]);
+      if (lane == 0) {
+        if (rank == 0)
+          mbar_arrive(&wready_bar[sw]);
+        else
+          mbar_arrive_remote(&wready_bar[sw], 0);
+      }
     }
 
     // ------------------------------------------------------------ epilogue (both CTAs)
