@@ -1084,16 +1084,21 @@ __global__ void __launch_bounds__(128, 2)
   {
     const int trow = 32 * warp + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(32 * warp) << 16);
-    for (int cb = 0; cb < rp / 32; ++cb) {
-      uint32_t v[32];
-      tmem_ld32(lane_base + 32 * cb, v);
+    const bool zero = !ok || n_local == 0;
+    // rp is a multiple of 64: two 32-column loads in flight per wait
+    for (int cb = 0; cb < rp / 32; cb += 2) {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lane_base + 32 * cb, v0);
+      tmem_ld32(lane_base + 32 * (cb + 1), v1);
       tmem_ld_wait();
       float* dst = red + trow * ldr + 32 * cb;
-      const bool zero = !ok || n_local == 0;
 #pragma unroll
-      for (int g = 0; g < 8; ++g)
+      for (int g = 0; g < 8; ++g) {
         *reinterpret_cast<uint4*>(dst + 4 * g) =
-            zero ? make_uint4(0, 0, 0, 0) : make_uint4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            zero ? make_uint4(0, 0, 0, 0) : make_uint4(v0[4 * g], v0[4 * g + 1], v0[4 * g + 2], v0[4 * g + 3]);
+        *reinterpret_cast<uint4*>(dst + 32 + 4 * g) =
+            zero ? make_uint4(0, 0, 0, 0) : make_uint4(v1[4 * g], v1[4 * g + 1], v1[4 * g + 2], v1[4 * g + 3]);
+      }
     }
   }
   // 2: every CTA of the cluster has parked its tile (all CTAs always take both
@@ -1111,13 +1116,20 @@ __global__ void __launch_bounds__(128, 2)
       const int rr = (p.mode == THIN_DA) ? r0 + idx % nr : r0 + idx / c4n;
       const int c4 = (p.mode == THIN_DA) ? idx / nr : idx % c4n;
       const uint32_t off = (static_cast<uint32_t>(rr) * ldr + 4u * static_cast<uint32_t>(c4)) * 4u;
+      // all peers' loads in flight first, then the sum in rank order
+      float4 v[8];
+#pragma unroll
+      for (int pr = 0; pr < 8; ++pr)
+        if (pr < S2) v[pr] = ld_cluster_f4(red_addr + off, static_cast<uint32_t>(pr));
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (int pr = 0; pr < S2; ++pr) {
-        const float4 v = ld_cluster_f4(red_addr + off, static_cast<uint32_t>(pr));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+#pragma unroll
+      for (int pr = 0; pr < 8; ++pr) {
+        if (pr < S2) {
+          acc.x += v[pr].x;
+          acc.y += v[pr].y;
+          acc.z += v[pr].z;
+          acc.w += v[pr].w;
+        }
       }
       const int64_t row = row0 + rr;
       if (row >= p.rows) continue;
