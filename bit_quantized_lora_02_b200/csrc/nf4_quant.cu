@@ -150,13 +150,22 @@ void quant_thresholds(float out[15]) {
 // |w/s| >= 2^-102 (checked exhaustively over all bf16 significand pairs);
 // smaller quotients all map to the exact-zero code either way.  Outside that
 // scale range the kernel falls back to IEEE division.
-__device__ __forceinline__ float quotient(float w, float s, float r, bool fast) {
-  if (fast) {
-    float y = __fmul_rn(w, r);
-    float e = __fmaf_rn(-s, y, w);
-    return __fmaf_rn(e, r, y);
-  }
-  return __fdiv_rn(w, s);
+//
+// Two-lane fp32 arithmetic (sm_100 packed f32x2): each lane is one IEEE
+// round-to-nearest fp32 operation, so a pair gives the same bits as two
+// scalar operations for half the instructions.
+__device__ __forceinline__ void mul2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2,%3};\n\tmov.b64 b, {%4,%5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0,%1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2_rn(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                        float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2,%3};\n\tmov.b64 b, {%4,%5};\n\tmov.b64 c, {%6,%7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0,%1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
 // One thread handles 16 consecutive weights (two 16-byte loads); 4 lanes share
@@ -176,7 +185,9 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
   __syncthreads();
 
   const int lane = tid & 31;
-  const uint32_t lut_lane = smem_u32(s_lut) + 8u * static_cast<uint32_t>(lane & 15);
+  // byte address of cell c in this lane's copy is lut_lane + 128 c; with
+  // c = bits(y) - kCellBiasBits the subtraction folds into the base (mod 2^32)
+  const uint32_t lut_lane = smem_u32(s_lut) + 8u * static_cast<uint32_t>(lane & 15) - 128u * kCellBiasBits;
   const int64_t ngroups = (N + 15) >> 4;                     // groups of 16 elements
   const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
   for (int64_t g0 = static_cast<int64_t>(blockIdx.x) * 256 + (tid & ~31); g0 < ngroups; g0 += stride) {
@@ -209,18 +220,33 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
     if (s != 0.0f) {
       const bool fast = (s >= 0x1p-60f) && (s <= 0x1p60f);
       const float r = __frcp_rn(s);
+      float xn[16];
+      if (fast) {
+        // y = RN(w r), e = fma(-s, y, w), xn = fma(e, r, y), two weights at a time
+#pragma unroll
+        for (int i = 0; i < 16; i += 2) {
+          float y0, y1, e0, e1;
+          mul2_rn(y0, y1, w[i], w[i + 1], r, r);
+          fma2_rn(e0, e1, -s, -s, y0, y1, w[i], w[i + 1]);
+          fma2_rn(xn[i], xn[i + 1], e0, e1, r, r, y0, y1);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xn[i] = __fdiv_rn(w[i], s);
+      }
       lo = 0;
       hi = 0;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float xn = quotient(w[i], s, r, fast);
-        const float y = __fmaf_rn(xn, 16.0f, kCellBias);
-        const uint32_t cell = __float_as_uint(y) - kCellBiasBits;
-        float2 e;
-        asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(e.x), "=f"(e.y) : "r"(lut_lane + cell * 128u));
-        const uint32_t q = __float_as_uint(e.y) + (xn > e.x ? 1u : 0u);
-        if (i < 8) lo |= q << (4 * i);
-        else hi |= q << (4 * (i - 8));
+      for (int i = 0; i < 16; i += 2) {
+        float y0, y1;
+        fma2_rn(y0, y1, xn[i], xn[i + 1], 16.0f, 16.0f, kCellBias, kCellBias);
+        float2 e0, e1;
+        asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(e0.x), "=f"(e0.y) : "r"(lut_lane + __float_as_uint(y0) * 128u));
+        asm("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(e1.x), "=f"(e1.y) : "r"(lut_lane + __float_as_uint(y1) * 128u));
+        const uint32_t q0 = __float_as_uint(e0.y) + (xn[i] > e0.x ? 1u : 0u);
+        const uint32_t q1 = __float_as_uint(e1.y) + (xn[i + 1] > e1.x ? 1u : 0u);
+        if (i < 8) lo += (q0 << (4 * i)) + (q1 << (4 * i + 4));
+        else hi += (q0 << (4 * (i - 8))) + (q1 << (4 * (i - 8) + 4));
       }
     }
     if (e0 < N) {
