@@ -74,8 +74,10 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the sources the many-token GEMM kernels are built from (the
+    kernels whose DRAM traffic profiles/traffic_*.txt records)."""
     h = hashlib.sha256()
-    for name in ("qlora_gemm.cu", "qlora_fewtok.cu", "qlora_device.cuh", "nf4_scale.cuh", "nf4_quant.cu"):
+    for name in ("qlora_gemm.cu", "qlora_device.cuh", "qlora_internal.h", "nf4_scale.cuh", "nf4_table.h"):
         with open(os.path.join(ROOT, "bit_quantized_lora_02_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
