@@ -72,8 +72,10 @@ typedef void *qlora_stream_t;
  *   c1    : G = ceil(M_b/256) fp32 second-level scales, c1 = 127 / max|s - mean|
  *           over the group (1.0 for an all-zero group); DQ only.
  *   mean  : 1 fp32, the mean of all M_b block scales; DQ only.
- * All pointers are device pointers; codes and c2 need no alignment beyond 4
- * bytes, the fp32 arrays 4 bytes. */
+ * All pointers are device pointers.  Alignment (checked on the host, else
+ * QLORA_ERR_ALIGNMENT): codes 4 bytes for nf4_quantize / nf4_dequantize and
+ * 16 bytes for qlora_linear_fwd / qlora_linear_bwd (read by TMA); c2 8 bytes;
+ * absmax, c1 and mean 4 bytes. */
 typedef struct {
   int64_t d;
   int64_t k;
