@@ -55,7 +55,7 @@ __all__ = [
     "nearest_code", "nf4_quantize", "pack_codes", "unpack_codes", "int8_absmax_quantize",
     "int8_dequantize", "exact_mean_f32", "double_quantize", "double_dequantize_scales",
     "nf4_dequantize", "quantize_tensor", "dequantize_tensor", "storage_bits_per_weight",
-    "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale",
+    "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale", "lora_merge",
 ]
 
 BLOCK = 64          # weights per NF4 block ([QLoRA-chkda] "QLoRA uses blocks of 64 weights")
@@ -306,3 +306,18 @@ def qlora_backward(dY, X, W_hat, A, B, alpha: float, r: int):
     dA = s * (U.T @ X)
     dB = s * (dY.T @ T)
     return dX, dA, dB
+
+
+# ----------------------------------------------------------------------------
+# LoRA merge  ([QLoRA-chkda] "Merging LoRA weights for inference")
+# ----------------------------------------------------------------------------
+def lora_merge(W_hat, A, B, alpha: float, r: int):
+    """W_merged = W + (alpha/r) B A in fp64: the adapter folded into the (here
+    reconstructed NF4) base weight, d x k.  Then X W_merged^T equals the
+    two-path forward up to rounding (the page's equivalence claim).
+
+    W_hat (d x k), A (r x k), B (d x r); bf16-bit arrays or floats.
+    """
+    W_hat, A, B = map(_f64, (W_hat, A, B))
+    s = float(lora_scale(alpha, r))
+    return W_hat + s * (B @ A)

@@ -333,6 +333,44 @@ def test_forward_merged_equivalence():
     assert np.allclose(Y, merged, rtol=1e-12, atol=1e-12)
 
 
+def test_merge_hand_example():
+    # d=3, k=2, r=1, alpha=2 -> s=2.  B A = [[1, 1], [0, 0], [2, 2]], so
+    # W + 2 B A = [[3, 2], [0, 1], [5, 5]] ([QLoRA-chkda] "Merging LoRA weights
+    # for inference": W_merged = W0 + (alpha/r) B A).
+    W = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])
+    A = np.array([[1.0, 1.0]])
+    B = np.array([[1.0], [0.0], [2.0]])
+    assert O.lora_merge(W, A, B, alpha=2.0, r=1).tolist() == [[3.0, 2.0], [0.0, 1.0], [5.0, 5.0]]
+
+
+def test_merge_bruteforce_sum():
+    _, W, A, B, _ = _tiny(3, d=4, k=5, r=3)
+    s = float(O.lora_scale(8.0, 3))
+    got = O.lora_merge(W, A, B, alpha=8.0, r=3)
+    for n in range(4):
+        for c in range(5):
+            ref = W[n, c]
+            acc = 0.0
+            for j in range(3):
+                acc += B[n, j] * A[j, c]
+            assert abs(got[n, c] - (ref + s * acc)) <= 1e-12 * (abs(ref) + abs(s * acc) + 1.0)
+
+
+def test_merge_matches_two_path_forward():
+    # the page's equivalence: before merging h = W0 x + (alpha/r) B (A x),
+    # after merging h = W_merged x
+    X, W, A, B, _ = _tiny(4)
+    Y, _ = O.qlora_forward(X, W, A, B, alpha=16.0, r=3)
+    Ym = X @ O.lora_merge(W, A, B, alpha=16.0, r=3).T
+    assert np.allclose(Y, Ym, rtol=1e-12, atol=1e-12)
+
+
+def test_merge_zero_adapter_or_scale_is_identity():
+    _, W, A, B, _ = _tiny(5)
+    assert np.array_equal(O.lora_merge(W, A, np.zeros_like(B), alpha=16.0, r=3), W)
+    assert np.array_equal(O.lora_merge(W, A, B, alpha=0.0, r=3), W)
+
+
 @pytest.mark.parametrize("shape", [(1, 1, 1, 1), (4, 6, 5, 2), (3, 8, 16, 4)])
 def test_backward_finite_differences(shape):
     m, d, k, r = shape
