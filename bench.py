@@ -519,6 +519,27 @@ def run_secondary(args, wl_name):
                                 "dequantize_frac_hbm": round(dbytes / (md * 1e-3) / 1e9 / hbm, 4)})
         metric, unit = "NF4 quantize GB/s (4096x11008, double quant)", "GB/s"
         value = [x for x in results if x["proj"].startswith("rect") and x["double_quant"]][0]["quantize_gbs"]
+    elif wl_name == "merge_sweep":
+        work = synth.WORKLOADS[wl_name]
+        r, alpha = work["r"], work["alpha"]
+        for pi, (name, d, k) in enumerate(work["proj"]):
+            q = Q.nf4_quantize(dev_bits(synth.weight(d, k, seed=pi)), True)
+            A = dev_bits(synth.lora_a(r, k, seed=pi))
+            B = dev_bits(synth.lora_b(d, r, seed=pi))
+            out = torch.empty(d, k, dtype=torch.bfloat16, device=dev)
+            fm = lambda: Q.qlora_lora_merge(q, A, B, alpha, out=out, stream=stream)  # noqa: E731
+            for _ in range(args.warmup):
+                fm()
+            mm = _timed(fm, iters, flush, stream)
+            n = d * k
+            nblk = n // 64
+            # algorithmic bytes: codes + c2 + c1 + mean read, merged bf16 written, adapters read once
+            mbytes = n // 2 + nblk + 4 * (-(-nblk // 256)) + 4 + 2 * n + 2 * r * (d + k)
+            results.append({"proj": f"{name}:{d}x{k}", "r": r, "merge_ms": round(mm, 4),
+                            "merge_gbs": round(mbytes / (mm * 1e-3) / 1e9, 1),
+                            "merge_frac_hbm": round(mbytes / (mm * 1e-3) / 1e9 / hbm, 4)})
+        metric, unit = "LoRA merge GB/s (W_merged = W^ + (alpha/r) B A, 11008x4096, r=64)", "GB/s"
+        value = [x for x in results if x["proj"].startswith("gate")][0]["merge_gbs"]
     else:
         raise SystemExit(f"unknown secondary workload {wl_name}")
     print(json.dumps({"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "workload": wl_name,
@@ -534,12 +555,12 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama7b_proj_set_m4096",
                     choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512",
-                             "decode_28672x8192", "quant_sweep"))
+                             "decode_28672x8192", "quant_sweep", "merge_sweep"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    if args.workload in ("decode_28672x8192", "quant_sweep"):
+    if args.workload in ("decode_28672x8192", "quant_sweep", "merge_sweep"):
         if args.impl == "reference":
             print(json.dumps({"impl": "reference", "unavailable": "secondary workloads are measured for this arm only"}))
             return

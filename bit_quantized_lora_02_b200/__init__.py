@@ -25,7 +25,8 @@ QLORA_OK = 0
 _STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTED", -3: "QLORA_ERR_ALIGNMENT",
            -4: "QLORA_ERR_WORKSPACE", -5: "QLORA_ERR_CUDA", -6: "QLORA_ERR_DEVICE"}
 
-EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_rank_pad", "qlora_linear_workspace_size",
+EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_lora_merge",
+           "qlora_rank_pad", "qlora_linear_workspace_size",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error",
            "qlora_profile_enable", "qlora_profile_read")
 
@@ -61,6 +62,7 @@ def lib() -> ctypes.CDLL:
     L.nf4_quantize.argtypes = [vp, ctypes.POINTER(QloraNF4), vp, c_sz, vp]
     L.nf4_quantize_noalloc.argtypes = [vp, ctypes.POINTER(QloraNF4), vp]
     L.nf4_dequantize.argtypes = [ctypes.POINTER(QloraNF4), vp, vp]
+    L.qlora_lora_merge.argtypes = [ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float, vp, vp]
     L.qlora_rank_pad.argtypes = [c_i32]
     L.qlora_rank_pad.restype = c_i32
     L.qlora_linear_workspace_size.argtypes = [c_i64, c_i64, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz)]
@@ -73,7 +75,8 @@ def lib() -> ctypes.CDLL:
     L.qlora_last_error.restype = ctypes.c_char_p
     L.qlora_profile_enable.argtypes = [c_i32]
     L.qlora_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
-    for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_linear_workspace_size",
+    for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_lora_merge",
+                 "qlora_linear_workspace_size",
                  "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
                  "qlora_profile_enable", "qlora_profile_read"):
         getattr(L, name).restype = c_i32
@@ -182,6 +185,18 @@ def nf4_dequantize(q: NF4Weight, out: Optional[torch.Tensor] = None, stream=None
         out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
     st = q.struct()
     _check(lib().nf4_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def qlora_lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W_merged = BF16(W^ + (alpha/r) B A) as a bf16 (d, k) tensor."""
+    r = A.shape[0]
+    if out is None:
+        out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
+    st = q.struct()
+    _check(lib().qlora_lora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha), out.data_ptr(),
+                                  _stream(stream)))
     return out
 
 

@@ -1,5 +1,5 @@
-// nf4_scale.cuh -- the per-block scale s^ of the NF4 weight inside the GEMM
-// kernels.
+// nf4_scale.cuh -- the per-block scale s^ of the NF4 weight and the expansion
+// of a block's codes to bf16, shared by the GEMM and merge kernels.
 //
 // "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora), "Double quantization
 // and double dequantization": with double quantization each 64-weight block
@@ -11,6 +11,8 @@
 #include <cstdint>
 
 #include <cuda_runtime.h>
+
+#include "qlora_device.cuh"
 
 namespace qlora {
 
@@ -72,6 +74,61 @@ __device__ __forceinline__ float scale_value(int dq, float mean, ScaleRaw r, Sca
     q = __fdiv_rn(w, r.a);
   }
   return __fadd_rn(q, mean);
+}
+
+// ============================================================================
+// Expansion of one 64-weight NF4 block (into the GEMMs' swizzled W rows and
+// the merged weight).
+//
+// The block's 16 reconstruction values T[j] = BF16(RN32(C[j] * s^)) are built
+// once per block (bit-identical to BF16(C[q] * s^) per weight), split into four
+// registers of low bytes and four of high bytes, and every 4-bit code is then
+// resolved with byte permutes: PRMT selects by the code's low 3 bits from each
+// half of the table and a sign-replicated mask of the code's top bit picks the
+// half.  About 2.75 integer instructions per weight, no shared-memory lookups.
+// ============================================================================
+struct Nf4Tab {
+  uint32_t L[4], H[4];
+};
+
+__device__ __forceinline__ Nf4Tab make_tab(float sh, const float (&C)[16]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(C[2 * i], sh), __fmul_rn(C[2 * i + 1], sh));
+  Nf4Tab t;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    t.L[i] = prmt(P[2 * i], P[2 * i + 1], 0x6420u);
+    t.H[i] = prmt(P[2 * i], P[2 * i + 1], 0x7531u);
+  }
+  return t;
+}
+
+// 8 codes (code i in bits 4i..4i+3) -> 8 bf16 (element i in halfword i).
+__device__ __forceinline__ uint4 dq8(uint32_t c, const Nf4Tab& t) {
+  const uint32_t xl = c & 0x7777u;
+  const uint32_t xh = (c >> 16) & 0x7777u;
+  const uint32_t d4 = c << 4;
+  const uint32_t ml = prmt(d4, c, 0xD9C8u);   // 0xFF in byte i iff code i >= 8 (i = 0..3)
+  const uint32_t mh = prmt(d4, c, 0xFBEAu);   // same for codes 4..7
+  uint4 o;
+  {
+    const uint32_t la = prmt(t.L[0], t.L[1], xl), lb = prmt(t.L[2], t.L[3], xl);
+    const uint32_t ha = prmt(t.H[0], t.H[1], xl), hb = prmt(t.H[2], t.H[3], xl);
+    const uint32_t lo = (la & ~ml) | (lb & ml);
+    const uint32_t hi = (ha & ~ml) | (hb & ml);
+    o.x = prmt(lo, hi, 0x5140u);
+    o.y = prmt(lo, hi, 0x7362u);
+  }
+  {
+    const uint32_t la = prmt(t.L[0], t.L[1], xh), lb = prmt(t.L[2], t.L[3], xh);
+    const uint32_t ha = prmt(t.H[0], t.H[1], xh), hb = prmt(t.H[2], t.H[3], xh);
+    const uint32_t lo = (la & ~mh) | (lb & mh);
+    const uint32_t hi = (ha & ~mh) | (hb & mh);
+    o.z = prmt(lo, hi, 0x5140u);
+    o.w = prmt(lo, hi, 0x7362u);
+  }
+  return o;
 }
 
 }  // namespace qlora

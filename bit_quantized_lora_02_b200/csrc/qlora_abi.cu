@@ -275,6 +275,21 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlo
   return ok();
 }
 
+int qlora_lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int32_t r, float alpha,
+                     uint16_t* W_out, qlora_stream_t stream) {
+  int64_t N = 0;
+  int rc = check_nf4(q, &N);
+  if (rc) return rc;
+  if ((rc = check_linear_shape(0, q->d, q->k, r))) return rc;
+  if (!aligned(q->codes, 16)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 16-byte aligned for the merge");
+  if ((rc = check_ptr16(A, "A", true)) || (rc = check_ptr16(B, "B", true)) || (rc = check_ptr16(W_out, "W_out", true)))
+    return rc;
+  if ((rc = bind_device(W_out))) return rc;
+  return check_cuda(launch_lora_merge(*q, A, B, r, alpha / static_cast<float>(r), W_out,
+                                      static_cast<cudaStream_t>(stream)),
+                    "qlora_lora_merge launch");
+}
+
 int qlora_nf4_codebook(float out[16]) {
   if (!out) return fail(QLORA_ERR_INVALID_ARG, "out is NULL");
   host_codebook(out);

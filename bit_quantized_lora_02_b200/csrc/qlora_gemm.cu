@@ -115,59 +115,6 @@ static bool map_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t r
                   CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// ============================================================================
-// Dequantisation of one 64-weight NF4 block into a 128-byte swizzled row.
-//
-// The block's 16 reconstruction values T[j] = BF16(RN32(C[j] * s^)) are built
-// once per block (bit-identical to BF16(C[q] * s^) per weight), split into four
-// registers of low bytes and four of high bytes, and every 4-bit code is then
-// resolved with byte permutes: PRMT selects by the code's low 3 bits from each
-// half of the table and a sign-replicated mask of the code's top bit picks the
-// half.  About 2.75 integer instructions per weight, no shared-memory lookups.
-// ============================================================================
-struct Nf4Tab {
-  uint32_t L[4], H[4];
-};
-
-__device__ __forceinline__ Nf4Tab make_tab(float sh, const float (&C)[16]) {
-  uint32_t P[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) P[i] = pack_bf16x2(__fmul_rn(C[2 * i], sh), __fmul_rn(C[2 * i + 1], sh));
-  Nf4Tab t;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    t.L[i] = prmt(P[2 * i], P[2 * i + 1], 0x6420u);
-    t.H[i] = prmt(P[2 * i], P[2 * i + 1], 0x7531u);
-  }
-  return t;
-}
-
-// 8 codes (code i in bits 4i..4i+3) -> 8 bf16 (element i in halfword i).
-__device__ __forceinline__ uint4 dq8(uint32_t c, const Nf4Tab& t) {
-  const uint32_t xl = c & 0x7777u;
-  const uint32_t xh = (c >> 16) & 0x7777u;
-  const uint32_t d4 = c << 4;
-  const uint32_t ml = prmt(d4, c, 0xD9C8u);   // 0xFF in byte i iff code i >= 8 (i = 0..3)
-  const uint32_t mh = prmt(d4, c, 0xFBEAu);   // same for codes 4..7
-  uint4 o;
-  {
-    const uint32_t la = prmt(t.L[0], t.L[1], xl), lb = prmt(t.L[2], t.L[3], xl);
-    const uint32_t ha = prmt(t.H[0], t.H[1], xl), hb = prmt(t.H[2], t.H[3], xl);
-    const uint32_t lo = (la & ~ml) | (lb & ml);
-    const uint32_t hi = (ha & ~ml) | (hb & ml);
-    o.x = prmt(lo, hi, 0x5140u);
-    o.y = prmt(lo, hi, 0x7362u);
-  }
-  {
-    const uint32_t la = prmt(t.L[0], t.L[1], xh), lb = prmt(t.L[2], t.L[3], xh);
-    const uint32_t ha = prmt(t.H[0], t.H[1], xh), hb = prmt(t.H[2], t.H[3], xh);
-    const uint32_t lo = (la & ~mh) | (lb & mh);
-    const uint32_t hi = (ha & ~mh) | (hb & mh);
-    o.z = prmt(lo, hi, 0x5140u);
-    o.w = prmt(lo, hi, 0x7362u);
-  }
-  return o;
-}
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
@@ -201,6 +148,7 @@ struct MainParams {
   int32_t steps_per_split;
   int32_t ext_steps;        // rp / 64
   int32_t splits;
+  int32_t ncp;              // paired kernel: 256-column pairs across the output
 };
 
 // ============================================================================
@@ -642,9 +590,13 @@ __global__ void __launch_bounds__(576, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  // the two CTAs of a pair are neighbours along x (peer CTAs of cta_group::2)
-  const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 256;   // output columns of the pair
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * 256;   // this CTA's tokens
+  // The two CTAs of a pair are neighbours along x (peer CTAs of cta_group::2).
+  // Clusters are numbered column pair first, so the clusters resident at one
+  // time share a few token tiles and each activation tile is read from DRAM
+  // about once.
+  const int64_t cl = static_cast<int64_t>(blockIdx.x) >> 1;
+  const int64_t n0 = (cl % p.ncp) * 256;                                 // output columns of the pair
+  const int64_t m0 = ((cl / p.ncp) * 2 + (blockIdx.x & 1)) * 256;       // this CTA's tokens
   const int64_t h0 = n0 + 128 * static_cast<int64_t>(rank);     // this CTA's half of the columns
   const int split = blockIdx.z;
   const int s_begin = split * p.steps_per_split;
@@ -1427,7 +1379,7 @@ static int launch_swap(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
   return 0;
 }
 
-// The paired kernel: clusters of two CTAs along the token tiles (grid x).
+// The paired kernel: clusters of two CTAs (grid x = 2 x token pairs x column pairs).
 template <bool BWD>
 static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tc, const CUtensorMap& te, const MainParams& mp,
                        dim3 grid, cudaStream_t st, const char** why) {
@@ -1529,8 +1481,8 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     grid = dim3(static_cast<unsigned>(ceil_div(d, 128)), 1, static_cast<unsigned>(mp.splits));
   } else {
     // token tiles rounded up to whole pairs (a CTA past M still dequantises its half)
-    grid = dim3(static_cast<unsigned>(2 * ceil_div(M, 512)), static_cast<unsigned>(ceil_div(d, 256)),
-                static_cast<unsigned>(mp.splits));
+    mp.ncp = static_cast<int32_t>(ceil_div(d, 256));
+    grid = dim3(static_cast<unsigned>(2 * ceil_div(M, 512) * mp.ncp), 1, static_cast<unsigned>(mp.splits));
   }
   switch (nt) {
     case 16: rc = launch_swap<16>(t_act, t_codes, t_ext, mp, grid, st, why); break;
@@ -1611,8 +1563,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
       *why = "tensor map encoding failed (backward)";
       return QLORA_ERR_CUDA;
     }
-    dim3 grid(static_cast<unsigned>(2 * ceil_div(M, 512)), static_cast<unsigned>(ceil_div(k, 256)),
-              static_cast<unsigned>(mp.splits));
+    mp.ncp = static_cast<int32_t>(ceil_div(k, 256));
+    dim3 grid(static_cast<unsigned>(2 * ceil_div(M, 512) * mp.ncp), 1, static_cast<unsigned>(mp.splits));
     rc = launch_pair<true>(t_act, t_codes, t_ext, mp, grid, st, why);
     if (rc) return rc;
     if (mp.splits > 1) {

@@ -28,6 +28,8 @@ void quant_thresholds(float out[15]);
 size_t quant_workspace_bytes(int64_t N, bool dq);
 cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, void* ws, cudaStream_t st);
 cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st);
+cudaError_t launch_lora_merge(const qlora_nf4_t& q, const uint16_t* A, const uint16_t* B, int r, float s,
+                              uint16_t* out, cudaStream_t st);
 // device address and size of the library-owned quantisation scratch (current device)
 cudaError_t noalloc_scratch(void** out, size_t* bytes);
 

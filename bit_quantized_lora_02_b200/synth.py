@@ -99,4 +99,5 @@ WORKLOADS = {
     "llama65b_block_m8192": dict(proj=PROJ_65B, m=8192, r=64, alpha=16.0, a_std=None, bwd=True),
     "proj_q_4096": dict(proj=[("q", 4096, 4096)], m=4096, r=64, alpha=16.0, a_std=None, bwd=True),
     "quant_sweep": dict(proj=[("sq", 4096, 4096), ("rect", 4096, 11008)], outliers=True),
+    "merge_sweep": dict(proj=[("q", 4096, 4096), ("gate", 11008, 4096), ("down", 4096, 11008)], r=64, alpha=16.0),
 }

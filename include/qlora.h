@@ -144,6 +144,24 @@ int nf4_quantize_noalloc(const uint16_t *W0, const qlora_nf4_t *q, qlora_stream_
  *   W_out : d*k bf16 (device, 16-byte aligned). */
 int nf4_dequantize(const qlora_nf4_t *q, uint16_t *W_out, qlora_stream_t stream);
 
+/* LoRA merge ("LoRA and QLoRA", "Merging LoRA weights for inference"): folds a
+ * trained adapter into the weight so inference needs one path,
+ *     W_out[n][c] = BF16(fma(s, acc[n][c], W^[n][c])),
+ *     acc[n][c]   = sum_j B[n][j] A[j][c]   (fp32 accumulation, order unspecified),
+ * with s = RN32(alpha / r) and W^ the reconstructed weight nf4_dequantize writes
+ * (the bf16 weight the forward uses), rounded once to bf16 (nearest even).  So
+ * X W_out^T equals the two-path qlora_linear_fwd output up to rounding.
+ * Re-quantising the merged weight is nf4_quantize on W_out (the page notes
+ * that merging into a quantized model costs precision).
+ *   q     : the quantized base, as for qlora_linear_fwd (k % 64 == 0,
+ *           d % 8 == 0, d <= 4194240; codes 16-byte aligned).
+ *   A     : r x k bf16, row-major;  B : d x r bf16, row-major;  1 <= r <= 256.
+ *   W_out : d x k bf16, row-major (device, 16-byte aligned); may not alias the
+ *           inputs.
+ * Stream-ordered; errors as for the other entry points. */
+int qlora_lora_merge(const qlora_nf4_t *q, const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                     uint16_t *W_out, qlora_stream_t stream);
+
 /* Columns of the saved adapter activation T_save (and of the internal U):
  * r rounded up to a multiple of 64. */
 int32_t qlora_rank_pad(int32_t r);

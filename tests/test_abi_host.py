@@ -106,6 +106,19 @@ def test_linear_rejects_null_inputs_without_gpu(L):
     assert L.qlora_linear_fwd(None, 0, ctypes.byref(st), None, None, 8, 16.0, None, None, None, 0, None) == 0
 
 
+def test_merge_validation_without_gpu(L):
+    st = Q.QloraNF4(512, 512, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+    rc = L.qlora_lora_merge(ctypes.byref(st), None, 0x20000, 8, 16.0, 0x30000, None)
+    assert rc == -1 and b"A" in L.qlora_last_error()
+    assert L.qlora_lora_merge(ctypes.byref(st), 0x10000, 0x20000, 0, 16.0, 0x30000, None) == -2     # r
+    assert L.qlora_lora_merge(ctypes.byref(st), 0x10000, 0x20000, 257, 16.0, 0x30000, None) == -2
+    assert L.qlora_lora_merge(ctypes.byref(st), 0x10000, 0x20000, 8, 16.0, 0x30008, None) == -3     # W_out
+    bad = Q.QloraNF4(512, 500, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+    assert L.qlora_lora_merge(ctypes.byref(bad), 0x10000, 0x20000, 8, 16.0, 0x30000, None) == -2    # k % 64
+    odd = Q.QloraNF4(512, 512, 64, 1, 0x1004, None, 0x2000, 0x3000, 0x4000)
+    assert L.qlora_lora_merge(ctypes.byref(odd), 0x10000, 0x20000, 8, 16.0, 0x30000, None) == -3    # codes
+
+
 def test_param_count_matches_buffer_shapes(golden):
     g = golden("lora_param_count.json")
     # A is r x k and B is d x r: the entries the backward writes
