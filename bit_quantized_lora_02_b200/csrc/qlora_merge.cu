@@ -11,17 +11,19 @@
 // unspecified) and one rounding to bf16 (nearest even).  Re-quantising the
 // merged weight is nf4_quantize on W_out.
 //
-// k_lora_merge: one CTA per 64 weight rows x 256 columns, 256 threads.
-//   1. For each 64-wide chunk of r, B's 64 x 64 and A's 64 x 256 tiles are
+// k_lora_merge: one CTA per 64 weight rows x 128 columns, 256 threads (three
+// CTAs per SM).
+//   0. Every thread first loads its 32 codes (16 bytes) and its block's
+//      constants, so their DRAM latency overlaps steps 1 and 2.
+//   1. For each 64-wide chunk of r, B's 64 x 64 and A's 64 x 128 tiles are
 //      copied to shared memory (zero padded past r, d and k) and every warp
-//      runs mma.sync.m16n8k16 (bf16 in, fp32 accumulate) over its 16 x 128
+//      runs mma.sync.m16n8k16 (bf16 in, fp32 accumulate) over its 16 x 64
 //      piece.  The contraction is tiny (r multiply-adds per weight); the tensor
 //      cores only keep it off the critical path.
 //   2. The fp32 tile goes to shared memory.
-//   3. Each thread takes one 64-weight NF4 block: 32 bytes of codes (two
-//      16-byte loads), the block scale, the 64 reconstructed weights, the fma
-//      with s * acc and 128 bytes of bf16 out (four threads per row, so a row's
-//      512 bytes are written contiguously).
+//   3. Each thread expands its half block (32 weights), adds s * acc with one
+//      fma and writes 64 bytes of bf16 (four threads per row, so a row's 256
+//      bytes are written contiguously).
 // Bound: HBM (0.5 B of codes + 2 B of output per weight).
 #include <cstdio>
 
@@ -35,14 +37,14 @@ namespace qlora {
 namespace {
 
 constexpr int kMergeRows = 64;
-constexpr int kMergeCols = 256;
+constexpr int kMergeCols = 128;
 constexpr int kRChunk = 64;
 constexpr int kBStride = kRChunk + 8;         // bf16 per row of the B tile (16 B pad: no ldmatrix conflicts)
 constexpr int kAStride = kMergeCols + 8;      // bf16 per row of the A tile
-// result tile: 8 floats of padding after every 64-column segment and a row
-// stride of 292 (= 4 mod 32) floats, so the epilogue's reads hit distinct banks
-constexpr int kRStride = 4 * 72 + 4;
-__device__ __forceinline__ int res_index(int row, int col) { return row * kRStride + col + 8 * (col >> 6); }
+// result tile: 8 floats of padding after every 32-column quarter and a row
+// stride of 164 (= 4 mod 32) floats, so the epilogue's reads hit distinct banks
+constexpr int kRStride = 4 * 40 + 4;
+__device__ __forceinline__ int res_index(int row, int col) { return row * kRStride + col + 8 * (col >> 5); }
 constexpr uint32_t kTileBytes = (kMergeRows * kBStride + kRChunk * kAStride) * 2;
 constexpr uint32_t kResBytes = kMergeRows * kRStride * 4;
 constexpr uint32_t kMergeSmem = kTileBytes > kResBytes ? kTileBytes : kResBytes;
@@ -66,7 +68,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(256) k_lora_merge(const uint8_t* __restrict__ codes, const ScaleSrc sc,
+__global__ void __launch_bounds__(256, 3) k_lora_merge(const uint8_t* __restrict__ codes, const ScaleSrc sc,
                                                     const uint16_t* __restrict__ A, const uint16_t* __restrict__ B,
                                                     int64_t d, int64_t k, int r, float s, uint16_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -79,11 +81,24 @@ __global__ void __launch_bounds__(256) k_lora_merge(const uint8_t* __restrict__ 
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * kMergeRows;
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kMergeCols;
   const int wr = warp >> 1;   // rows 16 wr .. 16 wr + 15
-  const int wc = warp & 1;    // columns 128 wc .. 128 wc + 127
+  const int wc = warp & 1;    // columns 64 wc .. 64 wc + 63
 
-  float acc[16][4];
+  // this thread's half block of the epilogue: row tid / 4, columns 32 (tid % 4) ..
+  const int row = tid >> 2, quarter = tid & 3;
+  const int64_t n = n0 + row;
+  const int64_t c = c0 + 32 * quarter;
+  const bool live = (n < d) && (c < k);
+  uint4 cw4 = make_uint4(0, 0, 0, 0);
+  ScaleRaw raw{};
+  if (live) {
+    cw4 = ldg_nc_v4(codes + ((n * k + c) >> 1));
+    raw = scale_fetch(sc, (n * k + c) >> 6);
+  }
+  const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
+
+  float acc[8][4];
 #pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
+  for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
 
@@ -98,7 +113,7 @@ __global__ void __launch_bounds__(256) k_lora_merge(const uint8_t* __restrict__ 
       sB[row * kBStride + j] = v;
     }
     // A (r x k, row-major; k % 64 == 0 so rows are 16-byte aligned): 64 rows
-    // x 256 columns, 16-byte loads
+    // x 128 columns, 16-byte loads
     for (int i = tid; i < kRChunk * (kMergeCols / 8); i += 256) {
       const int j = i / (kMergeCols / 8), c8 = i % (kMergeCols / 8);
       const int64_t c = c0 + 8 * c8;
@@ -115,13 +130,13 @@ __global__ void __launch_bounds__(256) k_lora_merge(const uint8_t* __restrict__ 
       uint32_t a0, a1, a2, a3;
       ldsm_x4(sB_addr + 2u * ((16 * wr + (lane & 15)) * kBStride + 16 * kk + 8 * (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {
+      for (int np = 0; np < 4; ++np) {
         // B operand (A rows j, columns c): two 8-column tiles, transposed
         // loads; lanes 0-7 k 0-7, 8-15 k 8-15 of tile 2np, 16-31 the same of
         // tile 2np + 1
         uint32_t b0, b1, b2, b3;
         const int krow = 16 * kk + (lane & 15);
-        const int ncol = 128 * wc + 16 * np + 8 * (lane >> 4);
+        const int ncol = 64 * wc + 16 * np + 8 * (lane >> 4);
         ldsm_x4_t(sA_addr + 2u * (krow * kAStride + ncol), b0, b1, b2, b3);
         mma_bf16_16816(acc[2 * np], a0, a1, a2, a3, b0, b1);
         mma_bf16_16816(acc[2 * np + 1], a0, a1, a2, a3, b2, b3);
@@ -131,47 +146,38 @@ __global__ void __launch_bounds__(256) k_lora_merge(const uint8_t* __restrict__ 
   }
 
   // fp32 tile to shared memory: fragment (nt, e) holds row 16 wr + lane/4 (+8
-  // for e >= 2), column 128 wc + 8 nt + 2 (lane % 4) + (e & 1)
+  // for e >= 2), column 64 wc + 8 nt + 2 (lane % 4) + (e & 1)
   {
     const int g = lane >> 2, q2 = 2 * (lane & 3);
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int col = 128 * wc + 8 * nt + q2;
+    for (int nt = 0; nt < 8; ++nt) {
+      const int col = 64 * wc + 8 * nt + q2;
       *reinterpret_cast<float2*>(sR + res_index(16 * wr + g, col)) = make_float2(acc[nt][0], acc[nt][1]);
       *reinterpret_cast<float2*>(sR + res_index(16 * wr + g + 8, col)) = make_float2(acc[nt][2], acc[nt][3]);
     }
   }
   __syncthreads();
 
-  // one NF4 block per thread: row tid / 4, columns 64 (tid % 4) ..
-  const int row = tid >> 2, seg = tid & 3;
-  const int64_t n = n0 + row;
-  const int64_t c = c0 + 64 * seg;
-  if (n >= d || c >= k) return;
-  const int64_t blk = (n * k + c) >> 6;
-  const uint8_t* cp = codes + ((n * k + c) >> 1);
-  const uint4 w0 = ldg_nc_v4(cp);
-  const uint4 w1 = ldg_nc_v4(cp + 16);
-  const uint32_t cw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+  if (!live) return;
   constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
   float C[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
   ScaleRecip recip;
-  const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
   // the block's reconstructed weights, as doubleDequant stores them:
   // BF16(RN32(C[q] * s^))
-  const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, scale_fetch(sc, blk), recip), C);
-  // segment seg of the row starts on bank group 8 seg (72 floats per
-  // segment), the next row 4 banks later: a quarter-warp's 16-byte reads (two
-  // rows x four segments) hit all 32 banks once
-  const float* rseg = sR + row * kRStride + 72 * seg;
+  const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, raw, recip), C);
+  // quarter q of the row starts on bank group 8 q (40 floats per quarter), the
+  // next row 4 banks later: a quarter-warp's 16-byte reads (two rows x four
+  // quarters) hit all 32 banks once
+  const float* rq = sR + row * kRStride + 40 * quarter;
   uint16_t* orow = out + n * k + c;
+  const uint32_t cw[4] = {cw4.x, cw4.y, cw4.z, cw4.w};
 #pragma unroll
-  for (int ch = 0; ch < 8; ++ch) {
+  for (int ch = 0; ch < 4; ++ch) {
     const uint4 wq = dq8(cw[ch], tab);   // 8 bf16 weights, element i in halfword i
-    const float4 lo = *reinterpret_cast<const float4*>(rseg + 8 * ch);
-    const float4 hi = *reinterpret_cast<const float4*>(rseg + 8 * ch + 4);
+    const float4 lo = *reinterpret_cast<const float4*>(rq + 8 * ch);
+    const float4 hi = *reinterpret_cast<const float4*>(rq + 8 * ch + 4);
     const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
     const uint32_t w4[4] = {wq.x, wq.y, wq.z, wq.w};
     uint32_t o[4];
