@@ -103,14 +103,24 @@ __global__ void __launch_bounds__(256, 3) k_lora_merge(const uint8_t* __restrict
     for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
 
   for (int j0 = 0; j0 < r; j0 += kRChunk) {
-    // B (d x r, row-major): 64 rows x 64 columns of the chunk, element loads
-    // (rows of B are 2r bytes, not always 16-byte multiples)
-    for (int i = tid; i < kMergeRows * kRChunk; i += 256) {
-      const int row = i / kRChunk, j = i % kRChunk;
-      const int64_t n = n0 + row;
-      uint16_t v = 0;
-      if (n < d && j0 + j < r) v = B[n * r + j0 + j];
-      sB[row * kBStride + j] = v;
+    // B (d x r, row-major): 64 rows x 64 columns of the chunk.  Rows are 2r
+    // bytes: 16-byte loads when r % 8 == 0, element loads otherwise.
+    if ((r & 7) == 0) {
+      for (int i = tid; i < kMergeRows * (kRChunk / 8); i += 256) {
+        const int row = i >> 3, j8 = i & 7;
+        const int64_t n = n0 + row;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (n < d && j0 + 8 * j8 < r) v = __ldg(reinterpret_cast<const uint4*>(B + n * r + j0 + 8 * j8));
+        *reinterpret_cast<uint4*>(sB + row * kBStride + 8 * j8) = v;
+      }
+    } else {
+      for (int i = tid; i < kMergeRows * kRChunk; i += 256) {
+        const int row = i / kRChunk, j = i % kRChunk;
+        const int64_t n = n0 + row;
+        uint16_t v = 0;
+        if (n < d && j0 + j < r) v = B[n * r + j0 + j];
+        sB[row * kBStride + j] = v;
+      }
     }
     // A (r x k, row-major; k % 64 == 0 so rows are 16-byte aligned): 64 rows
     // x 128 columns, 16-byte loads
