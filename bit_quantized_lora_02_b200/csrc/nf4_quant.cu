@@ -183,6 +183,8 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
   for (int i = tid; i < 33 * 16; i += 256) s_lut[i] = make_float2(lut.thr[i >> 4], lut.base[i >> 4]);
   if (kDQ) s_hist[tid] = 0;
   __syncthreads();
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int lane = tid & 31;
   // byte address of cell c in this lane's copy is lut_lane + 128 c; with
@@ -283,6 +285,8 @@ __global__ void __launch_bounds__(256) k_nf4_quant(const uint16_t* __restrict__ 
 }
 
 __global__ void k_zero_u64(unsigned long long* p, int n) {
+  griddep_launch_dependents();
+  griddep_wait();   // the previous call's constants kernel may still read the histogram
   for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0ull;
 }
 
@@ -371,6 +375,8 @@ __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ 
                                                    float* __restrict__ mean_out, int8_t* __restrict__ c2,
                                                    float* __restrict__ c1) {
   __shared__ float s_mean;
+  griddep_launch_dependents();
+  griddep_wait();
   const int lane = threadIdx.x & 31;
   if (threadIdx.x < 32) {
     const float m = exact_mean_warp(hist, nblocks);   // every CTA derives the same value
@@ -445,6 +451,8 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
     for (int j = 0; j < 16; ++j) s_C[j] = __uint_as_float(kCB[j]);
   }
   __syncthreads();
+  griddep_launch_dependents();
+  griddep_wait();
   const float mu = kDQ ? *mean : 0.0f;
   const int64_t ngroups = (N + 7) >> 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -501,7 +509,10 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
   if (!q.double_quant) {
     {
       ProfScope ps_(QLORA_KC_QUANT, st);
-      k_nf4_quant<false><<<grid, 256, 0, st>>>(W, N, q.codes, q.absmax, nullptr, nullptr, quant_lut());
+      const cudaError_t e = launch_pdl(k_nf4_quant<false>, dim3(grid), dim3(256), 0, st, nullptr, W, N, q.codes,
+                                       q.absmax, static_cast<uint16_t*>(nullptr),
+                                       static_cast<unsigned long long*>(nullptr), quant_lut());
+      if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
   }
@@ -509,11 +520,14 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
   auto* amax16 = reinterpret_cast<uint16_t*>(static_cast<char*>(ws) + 256 * sizeof(unsigned long long));
   {
     ProfScope ps_(QLORA_KC_DQ_CONST, st);
-    k_zero_u64<<<1, 256, 0, st>>>(hist, 256);
+    const cudaError_t e = launch_pdl(k_zero_u64, dim3(1), dim3(256), 0, st, nullptr, hist, 256);
+    if (e != cudaSuccess) return e;
   }
   {
     ProfScope ps_(QLORA_KC_QUANT, st);
-    k_nf4_quant<true><<<grid, 256, 0, st>>>(W, N, q.codes, nullptr, amax16, hist, quant_lut());
+    const cudaError_t e = launch_pdl(k_nf4_quant<true>, dim3(grid), dim3(256), 0, st, nullptr, W, N, q.codes,
+                                     static_cast<float*>(nullptr), amax16, hist, quant_lut());
+    if (e != cudaSuccess) return e;
   }
   const int64_t ngroups = (nblk + 255) / 256;
   {
@@ -521,7 +535,9 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
     // every CTA derives the mean itself, so keep the grid near one wave and loop over groups
     const int64_t want = (ngroups + 7) / 8;
     const int grid_g = static_cast<int>(want < 2 * num_sms() ? want : 2 * num_sms());
-    k_dq_groups<<<grid_g, 256, 0, st>>>(amax16, nblk, hist, q.mean, q.c2, q.c1);
+    const cudaError_t e = launch_pdl(k_dq_groups, dim3(grid_g), dim3(256), 0, st, nullptr, amax16, nblk, hist,
+                                     q.mean, q.c2, q.c1);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -529,10 +545,14 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
 cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st) {
   const int grid = grid_for((N + 7) / 8);
   ProfScope ps_(QLORA_KC_DEQUANT, st);
-  if (q.double_quant)
-    k_nf4_dequant<true><<<grid, 256, 0, st>>>(q.codes, N, nullptr, q.c2, q.c1, q.mean, out);
-  else
-    k_nf4_dequant<false><<<grid, 256, 0, st>>>(q.codes, N, q.absmax, nullptr, nullptr, nullptr, out);
+  const cudaError_t e =
+      q.double_quant
+          ? launch_pdl(k_nf4_dequant<true>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
+                       static_cast<const float*>(nullptr), q.c2, q.c1, q.mean, out)
+          : launch_pdl(k_nf4_dequant<false>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, q.absmax,
+                       static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
+                       static_cast<const float*>(nullptr), out);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

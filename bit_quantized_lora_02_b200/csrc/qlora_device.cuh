@@ -256,4 +256,18 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t r, uint32_t c) {
   return (r >> 3) * 1024u + (r & 7u) * 128u + ((c ^ (r & 7u)) << 4);
 }
 
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may start while the kernel before it in the
+// stream is still running.  griddep_wait() returns once that kernel has
+// completed and its memory operations are visible; every such kernel calls it
+// on every path, before its first access to memory another kernel may have
+// written, so that its own completion also implies its predecessor's.
+// griddep_launch_dependents() lets the next kernel's CTAs be scheduled; kernels
+// holding TMEM call it only after their allocation, so a waiting dependent CTA
+// on the same SM can never hold the columns a running CTA still needs.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace qlora

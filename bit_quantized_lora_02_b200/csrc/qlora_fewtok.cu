@@ -209,10 +209,6 @@ __device__ __forceinline__ float ld_cluster_f32(const void* local, uint32_t rank
   return v;
 }
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 // The CTA whose item range holds item i (ranges: [c I / G, (c+1) I / G)).
 __device__ __forceinline__ int cta_of_item(int64_t i, int items, int G) {

@@ -236,6 +236,8 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();   // after the TMEM allocation
+  griddep_wait();                // inputs written by the previous kernel
 
   auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
   auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
@@ -631,6 +633,8 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();   // after the TMEM allocation
+  griddep_wait();                // inputs written by the previous kernel
 
   auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
   auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
@@ -969,6 +973,8 @@ __global__ void __launch_bounds__(128, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  griddep_launch_dependents();   // after the TMEM allocation
+  griddep_wait();                // inputs written by the previous kernel
   auto a_tile = [&](int st) { return base + st * stage_bytes; };
   auto b_tile = [&](int st) { return base + st * stage_bytes + Cfg::kABytes; };
 
@@ -1122,6 +1128,8 @@ __global__ void __launch_bounds__(128, 2)
 // out_bf16[i] = BF16(scale * sum_s partial[s][i]), n4 = count / 4
 __global__ void k_reduce_bf16(const float* __restrict__ partial, int splits, int64_t count, float scale,
                               uint16_t* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t n4 = count >> 2;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -1140,6 +1148,8 @@ __global__ void k_reduce_bf16(const float* __restrict__ partial, int splits, int
 // Bt[j][n] = B[n][j] for j < r, 0 for r <= j < rp
 __global__ void k_transpose_B(const uint16_t* __restrict__ B, int64_t d, int r, int rp, uint16_t* __restrict__ Bt) {
   __shared__ uint16_t tile[32][34];
+  griddep_launch_dependents();
+  griddep_wait();
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * 32;
   const int j0 = blockIdx.y * 32;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
@@ -1316,22 +1326,12 @@ static int launch_thin(const CUtensorMap& ta, const CUtensorMap& tb, ThinParams 
     *why = "smem attribute (thin GEMM)";
     return QLORA_ERR_CUDA;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(real));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(real);
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaError_t e;
   {
     ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    e = cudaLaunchKernelEx(&cfg, k_thin<kAMN, kBMN>, ta, tb, tp);
+    const dim3 cl(1, static_cast<unsigned>(real), 1);
+    e = launch_pdl(k_thin<kAMN, kBMN>, dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(real)), dim3(128), smem,
+                   st, &cl, ta, tb, tp);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     *why = "thin GEMM launch";
@@ -1371,9 +1371,14 @@ static int launch_swap(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
     *why = "smem attribute (swapped GEMM)";
     return QLORA_ERR_CUDA;
   }
+  cudaError_t e;
   {
     ProfScope ps_(QLORA_KC_FWD_GEMM, st);
-    k_qlora_swap<NT><<<grid, Cfg::kThreads, Cfg::kSmemBytes, st>>>(ta, tc, te, mp);
+    e = launch_pdl(k_qlora_swap<NT>, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, nullptr, ta, tc, te, mp);
+  }
+  if (e != cudaSuccess) {
+    *why = "swapped GEMM launch";
+    return QLORA_ERR_CUDA;
   }
   QL_CHECK_LAUNCH("swapped GEMM launch");
   return 0;
@@ -1388,22 +1393,11 @@ static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
     *why = "smem attribute (paired GEMM)";
     return QLORA_ERR_CUDA;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(Cfg::kThreads);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   cudaError_t e;
   {
     ProfScope ps_(BWD ? QLORA_KC_BWD_GEMM : QLORA_KC_FWD_GEMM, st);
-    e = cudaLaunchKernelEx(&cfg, k_qlora_pair<BWD>, ta, tc, te, mp);
+    const dim3 cl(2, 1, 1);
+    e = launch_pdl(k_qlora_pair<BWD>, grid, dim3(Cfg::kThreads), Cfg::kSmemBytes, st, &cl, ta, tc, te, mp);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -1496,7 +1490,8 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     const int64_t count = M * d;
     {
       ProfScope ps_(QLORA_KC_AUX, st);
-      k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.Y);
+      (void)launch_pdl(k_reduce_bf16, dim3(static_cast<unsigned>(grid1d(count / 4, 256))), dim3(256), 0, st,
+                       nullptr, mp.partial, mp.splits, count, 1.0f, a.Y);
     }
     QL_CHECK_LAUNCH("reduce launch (forward)");
   }
@@ -1533,8 +1528,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
     {
       ProfScope ps_(QLORA_KC_AUX, st);
-      k_transpose_B<<<dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)), 256, 0, st>>>(
-          a.B, d, r, rp, Bt);
+      (void)launch_pdl(k_transpose_B, dim3(static_cast<unsigned>(ceil_div(d, 32)), static_cast<unsigned>(rp / 32)),
+                       dim3(256), 0, st, nullptr, a.B, d, r, rp, Bt);
     }
     QL_CHECK_LAUNCH("transpose launch");
     rc = run_lowrank_down(a.dY, M, d, Bt, rp, false, rp, a.s, pl.splits_U, U, st, why);
@@ -1571,7 +1566,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
       const int64_t count = M * k;
       {
         ProfScope ps_(QLORA_KC_AUX, st);
-        k_reduce_bf16<<<grid1d(count / 4, 256), 256, 0, st>>>(mp.partial, mp.splits, count, 1.0f, a.dX);
+        (void)launch_pdl(k_reduce_bf16, dim3(static_cast<unsigned>(grid1d(count / 4, 256))), dim3(256), 0, st,
+                         nullptr, mp.partial, mp.splits, count, 1.0f, a.dX);
       }
       QL_CHECK_LAUNCH("reduce launch (dX)");
     }

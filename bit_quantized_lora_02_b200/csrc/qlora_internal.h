@@ -71,6 +71,34 @@ int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensor
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device); the
 // attribute call costs host time on every launch otherwise.  Instantiations of
 // one kernel template share a function type, so the key is the address.
+// Launch with programmatic dependent launch allowed (the kernel calls
+// griddep_wait() before touching memory) and, when `cluster` is given, as
+// thread-block clusters of that shape.
+template <typename... ExpTypes, typename... ActTypes>
+cudaError_t launch_pdl(void (*kernel)(ExpTypes...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const dim3* cluster, ActTypes&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster->x;
+    attr[n].val.clusterDim.y = cluster->y;
+    attr[n].val.clusterDim.z = cluster->z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<ActTypes&&>(args)...);
+}
+
 template <typename K>
 cudaError_t set_smem(K kernel, uint32_t bytes) {
   static std::mutex mu;

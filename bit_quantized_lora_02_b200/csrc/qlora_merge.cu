@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(256, 3) k_lora_merge(const uint8_t* __restrict
   uint16_t* sB = reinterpret_cast<uint16_t*>(smem);
   uint16_t* sA = sB + kMergeRows * kBStride;
   float* sR = reinterpret_cast<float*>(smem);   // after the contraction
+  griddep_launch_dependents();
+  griddep_wait();
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -218,7 +220,9 @@ cudaError_t launch_lora_merge(const qlora_nf4_t& q, const uint16_t* A, const uin
                   static_cast<unsigned>((q.d + kMergeRows - 1) / kMergeRows));
   {
     ProfScope ps_(QLORA_KC_AUX, st);
-    k_lora_merge<<<grid, 256, kMergeSmem, st>>>(q.codes, sc, A, B, q.d, q.k, r, s, out);
+    const cudaError_t el = launch_pdl(k_lora_merge, grid, dim3(256), kMergeSmem, st, nullptr, q.codes, sc, A,
+                                      B, q.d, q.k, r, s, out);
+    if (el != cudaSuccess) return el;
   }
   return cudaGetLastError();
 }
