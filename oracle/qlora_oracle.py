@@ -56,6 +56,7 @@ __all__ = [
     "int8_dequantize", "exact_mean_f32", "double_quantize", "double_dequantize_scales",
     "nf4_dequantize", "quantize_tensor", "dequantize_tensor", "storage_bits_per_weight",
     "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale", "lora_merge",
+    "FP8_MAX", "fp8_e4m3_encode", "fp8_e4m3_decode", "double_quantize_fp8", "double_dequantize_scales_fp8",
 ]
 
 BLOCK = 64          # weights per NF4 block ([QLoRA-chkda] "QLoRA uses blocks of 64 weights")
@@ -222,6 +223,86 @@ def double_dequantize_scales(c2: np.ndarray, c1: np.ndarray, mean, group: int = 
     c2 = np.asarray(c2, dtype=np.int8)
     g = np.arange(c2.size) // group
     deq = (c2.astype(np.float32) / np.asarray(c1, np.float32)[g]).astype(np.float32)
+    return (deq + np.float32(mean)).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) second-level constants: the page's "c2_FP8" label ([QLoRA-chkda]
+# "Double quantization and double dequantization") read literally.  E4M3 is
+# 1 sign, 4 exponent (bias 7) and 3 mantissa bits; exponent field 15 with
+# mantissa 7 is NaN, so the largest finite value is 448, and exponent field 0
+# holds the subnormals m * 2^-9.  The group scale maps max|v| to 448 the way
+# the Int8 reading maps it to 127: c1 = RN32(448 / max|v|).
+# ----------------------------------------------------------------------------
+FP8_MAX = 448.0
+
+
+def fp8_e4m3_encode(x: np.ndarray) -> np.ndarray:
+    """fp32 -> E4M3 bits, round to nearest even; magnitudes past 448 saturate
+    to 448 (c1 * v never exceeds 448 by more than an fp32 rounding)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64).ravel()
+    out = np.empty(x.size, np.uint8)
+    for i, v in enumerate(x.tolist()):
+        sign = 0x80 if math.copysign(1.0, v) < 0 else 0
+        a = abs(v)
+        if a >= 2.0 ** -6:
+            e = math.floor(math.log2(a))
+            if 2.0 ** e > a:          # guard log2 rounding
+                e -= 1
+            elif 2.0 ** (e + 1) <= a:
+                e += 1
+            q = round((a / 2.0 ** e - 1.0) * 8.0)   # round() is half-to-even on the exact value
+            if q == 8:
+                e, q = e + 1, 0
+            if e > 8 or (e == 8 and q > 6):
+                e, q = 8, 6
+            out[i] = sign | ((e + 7) << 3) | q
+        else:
+            q = round(a / 2.0 ** -9)                # subnormal step 2^-9; q = 8 is the smallest normal
+            out[i] = sign | q
+    return out
+
+
+def fp8_e4m3_decode(b: np.ndarray) -> np.ndarray:
+    """E4M3 bits -> fp32 (exact)."""
+    b = np.asarray(b, dtype=np.uint8).ravel()
+    out = np.empty(b.size, np.float32)
+    for i, v in enumerate(b.tolist()):
+        sign = -1.0 if v & 0x80 else 1.0
+        e, m = (v >> 3) & 15, v & 7
+        if e == 15 and m == 7:
+            out[i] = np.nan
+        elif e == 0:
+            out[i] = sign * m * 2.0 ** -9
+        else:
+            out[i] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return out
+
+
+def double_quantize_fp8(absmax: np.ndarray, group: int = DQ_GROUP):
+    """Second-level quantisation with E4M3 constants: v = RN32(s - mean), per
+    group c1 = RN32(448 / max|v|) (1 for an all-zero group) and
+    c2 = E4M3(RN32(c1 * v)).  Returns (c2 uint8[M_b], c1 f32[G], mean f32)."""
+    absmax = np.asarray(absmax, dtype=np.float32)
+    mu = exact_mean_f32(absmax)
+    v = (absmax - mu).astype(np.float32)
+    ng = -(-absmax.size // group)
+    c2 = np.empty(absmax.size, np.uint8)
+    c1 = np.empty(ng, np.float32)
+    for g in range(ng):
+        vg = v[g * group:(g + 1) * group]
+        m = np.float32(np.max(np.abs(vg))) if vg.size else np.float32(0)
+        c = np.float32(1.0) if m == 0 else np.float32(np.float32(FP8_MAX) / m)
+        c1[g] = c
+        c2[g * group:(g + 1) * group] = fp8_e4m3_encode((c * vg).astype(np.float32))
+    return c2, c1, mu
+
+
+def double_dequantize_scales_fp8(c2: np.ndarray, c1: np.ndarray, mean, group: int = DQ_GROUP) -> np.ndarray:
+    """scales[j] = RN32(RN32(decode(c2[j]) / c1[j // 256]) + mean)."""
+    c2 = np.asarray(c2, dtype=np.uint8)
+    g = np.arange(c2.size) // group
+    deq = (fp8_e4m3_decode(c2) / np.asarray(c1, np.float32)[g]).astype(np.float32)
     return (deq + np.float32(mean)).astype(np.float32)
 
 

@@ -276,6 +276,65 @@ def test_dq_off_reduces_to_single_level():
     assert np.array_equal(O.dequantize_tensor(q), O.nf4_dequantize(codes, absmax))
 
 
+def _torch_e4m3_bits(x):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_fp8_encode_matches_library_conversion():
+    # every finite bf16 value with |x| <= 464 (past 464 the library gives NaN and
+    # the oracle saturates; c1 * v never gets there), then a wide fp32 sample
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    x = O.bf16_bits_to_f32(bits)
+    x = x[np.isfinite(x) & (np.abs(x) <= 464.0)]
+    assert np.array_equal(O.fp8_e4m3_encode(x), _torch_e4m3_bits(x))
+    rng = np.random.default_rng(7)
+    y = (rng.uniform(-1, 1, 20000) * 2.0 ** rng.integers(-12, 9, 20000)).astype(np.float32)
+    y = y[np.abs(y) <= 464.0]
+    assert np.array_equal(O.fp8_e4m3_encode(y), _torch_e4m3_bits(y))
+
+
+def test_fp8_ties_round_to_even():
+    vals = O.fp8_e4m3_decode(np.arange(0x7F, dtype=np.uint8)).astype(np.float64)   # 0 .. 448, ascending
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mids.astype(np.float64), (vals[:-1] + vals[1:]) / 2)      # exact in fp32
+    got = O.fp8_e4m3_encode(mids)
+    even = np.where(np.arange(1, 0x7F) % 2 == 0, np.arange(1, 0x7F), np.arange(0, 0x7E))
+    assert np.array_equal(got, even.astype(np.uint8))
+
+
+def test_fp8_decode_all_codes():
+    import torch
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float32).numpy()
+    got = O.fp8_e4m3_decode(np.arange(256, dtype=np.uint8))
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+    assert O.fp8_e4m3_decode(np.array([0x7E, 0x01, 0x08, 0x38, 0xC0], np.uint8)).tolist() == [448.0, 2.0 ** -9,
+                                                                                             2.0 ** -6, 1.0, -2.0]
+
+
+def test_double_quant_fp8_group_max_and_error_bound():
+    rng = np.random.default_rng(8)
+    s = np.abs(rng.standard_normal(1000) * 0.02 + 0.05).astype(np.float32)
+    c2, c1, mu = O.double_quantize_fp8(s)
+    v = (s - mu).astype(np.float32)
+    for g in range(len(c1)):
+        dec = O.fp8_e4m3_decode(c2[g * 256:(g + 1) * 256])
+        assert np.max(np.abs(dec)) == 448.0          # the group's largest |v| lands on the top code
+        assert c1[g] == np.float32(np.float32(448.0) / np.max(np.abs(v[g * 256:(g + 1) * 256])))
+    sh = O.double_dequantize_scales_fp8(c2, c1, mu).astype(np.float64)
+    g = np.arange(s.size) // 256
+    bound = 2.0 ** -4 * np.abs(v) + 2.0 ** -10 / c1[g] + 4 * 2.0 ** -24 * (np.abs(s) + np.abs(v))
+    assert np.all(np.abs(sh - s) <= bound)
+
+
+def test_double_quant_fp8_zero_group():
+    s = np.full(300, 0.25, np.float32)
+    c2, c1, mu = O.double_quantize_fp8(s)
+    assert mu == np.float32(0.25) and np.all(c2 == 0) and np.all(c1 == 1.0)
+    assert np.array_equal(O.double_dequantize_scales_fp8(c2, c1, mu), s)
+
+
 def test_storage_accounting(golden):
     g = golden("storage_accounting.json")
     before = O.storage_bits_per_weight(False)
