@@ -502,7 +502,7 @@ def run_secondary(args, wl_name):
             W = dev_bits(synth.weight(d, k, seed=pi, outliers=True))
             n = d * k
             nblk = -(-n // 64)
-            for dq in (True, False):
+            for dq in (1, 2, 0):   # Int8 constants, E4M3 constants, DQ off
                 q = Q.nf4_alloc(d, k, dq, dev)
                 wsz = Q.qlora_nf4_sizes(d, k, 64, dq)[1]
                 qws = torch.empty(max(wsz, 16), dtype=torch.uint8, device=dev)
@@ -517,13 +517,14 @@ def run_secondary(args, wl_name):
                 consts = (nblk + 4 * (-(-nblk // 256)) + 4) if dq else 4 * nblk
                 qbytes = 2 * n + (n + 1) // 2 + consts + (2 * nblk * 2 if dq else 0)   # + bf16 scale scratch write/read
                 dbytes = (n + 1) // 2 + consts + 2 * n
-                results.append({"proj": f"{name}:{d}x{k}", "double_quant": dq,
+                results.append({"proj": f"{name}:{d}x{k}", "double_quant": bool(dq),
+                                "dq_format": ("off", "int8", "fp8")[dq],
                                 "quantize_ms": round(mq, 4), "quantize_gbs": round(qbytes / (mq * 1e-3) / 1e9, 1),
                                 "quantize_frac_hbm": round(qbytes / (mq * 1e-3) / 1e9 / hbm, 4),
                                 "dequantize_ms": round(md, 4), "dequantize_gbs": round(dbytes / (md * 1e-3) / 1e9, 1),
                                 "dequantize_frac_hbm": round(dbytes / (md * 1e-3) / 1e9 / hbm, 4)})
         metric, unit = "NF4 quantize GB/s (4096x11008, double quant)", "GB/s"
-        value = [x for x in results if x["proj"].startswith("rect") and x["double_quant"]][0]["quantize_gbs"]
+        value = [x for x in results if x["proj"].startswith("rect") and x["dq_format"] == "int8"][0]["quantize_gbs"]
     elif wl_name == "merge_sweep":
         work = synth.WORKLOADS[wl_name]
         r, alpha = work["r"], work["alpha"]

@@ -107,7 +107,7 @@ class NF4Weight:
     """Device buffers of one quantized weight (layout of ``qlora_nf4_t``)."""
     d: int
     k: int
-    double_quant: bool
+    double_quant: int          # 0: fp32 absmax; 1 (or True): Int8 c2; 2: FP8 E4M3 c2
     codes: torch.Tensor
     absmax: Optional[torch.Tensor] = None
     c2: Optional[torch.Tensor] = None
@@ -140,10 +140,12 @@ def nf4_alloc(d: int, k: int, double_quant: bool = True, device=None) -> NF4Weig
         # 16 extra bytes of slack keep vector accesses inside the allocation
         return torch.empty(max(n // esize, 1) + 16 // esize, dtype=dtype, device=device)
     codes = buf(sizes[0], torch.uint8, 1)
-    if double_quant:
-        return NF4Weight(d, k, True, codes, None, buf(sizes[2], torch.int8, 1), buf(sizes[3], torch.float32, 4),
+    mode = int(double_quant)
+    if mode:
+        c2_dtype = torch.uint8 if mode == 2 else torch.int8   # E4M3 bytes / Int8
+        return NF4Weight(d, k, mode, codes, None, buf(sizes[2], c2_dtype, 1), buf(sizes[3], torch.float32, 4),
                          buf(sizes[4], torch.float32, 4))
-    return NF4Weight(d, k, False, codes, buf(sizes[1], torch.float32, 4))
+    return NF4Weight(d, k, 0, codes, buf(sizes[1], torch.float32, 4))
 
 
 def nf4_quantize(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4Weight] = None,

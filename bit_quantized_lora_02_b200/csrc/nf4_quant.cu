@@ -18,13 +18,17 @@
 //   k_dq_groups    warp 0 of each CTA: exact sum of the histogram in 32-bit
 //                  limbs, rounded once to fp64, divided, rounded to fp32 (the
 //                  mean); then one warp per group of 256 scales: subtract the
-//                  mean, absmax, c1 = 127 / absmax, c2 = round-half-even(c1 v).
+//                  mean, absmax, c1 = 127 / absmax, c2 = round-half-even(c1 v);
+//                  with E4M3 constants (the page's "c2_FP8" label) c1 =
+//                  448 / absmax and c2 = E4M3(c1 v), nearest even.
 //   k_nf4_dequant  one pass over the codes: scale reconstruction and
 //                  BF16(C[q] * s^), 16-byte vector stores.
 #include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+
+#include <cuda_fp8.h>
 
 #include "nf4_table.h"
 #include "qlora_device.cuh"
@@ -370,6 +374,10 @@ __device__ float exact_mean_warp(const unsigned long long* __restrict__ hist, in
 // ----------------------------------------------------------------------------
 // Double quantisation of the scales: one warp per group of 256.
 // ----------------------------------------------------------------------------
+// kFP8: the constants are E4M3 bytes, c1 = RN32(448 / max|v|) and
+// c2 = E4M3(RN32(c1 v)) rounded to nearest even, saturating at 448 (c1 v can
+// pass 448 only by an fp32 rounding).  Otherwise symmetric Int8 as above.
+template <bool kFP8>
 __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ absmax_bf16, int64_t nblocks,
                                                    const unsigned long long* __restrict__ hist,
                                                    float* __restrict__ mean_out, int8_t* __restrict__ c2,
@@ -412,16 +420,21 @@ __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ 
     for (int i = 0; i < 8; ++i) am = fmaxf(am, fabsf(v[i]));
 #pragma unroll
     for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-    const float c = (am == 0.0f) ? 1.0f : __fdiv_rn(127.0f, am);
+    const float c = (am == 0.0f) ? 1.0f : __fdiv_rn(kFP8 ? 448.0f : 127.0f, am);
     uint32_t lo = 0, hi = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      int q = 0;
-      if (am != 0.0f) {
-        q = __float2int_rn(__fmul_rn(c, v[i]));
-        q = max(-127, min(127, q));
+      uint32_t b;
+      if (kFP8) {
+        b = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fmul_rn(c, v[i]), __NV_SATFINITE, __NV_E4M3));
+      } else {
+        int q = 0;
+        if (am != 0.0f) {
+          q = __float2int_rn(__fmul_rn(c, v[i]));
+          q = max(-127, min(127, q));
+        }
+        b = static_cast<uint32_t>(q) & 0xFFu;
       }
-      const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
       if (i < 4) lo |= b << (8 * i);
       else hi |= b << (8 * (i - 4));
     }
@@ -439,7 +452,8 @@ __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ 
 // ----------------------------------------------------------------------------
 // Standalone double dequantisation: W_out[i] = BF16(RN32(C[q_i] * s^_j)).
 // ----------------------------------------------------------------------------
-template <bool kDQ>
+// kDQ: 0 = fp32 absmax per block, 1 = Int8 c2, 2 = E4M3 c2.
+template <int kDQ>
 __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__ codes, int64_t N,
                                                      const float* __restrict__ absmax, const int8_t* __restrict__ c2,
                                                      const float* __restrict__ c1, const float* __restrict__ mean,
@@ -460,8 +474,14 @@ __global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__
     const int64_t e0 = g << 3;
     const int64_t blk = e0 >> 6;
     float sh;
-    if (kDQ) sh = __fadd_rn(__fdiv_rn(static_cast<float>(c2[blk]), c1[blk >> 8]), mu);
-    else sh = absmax[blk];
+    if (kDQ == 1) {
+      sh = __fadd_rn(__fdiv_rn(static_cast<float>(c2[blk]), c1[blk >> 8]), mu);
+    } else if (kDQ == 2) {
+      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c2[blk]), __NV_E4M3);
+      sh = __fadd_rn(__fdiv_rn(__half2float(__half(hr)), c1[blk >> 8]), mu);   // E4M3 -> fp32 is exact
+    } else {
+      sh = absmax[blk];
+    }
     const bool full = (e0 + 8 <= N);
     uint32_t cw;
     if (full) {
@@ -535,8 +555,12 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
     // every CTA derives the mean itself, so keep the grid near one wave and loop over groups
     const int64_t want = (ngroups + 7) / 8;
     const int grid_g = static_cast<int>(want < 2 * num_sms() ? want : 2 * num_sms());
-    const cudaError_t e = launch_pdl(k_dq_groups, dim3(grid_g), dim3(256), 0, st, nullptr, amax16, nblk, hist,
-                                     q.mean, q.c2, q.c1);
+    const cudaError_t e =
+        q.double_quant == 2
+            ? launch_pdl(k_dq_groups<true>, dim3(grid_g), dim3(256), 0, st, nullptr, amax16, nblk, hist, q.mean, q.c2,
+                         q.c1)
+            : launch_pdl(k_dq_groups<false>, dim3(grid_g), dim3(256), 0, st, nullptr, amax16, nblk, hist, q.mean,
+                         q.c2, q.c1);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -546,10 +570,13 @@ cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cu
   const int grid = grid_for((N + 7) / 8);
   ProfScope ps_(QLORA_KC_DEQUANT, st);
   const cudaError_t e =
-      q.double_quant
-          ? launch_pdl(k_nf4_dequant<true>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
+      q.double_quant == 2
+          ? launch_pdl(k_nf4_dequant<2>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
                        static_cast<const float*>(nullptr), q.c2, q.c1, q.mean, out)
-          : launch_pdl(k_nf4_dequant<false>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, q.absmax,
+      : q.double_quant
+          ? launch_pdl(k_nf4_dequant<1>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
+                       static_cast<const float*>(nullptr), q.c2, q.c1, q.mean, out)
+          : launch_pdl(k_nf4_dequant<0>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, q.absmax,
                        static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
                        static_cast<const float*>(nullptr), out);
   if (e != cudaSuccess) return e;

@@ -94,8 +94,8 @@ static int check_nf4(const qlora_nf4_t* q, int64_t* N) {
   if (!elem_count(q->d, q->k, N)) return fail(QLORA_ERR_INVALID_ARG, "bad weight shape d=%lld k=%lld",
                                                 (long long)q->d, (long long)q->k);
   if (q->blocksize != 64) return fail(QLORA_ERR_UNSUPPORTED, "blocksize %d not supported (64 only)", q->blocksize);
-  if (q->double_quant != 0 && q->double_quant != 1)
-    return fail(QLORA_ERR_INVALID_ARG, "double_quant must be 0 or 1");
+  if (q->double_quant < 0 || q->double_quant > 2)
+    return fail(QLORA_ERR_INVALID_ARG, "double_quant must be 0, 1 or 2");
   if (*N == 0) return ok();
   if (!q->codes) return fail(QLORA_ERR_INVALID_ARG, "codes is NULL");
   if (!aligned(q->codes, 4)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 4-byte aligned");
@@ -118,7 +118,7 @@ int qlora_nf4_sizes(int64_t d, int64_t k, int32_t blocksize, int32_t double_quan
   if (!sizes) return fail(QLORA_ERR_INVALID_ARG, "sizes is NULL");
   if (!elem_count(d, k, &N)) return fail(QLORA_ERR_INVALID_ARG, "bad weight shape");
   if (blocksize != 64) return fail(QLORA_ERR_UNSUPPORTED, "blocksize %d not supported (64 only)", blocksize);
-  if (double_quant != 0 && double_quant != 1) return fail(QLORA_ERR_INVALID_ARG, "double_quant must be 0 or 1");
+  if (double_quant < 0 || double_quant > 2) return fail(QLORA_ERR_INVALID_ARG, "double_quant must be 0, 1 or 2");
   const int64_t nblk = ceil_div(N, 64);
   const int64_t ngrp = ceil_div(nblk, 256);
   sizes[QLORA_BUF_CODES] = static_cast<size_t>((N + 1) / 2);
@@ -207,6 +207,14 @@ int qlora_linear_workspace_size(int64_t M, int64_t d, int64_t k, int32_t r, int3
   return ok();
 }
 
+// E4M3 second-level constants are supported by quantisation and the standalone
+// dequantisation only; the fused kernels decode Int8 constants.
+static int check_dq_mode_fused(const qlora_nf4_t* q, const char* what) {
+  if (q->double_quant == 2)
+    return fail(QLORA_ERR_UNSUPPORTED, "%s: E4M3 second-level constants (double_quant = 2) are not supported", what);
+  return QLORA_OK;
+}
+
 // The tensor-core kernels read the packed codes with TMA: 16-byte alignment.
 static int check_codes_tma(const qlora_nf4_t* q) {
   if (!aligned(q->codes, 16)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 16-byte aligned for the linear layer");
@@ -225,6 +233,7 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const u
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
+  if ((rc = check_dq_mode_fused(q, "qlora_linear_fwd"))) return rc;
   if ((rc = check_linear_shape(M, q->d, q->k, r))) return rc;
   if (M == 0) return ok();
   if ((rc = check_codes_tma(q))) return rc;
@@ -252,6 +261,7 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlo
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
+  if ((rc = check_dq_mode_fused(q, "qlora_linear_bwd"))) return rc;
   if ((rc = check_linear_shape(M, q->d, q->k, r))) return rc;
   if ((rc = check_ptr16(dA, "dA", true)) || (rc = check_ptr16(dB, "dB", true))) return rc;
   if (M > 0 && (rc = check_codes_tma(q))) return rc;
@@ -280,6 +290,7 @@ int qlora_lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
+  if ((rc = check_dq_mode_fused(q, "qlora_lora_merge"))) return rc;
   if ((rc = check_linear_shape(0, q->d, q->k, r))) return rc;
   if (!aligned(q->codes, 16)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 16-byte aligned for the merge");
   if ((rc = check_ptr16(A, "A", true)) || (rc = check_ptr16(B, "B", true)) || (rc = check_ptr16(W_out, "W_out", true)))

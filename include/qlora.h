@@ -67,10 +67,13 @@ typedef void *qlora_stream_t;
  *           first); an odd N pads the last high nibble with 0.
  *   absmax: M_b = ceil(N/64) fp32 block scales (the block's max |w|); used and
  *           written only when double_quant == 0 (may be NULL otherwise).
- *   c2    : M_b int8 quantized deviations (s_j - mean) * c1[g], round half to
- *           even; DQ only.
- *   c1    : G = ceil(M_b/256) fp32 second-level scales, c1 = 127 / max|s - mean|
- *           over the group (1.0 for an all-zero group); DQ only.
+ *   c2    : M_b 8-bit quantized deviations (s_j - mean) * c1[g]; DQ only.
+ *           double_quant == 1: int8, round half to even.
+ *           double_quant == 2: OCP FP8 E4M3 bytes (the page's "c2_FP8"), round
+ *           to nearest even, saturating at 448.
+ *   c1    : G = ceil(M_b/256) fp32 second-level scales over the group, 127 /
+ *           max|s - mean| (Int8) or 448 / max|s - mean| (E4M3); 1.0 for an
+ *           all-zero group; DQ only.
  *   mean  : 1 fp32, the mean of all M_b block scales; DQ only.
  * All pointers are device pointers.  Alignment (checked on the host, else
  * QLORA_ERR_ALIGNMENT): codes 4 bytes for nf4_quantize / nf4_dequantize and
@@ -80,7 +83,10 @@ typedef struct {
   int64_t d;
   int64_t k;
   int32_t blocksize;     /* weights per NF4 block; only 64 is supported       */
-  int32_t double_quant;  /* 0: fp32 absmax per block; 1: int8 c2 + fp32 c1    */
+  int32_t double_quant;  /* 0: fp32 absmax per block; 1: int8 c2 + fp32 c1;   *
+                          * 2: E4M3 c2 + fp32 c1 (nf4_quantize, nf4_dequantize *
+                          * and the sizes query only; the linear layer and the *
+                          * merge return QLORA_ERR_UNSUPPORTED)                 */
   uint8_t *codes;
   float *absmax;
   int8_t *c2;

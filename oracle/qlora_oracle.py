@@ -316,21 +316,25 @@ def nf4_dequantize(codes: np.ndarray, scales: np.ndarray, blocksize: int = BLOCK
     return bf16_round_bits(prod)
 
 
-def quantize_tensor(w_bits: np.ndarray, double_quant: bool = True, blocksize: int = BLOCK) -> dict:
-    """Full quantisation of a bf16 weight (bits): codes, packed bytes and constants."""
+def quantize_tensor(w_bits: np.ndarray, double_quant: bool = True, blocksize: int = BLOCK,
+                    dq_fp8: bool = False) -> dict:
+    """Full quantisation of a bf16 weight (bits): codes, packed bytes and constants.
+    dq_fp8 selects E4M3 second-level constants instead of Int8."""
     w = bf16_bits_to_f32(np.asarray(w_bits).ravel())
     codes, absmax = nf4_quantize(w, blocksize)
     out = {"n": w.size, "codes": codes, "packed": pack_codes(codes), "absmax": absmax,
-           "double_quant": bool(double_quant)}
+           "double_quant": bool(double_quant), "dq_fp8": bool(double_quant and dq_fp8)}
     if double_quant:
-        c2, c1, mu = double_quantize(absmax)
+        c2, c1, mu = double_quantize_fp8(absmax) if dq_fp8 else double_quantize(absmax)
         out.update(c2=c2, c1=c1, mean=mu)
     return out
 
 
 def dequantize_tensor(q: dict, blocksize: int = BLOCK) -> np.ndarray:
     """doubleDequant (or single dequant when DQ is off); returns bf16 bits."""
-    if q["double_quant"]:
+    if q["double_quant"] and q.get("dq_fp8"):
+        scales = double_dequantize_scales_fp8(q["c2"], q["c1"], q["mean"])
+    elif q["double_quant"]:
         scales = double_dequantize_scales(q["c2"], q["c1"], q["mean"])
     else:
         scales = q["absmax"]

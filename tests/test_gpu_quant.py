@@ -14,20 +14,21 @@ if torch.cuda.is_available():
     from gpu_util import dev_bf16, gpu_quantized_arrays, host_bits
 
 
-def _roundtrip(bits: np.ndarray, dq: bool):
-    """GPU quantize + dequantize vs the oracle; all outputs bit-exact."""
+def _roundtrip(bits: np.ndarray, dq):
+    """GPU quantize + dequantize vs the oracle; all outputs bit-exact.
+    dq: False (fp32 absmax), True (Int8 constants) or 2 (E4M3 constants)."""
     d, k = bits.shape if bits.ndim == 2 else (1, bits.size)
     W = dev_bf16(bits.reshape(d, k))
     q = Q.nf4_quantize(W, double_quant=dq)
     Wh = Q.nf4_dequantize(q)
     torch.cuda.synchronize()
-    ref = O.quantize_tensor(bits.reshape(-1), double_quant=dq)
+    ref = O.quantize_tensor(bits.reshape(-1), double_quant=bool(dq), dq_fp8=(dq == 2))
     got = gpu_quantized_arrays(q, ref["n"])
     assert np.array_equal(got["packed"], ref["packed"]), "packed codes"
     if dq:
         assert np.array_equal(got["mean"].view(np.uint32), np.array([ref["mean"]], np.float32).view(np.uint32)), "mean"
         assert np.array_equal(got["c1"].view(np.uint32), ref["c1"].view(np.uint32)), "c1"
-        assert np.array_equal(got["c2"], ref["c2"]), "c2"
+        assert np.array_equal(got["c2"].view(np.uint8), ref["c2"].view(np.uint8)), "c2"
     else:
         assert np.array_equal(got["absmax"].view(np.uint32), ref["absmax"].view(np.uint32)), "absmax"
     ref_w = O.dequantize_tensor(ref)
@@ -36,14 +37,14 @@ def _roundtrip(bits: np.ndarray, dq: bool):
     return q
 
 
-@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("dq", [True, False, 2])
 def test_tiny_layer_weight(dq):
     """The tiny layer: W0 512 x 512 ~ N(0, 0.02), blocksize 64, DQ groups of 256."""
     _roundtrip(synth.weight(512, 512, seed=0), dq)
 
 
 @pytest.mark.parametrize("shape", [(3, 37), (5, 200), (1, 64 * 257 + 9), (7, 1000), (2, 8), (1, 1), (130, 64)])
-@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("dq", [True, False, 2])
 def test_ragged_sizes(shape, dq):
     """N not a multiple of 8 or 64, partial last DQ group, single element."""
     d, k = shape
@@ -58,13 +59,14 @@ def test_zero_blocks_and_signs():
     w[2, 128:192] = -np.abs(w[2, 128:192])
     w[3, :] = 0.0                    # whole rows of zeros
     w[4, 5] = 3.0                    # large outlier
-    for dq in (True, False):
+    for dq in (True, False, 2):
         _roundtrip(O.bf16_round_bits(w), dq)
 
 
-def test_all_zero_tensor():
+@pytest.mark.parametrize("dq", [True, 2])
+def test_all_zero_tensor(dq):
     bits = np.zeros((4, 256), np.uint16)
-    q = _roundtrip(bits, True)
+    q = _roundtrip(bits, dq)
     assert float(q.mean[0]) == 0.0
 
 
@@ -115,7 +117,7 @@ def test_subnormal_scales():
 
 
 @pytest.mark.parametrize("shape", [(4096, 4096), (4096, 11008)])
-@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("dq", [True, False, 2])
 def test_quant_sweep_full_size(shape, dq):
     """Quantisation sweep: W0 ~ N(0, 0.02) with 1% N(0, 0.2) outliers."""
     d, k = shape
