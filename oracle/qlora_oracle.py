@@ -42,6 +42,11 @@ R6  Scale reconstruction s^_j = RN32(RN32(c2_j / c1_g) + mu);
 R7  Forward Y = X W^T + (alpha/r) (X A^T) B^T with W^ the reconstructed bf16
     weights; backward derived by calculus (the pages print no formulas):
     U = dY B, dX = dY W^ + s U A, dA = s U^T X, dB = s dY^T T, T = X A^T.
+R8  Merge ([QLoRA-chkda] "Merging LoRA weights for inference"): the base is
+    the reconstructed W^, W_merged = W^ + s B A.
+R9  FP8 second-level constants (the page's "c2_FP8" label): OCP E4M3 bytes,
+    c1 = RN32(448 / max|v|) per group, c2 = E4M3(RN32(c1 v)) nearest even,
+    saturating at 448; s^ = RN32(RN32(decode(c2) / c1) + mean).
 """
 from __future__ import annotations
 
