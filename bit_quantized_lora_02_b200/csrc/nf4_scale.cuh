@@ -49,8 +49,10 @@ __device__ __forceinline__ ScaleRaw scale_fetch(const ScaleSrc& s, int64_t blk) 
 // blocks, so it changes rarely), and one residual correction:
 //     y = RN(c2 rc);  e = fma(-c1, y, c2);  q = fma(e, rc, y).
 // For integer |c2| <= 127 and c1 in [2^-60, 2^60] this equals IEEE division
-// for every fp32 significand of c1 (checked exhaustively on the host); outside
-// that range the IEEE division is used.
+// for every fp32 significand of c1, and so it does for every finite E4M3 value
+// as numerator (a zero numerator of either sign gives +0, which leaves
+// RN(q + mean) unchanged); tests/host_checks/division_check.c checks both
+// exhaustively.  Outside that range the IEEE division is used.
 struct ScaleRecip {
   float c1 = 0.0f;   // constant the reciprocal belongs to (0 never occurs: c1 > 0)
   float rc = 0.0f;
