@@ -47,6 +47,10 @@ R8  Merge ([QLoRA-chkda] "Merging LoRA weights for inference"): the base is
 R9  FP8 second-level constants (the page's "c2_FP8" label): OCP E4M3 bytes,
     c1 = RN32(448 / max|v|) per group, c2 = E4M3(RN32(c1 v)) nearest even,
     saturating at 448; s^ = RN32(RN32(decode(c2) / c1) + mean).
+R10 Adapter dropout ([FromZero2AI] lora_dropout): on the adapter input only,
+    keep decisions from Philox4x32-10 keyed by (seed, offset) and the flat
+    element index, kept values scaled by RN32(1 / RN32(1 - p)); the backward
+    reuses the same decisions.
 """
 from __future__ import annotations
 
@@ -62,6 +66,7 @@ __all__ = [
     "nf4_dequantize", "quantize_tensor", "dequantize_tensor", "storage_bits_per_weight",
     "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale", "lora_merge",
     "FP8_MAX", "fp8_e4m3_encode", "fp8_e4m3_decode", "double_quantize_fp8", "double_dequantize_scales_fp8",
+    "philox4x32_10", "dropout_keep", "dropout_scale", "qlora_forward_dropout", "qlora_backward_dropout",
 ]
 
 BLOCK = 64          # weights per NF4 block ([QLoRA-chkda] "QLoRA uses blocks of 64 weights")
@@ -411,3 +416,77 @@ def lora_merge(W_hat, A, B, alpha: float, r: int):
     W_hat, A, B = map(_f64, (W_hat, A, B))
     s = float(lora_scale(alpha, r))
     return W_hat + s * (B @ A)
+
+
+# ----------------------------------------------------------------------------
+# Adapter dropout  ([FromZero2AI] LoRA configuration, lora_dropout = 0.05):
+# dropout on the adapter's input only, h = W x + s B A drop(x), as a PEFT-style
+# LoRA layer applies it.  The pages name no random-number generator; the keep
+# decisions come from the counter-based Philox4x32-10 generator (Salmon, Moraes,
+# Dror and Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), so a
+# kernel can regenerate the decision for any element from (seed, offset, flat
+# index) and the backward needs no stored mask.
+# ----------------------------------------------------------------------------
+PHILOX_MUL = (0xD2511F53, 0xCD9E8D57)
+PHILOX_WEYL = (0x9E3779B9, 0xBB67AE85)
+
+
+def philox4x32_10(ctr: np.ndarray, key) -> np.ndarray:
+    """Philox4x32 with 10 rounds: ctr (N, 4) uint32, key (2,) -> (N, 4) uint32."""
+    c = [np.asarray(ctr, np.uint64)[:, i].copy() for i in range(4)]
+    k0, k1 = np.uint64(int(key[0]) & 0xFFFFFFFF), np.uint64(int(key[1]) & 0xFFFFFFFF)
+    m0, m1 = np.uint64(PHILOX_MUL[0]), np.uint64(PHILOX_MUL[1])
+    mask = np.uint64(0xFFFFFFFF)
+    for rnd in range(10):
+        p0, p1 = m0 * c[0], m1 * c[2]                 # exact 64-bit products of 32-bit words
+        hi0, lo0 = p0 >> np.uint64(32), p0 & mask
+        hi1, lo1 = p1 >> np.uint64(32), p1 & mask
+        c = [(hi1 ^ c[1] ^ k0) & mask, lo1, (hi0 ^ c[3] ^ k1) & mask, lo0]
+        if rnd < 9:
+            k0 = (k0 + np.uint64(PHILOX_WEYL[0])) & mask
+            k1 = (k1 + np.uint64(PHILOX_WEYL[1])) & mask
+    return np.stack(c, axis=1).astype(np.uint32)
+
+
+def dropout_keep(M: int, k: int, p: float, seed: int, offset: int = 0) -> np.ndarray:
+    """Keep mask (M x k, bool) for dropout probability p.  Element i = m k + j
+    uses word i % 4 of Philox4x32-10 at counter (i // 4 low and high 32 bits,
+    offset low and high 32 bits) under key (seed low and high 32 bits); with
+    u = (word >> 8) 2^-24 (uniform on [0, 1) with 24 bits, exact in fp32) the
+    element is kept when u >= RN32(p)."""
+    n = M * k
+    q = np.arange((n + 3) // 4, dtype=np.uint64)
+    ctr = np.stack([q & np.uint64(0xFFFFFFFF), q >> np.uint64(32),
+                    np.full_like(q, offset & 0xFFFFFFFF), np.full_like(q, (offset >> 32) & 0xFFFFFFFF)], axis=1)
+    words = philox4x32_10(ctr, (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)).reshape(-1)[:n]
+    u = (words >> np.uint32(8)).astype(np.float64) * 2.0 ** -24
+    return (u >= float(np.float32(p))).reshape(M, k)
+
+
+def dropout_scale(p: float) -> np.float32:
+    """Scale of the kept activations: RN32(1 / RN32(1 - p))."""
+    return np.float32(np.float32(1.0) / np.float32(np.float32(1.0) - np.float32(p)))
+
+
+def qlora_forward_dropout(X, W_hat, A, B, alpha: float, r: int, keep: np.ndarray, p: float):
+    """Y = X W^T + s (drop(X) A^T) B^T with drop(X) = X * keep * scale; returns
+    (Y, T) in fp64, T = drop(X) A^T."""
+    X, W_hat, A, B = map(_f64, (X, W_hat, A, B))
+    s = float(lora_scale(alpha, r))
+    Xd = X * keep * float(dropout_scale(p))
+    T = Xd @ A.T
+    return X @ W_hat.T + s * (T @ B.T), T
+
+
+def qlora_backward_dropout(dY, X, W_hat, A, B, alpha: float, r: int, keep: np.ndarray, p: float):
+    """Gradients of qlora_forward_dropout for a fixed mask: dX, dA, dB."""
+    dY, X, W_hat, A, B = map(_f64, (dY, X, W_hat, A, B))
+    s = float(lora_scale(alpha, r))
+    g = keep * float(dropout_scale(p))
+    Xd = X * g
+    T = Xd @ A.T
+    U = dY @ B
+    dX = dY @ W_hat + s * (U @ A) * g
+    dA = s * (U.T @ Xd)
+    dB = s * (dY.T @ T)
+    return dX, dA, dB

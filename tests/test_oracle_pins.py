@@ -335,6 +335,78 @@ def test_double_quant_fp8_zero_group():
     assert np.array_equal(O.double_dequantize_scales_fp8(c2, c1, mu), s)
 
 
+# Known-answer vectors of Philox4x32-10, as published with the generator's
+# reference implementation (Salmon, Moraes, Dror and Shaw, "Parallel Random
+# Numbers: As Easy as 1, 2, 3", SC 2011): (counter, key) -> output.
+PHILOX_KAT = [
+    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
+     (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+    ((0xffffffff, 0xffffffff, 0xffffffff, 0xffffffff), (0xffffffff, 0xffffffff),
+     (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+]
+
+
+def test_philox_known_answers():
+    for ctr, key, want in PHILOX_KAT:
+        got = O.philox4x32_10(np.array([ctr], np.uint32), key)[0]
+        assert [int(v) for v in got] == list(want)
+
+
+def test_dropout_keep_fraction():
+    n, p = 1 << 20, 0.05
+    keep = O.dropout_keep(1024, 1024, p, seed=77)
+    assert keep.shape == (1024, 1024)
+    assert abs(keep.mean() - (1 - p)) <= 5 * np.sqrt(p * (1 - p) / n)
+
+
+def test_dropout_keep_structure():
+    a = O.dropout_keep(12, 40, 0.3, seed=5)
+    assert np.array_equal(a, O.dropout_keep(1, 480, 0.3, seed=5).reshape(12, 40))   # flat index only
+    assert not np.array_equal(a, O.dropout_keep(12, 40, 0.3, seed=6))
+    assert not np.array_equal(a, O.dropout_keep(12, 40, 0.3, seed=5, offset=1))
+    assert O.dropout_keep(7, 9, 0.0, seed=1).all()
+    assert not O.dropout_keep(7, 9, 1.0, seed=1).any()
+    # a larger p keeps a subset of what a smaller p keeps (same draws)
+    assert not (O.dropout_keep(12, 40, 0.6, seed=5) & ~a).any()
+
+
+def test_dropout_p0_is_the_plain_layer():
+    X, W, A, B, dY = _tiny(11)
+    keep = np.ones(X.shape, bool)
+    Y, T = O.qlora_forward_dropout(X, W, A, B, 16.0, 3, keep, 0.0)
+    Y0, T0 = O.qlora_forward(X, W, A, B, 16.0, 3)
+    assert np.array_equal(Y, Y0) and np.array_equal(T, T0)
+    for g, g0 in zip(O.qlora_backward_dropout(dY, X, W, A, B, 16.0, 3, keep, 0.0),
+                     O.qlora_backward(dY, X, W, A, B, 16.0, 3)):
+        assert np.array_equal(g, g0)
+
+
+def test_dropout_backward_finite_differences():
+    X, W, A, B, dY = _tiny(12)
+    keep = O.dropout_keep(*X.shape, 0.4, seed=3)
+    assert keep.any() and not keep.all()
+    dX, dA, dB = O.qlora_backward_dropout(dY, X, W, A, B, 16.0, 3, keep, 0.4)
+
+    def loss(X_, A_, B_):
+        Y, _ = O.qlora_forward_dropout(X_, W, A_, B_, 16.0, 3, keep, 0.4)
+        return float(np.sum(Y * dY))
+
+    h = 1e-6
+    for arr, grad in ((X, dX), (A, dA), (B, dB)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + h
+            lp = loss(X, A, B)
+            arr[idx] = old - h
+            lm = loss(X, A, B)
+            arr[idx] = old
+            num[idx] = (lp - lm) / (2 * h)
+        assert np.allclose(num, grad, rtol=1e-6, atol=1e-6)
+
+
 def test_storage_accounting(golden):
     g = golden("storage_accounting.json")
     before = O.storage_bits_per_weight(False)
