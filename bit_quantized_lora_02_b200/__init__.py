@@ -93,6 +93,26 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _expect(t: Optional[torch.Tensor], name: str, shape, dtype, required: bool = True) -> None:
+    """The C ABI sees raw pointers only: check dtype, exact shape and row-major
+    contiguity here, so that a mismatched tensor raises instead of being read
+    or written past its end."""
+    if t is None:
+        if required:
+            raise ValueError(f"{name} is required")
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(int(x) for x in shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def _stream(stream) -> Optional[int]:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -154,12 +174,13 @@ def nf4_quantize(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4W
     assert W0.dtype == torch.bfloat16 and W0.dim() == 2 and W0.is_contiguous()
     d, k = W0.shape
     q = out or nf4_alloc(d, k, double_quant, W0.device)
+    if (q.d, q.k) != (d, k):
+        raise ValueError(f"out describes a {q.d}x{q.k} weight, W0 is {d}x{k}")
     _, ws_bytes = qlora_nf4_sizes(d, k, 64, q.double_quant)
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=W0.device)
     st = q.struct()
-    _check(lib().nf4_quantize(W0.data_ptr(), ctypes.byref(st), _ptr(workspace),
-                              0 if workspace is None else workspace.numel() * workspace.element_size(),
+    _check(lib().nf4_quantize(W0.data_ptr(), ctypes.byref(st), _ptr(workspace), _nbytes(workspace),
                               _stream(stream)))
     return q
 
@@ -185,6 +206,7 @@ def nf4_dequantize(q: NF4Weight, out: Optional[torch.Tensor] = None, stream=None
     """doubleDequant into a bf16 (d, k) tensor."""
     if out is None:
         out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
+    _expect(out, "out", (q.d, q.k), torch.bfloat16)
     st = q.struct()
     _check(lib().nf4_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)))
     return out
@@ -196,6 +218,9 @@ def qlora_lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: floa
     r = A.shape[0]
     if out is None:
         out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
+    _expect(A, "A", (r, q.k), torch.bfloat16)
+    _expect(B, "B", (q.d, r), torch.bfloat16)
+    _expect(out, "out", (q.d, q.k), torch.bfloat16)
     st = q.struct()
     _check(lib().qlora_lora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha), out.data_ptr(),
                                   _stream(stream)))
@@ -223,13 +248,17 @@ def qlora_linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Te
         Y = torch.empty(M, q.d, dtype=torch.bfloat16, device=dev)
     if T_save is None and save_T:
         T_save = torch.empty(M, qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
+    _expect(X, "X", (M, q.k), torch.bfloat16)
+    _expect(A, "A", (r, q.k), torch.bfloat16)
+    _expect(B, "B", (q.d, r), torch.bfloat16)
+    _expect(Y, "Y", (M, q.d), torch.bfloat16)
+    _expect(T_save, "T_save", (M, qlora_rank_pad(r)), torch.bfloat16, required=False)
     if workspace is None:
         n = qlora_linear_workspace_size(M, q.d, q.k, r, False)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
     st = q.struct()
     _check(lib().qlora_linear_fwd(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha),
-                                  Y.data_ptr(), _ptr(T_save), _ptr(workspace),
-                                  0 if workspace is None else workspace.numel(), _stream(stream)))
+                                  Y.data_ptr(), _ptr(T_save), _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return Y, T_save
 
 
@@ -247,13 +276,21 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.T
         dA = torch.empty(r, q.k, dtype=torch.float32, device=dev)
     if dB is None:
         dB = torch.empty(q.d, r, dtype=torch.float32, device=dev)
+    _expect(dY, "dY", (M, q.d), torch.bfloat16)
+    _expect(X, "X", (M, q.k), torch.bfloat16, required=False)
+    _expect(A, "A", (r, q.k), torch.bfloat16)
+    _expect(B, "B", (q.d, r), torch.bfloat16)
+    _expect(T_save, "T_save", (M, qlora_rank_pad(r)), torch.bfloat16, required=False)
+    _expect(dX, "dX", (M, q.k), torch.bfloat16, required=False)
+    _expect(dA, "dA", (r, q.k), torch.float32)
+    _expect(dB, "dB", (q.d, r), torch.float32)
     if workspace is None:
         n = qlora_linear_workspace_size(M, q.d, q.k, r, True)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
     st = q.struct()
     _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
                                   float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
-                                  _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream(stream)))
+                                  _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return dX, dA, dB
 
 
