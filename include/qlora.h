@@ -14,8 +14,10 @@
  *     "NF4: Choose the codebook to fit the distribution" (the 16-value table),
  *     "Quantizing and dequantizing with the codebook" (blockwise NF4, blocks of 64),
  *     "Double quantization and double dequantization" (8-bit block constants in
- *       groups of 256 with an FP32 second-level scale and a stored mean; the
- *       QLoRA expression; backpropagation through the reconstructed base).
+ *       groups of 256 with an FP32 second-level scale and a stored mean, Int8 or
+ *       the "c2_FP8" E4M3 variant; the QLoRA expression; backpropagation through
+ *       the reconstructed base),
+ *     "Merging LoRA weights for inference" (qlora_lora_merge).
  *   "LoRA and QLoRA: Efficient Fine-Tuning of Large Language Models"
  *     (fromzero2ai.dev): section "Low-Rank Matrix Factorization".
  *
