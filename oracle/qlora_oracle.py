@@ -64,7 +64,7 @@ __all__ = [
     "nearest_code", "nf4_quantize", "pack_codes", "unpack_codes", "int8_absmax_quantize",
     "int8_dequantize", "exact_mean_f32", "double_quantize", "double_dequantize_scales",
     "nf4_dequantize", "quantize_tensor", "dequantize_tensor", "storage_bits_per_weight",
-    "lora_trainable_params", "qlora_forward", "qlora_backward", "lora_scale", "lora_merge",
+    "lora_trainable_params", "qlora_forward", "qlora_backward", "qlora_adapter_grads", "lora_scale", "lora_merge",
     "FP8_MAX", "fp8_e4m3_encode", "fp8_e4m3_decode", "double_quantize_fp8", "double_dequantize_scales_fp8",
     "philox4x32_10", "dropout_keep", "dropout_scale", "qlora_forward_dropout", "qlora_backward_dropout",
 ]
@@ -391,15 +391,23 @@ def qlora_forward(X, W_hat, A, B, alpha: float, r: int):
     return X @ W_hat.T + s * (T @ B.T), T
 
 
+def qlora_adapter_grads(dY, X, A, B, alpha: float, r: int):
+    """The adapter gradients alone (no base weight involved):
+    dA = s (dY B)^T X and dB = s dY^T (X A^T); returns (dA, dB) in fp64."""
+    dY, X, A, B = map(_f64, (dY, X, A, B))
+    s = float(lora_scale(alpha, r))
+    T = X @ A.T
+    U = dY @ B
+    return s * (U.T @ X), s * (dY.T @ T)
+
+
 def qlora_backward(dY, X, W_hat, A, B, alpha: float, r: int):
     """Gradients of the forward for the frozen base (no dW0): returns dX, dA, dB."""
     dY, X, W_hat, A, B = map(_f64, (dY, X, W_hat, A, B))
     s = float(lora_scale(alpha, r))
-    T = X @ A.T
     U = dY @ B
     dX = dY @ W_hat + s * (U @ A)
-    dA = s * (U.T @ X)
-    dB = s * (dY.T @ T)
+    dA, dB = qlora_adapter_grads(dY, X, A, B, alpha, r)
     return dX, dA, dB
 
 

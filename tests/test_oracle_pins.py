@@ -194,6 +194,66 @@ def test_roundtrip_error_bound():
     assert np.max(half) == pytest.approx(0.15190, abs=5e-5)
 
 
+def _bf16_rational(bits32: int) -> int:
+    """Nearest bf16 (ties to even) of one finite fp32 bit pattern, decided on
+    exact rationals between the two bf16 neighbours of the magnitude."""
+    sign, mag = bits32 & 0x80000000, bits32 & 0x7FFFFFFF
+    x = Fraction(float(np.array(mag, np.uint32).view(np.float32)))
+    lo = mag >> 16
+    hi = lo + 1
+
+    def val(b):
+        if b >= 0x7F80:
+            return None                       # rounding up past the largest finite value overflows
+        return Fraction(float(np.array(b << 16, np.uint32).view(np.float32)))
+    vlo, vhi = val(lo), val(hi)
+    if vhi is None:
+        # beyond the largest finite bf16: round to nearest with the overflow
+        # threshold halfway to 2^128
+        vhi = Fraction(2) ** 128
+    dlo, dhi = x - vlo, vhi - x
+    pick = lo if (dlo < dhi or (dlo == dhi and lo % 2 == 0)) else hi
+    return (sign >> 16) | pick
+
+
+def test_bf16_rounding_ties_and_carries():
+    """Every tie pattern (low 16 bits exactly 0x8000) at every finite exponent,
+    both parities of the kept last bit, with and without a carry into the
+    exponent, both signs; plus the patterns one step off the tie.  Checked
+    against exact-rational rounding and against PyTorch's fp32 -> bf16."""
+    import torch
+    pats = []
+    for e in range(0, 255):
+        for m_hi in (0x00, 0x01, 0x3E, 0x3F, 0x40, 0x7E, 0x7F):
+            for low in (0x8000, 0x7FFF, 0x8001, 0x0000, 0xFFFF):
+                for sign in (0, 0x80000000):
+                    pats.append(sign | (e << 23) | (m_hi << 16) | low)
+    u = np.array(pats, np.uint32)
+    x = u.view(np.float32)
+    got = O.bf16_round_bits(x)
+    want = np.array([_bf16_rational(int(b)) for b in pats], np.uint16)
+    assert np.array_equal(got, want)
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    # a tie with an odd kept bit rounds up and one with an even kept bit down
+    assert O.bf16_round_bits(np.array([0x3F818000], np.uint32).view(np.float32))[0] == 0x3F82
+    assert O.bf16_round_bits(np.array([0x3F808000], np.uint32).view(np.float32))[0] == 0x3F80
+    # the carry out of the mantissa moves into the exponent
+    assert O.bf16_round_bits(np.array([0x3FFF8000], np.uint32).view(np.float32))[0] == 0x4000
+
+
+def test_bf16_rounding_wide_sample():
+    import torch
+    rng = np.random.default_rng(17)
+    u = rng.integers(0, 1 << 32, size=1 << 20, dtype=np.uint64).astype(np.uint32)
+    u = u[(u & 0x7F800000) != 0x7F800000]            # finite inputs only
+    x = u.view(np.float32)
+    ref = torch.from_numpy(x.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.bf16_round_bits(x), ref)
+    for b in u[:2000].tolist():
+        assert O.bf16_round_bits(np.array([b], np.uint32).view(np.float32))[0] == _bf16_rational(b)
+
+
 def test_nf4_beats_uniform_codebook_on_gaussian_blocks():
     """Contrast from the page: finer spacing near zero lowers the error on
     bell-shaped blocks compared with 16 evenly spaced values."""
@@ -405,6 +465,30 @@ def test_dropout_backward_finite_differences():
             arr[idx] = old
             num[idx] = (lp - lm) / (2 * h)
         assert np.allclose(num, grad, rtol=1e-6, atol=1e-6)
+
+
+def test_dropout_scale_against_exact_rationals():
+    """RN32(1 / RN32(1 - p)): both roundings taken on exact rationals; a scale
+    of (1 - p) instead of its reciprocal, or a missing rounding, fails."""
+    for p in (0.05, 0.1, 0.5, 0.3, 0.9):
+        p32 = Fraction(float(np.float32(p)))
+        one_minus = rn32(Fraction(1) - p32)
+        want = rn32(Fraction(1) / Fraction(float(one_minus)))
+        got = O.dropout_scale(p)
+        assert got.dtype == np.float32
+        assert got.view(np.uint32) == want.view(np.uint32), p
+    assert O.dropout_scale(0.0) == np.float32(1.0)
+    assert O.dropout_scale(0.5) == np.float32(2.0)
+
+
+def test_dropout_preserves_the_mean():
+    """Inverted dropout keeps E[drop(x)] = x: over 2^20 elements the mean of
+    keep * scale is 1 within 5 sigma (sigma = scale sqrt(p (1 - p) / n))."""
+    n, p = 1 << 20, 0.05
+    keep = O.dropout_keep(1024, 1024, p, seed=123)
+    scale = float(O.dropout_scale(p))
+    m = float(np.mean(keep * scale))
+    assert abs(m - 1.0) <= 5 * scale * np.sqrt(p * (1 - p) / n)
 
 
 def test_storage_accounting(golden):
