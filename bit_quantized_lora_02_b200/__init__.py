@@ -109,6 +109,13 @@ def _expect(t: Optional[torch.Tensor], name: str, shape, dtype, required: bool =
         raise ValueError(f"{name} must be contiguous (row-major)")
 
 
+def _same_device(dev, **tensors) -> None:
+    """Every pointer of one call must live on the device the call runs on."""
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the call runs on {dev}")
+
+
 def _nbytes(t: Optional[torch.Tensor]) -> int:
     return 0 if t is None else t.numel() * t.element_size()
 
@@ -135,8 +142,36 @@ class NF4Weight:
     mean: Optional[torch.Tensor] = None
     blocksize: int = 64
 
-    def struct(self) -> QloraNF4:
-        return QloraNF4(self.d, self.k, self.blocksize, int(self.double_quant), _ptr(self.codes), _ptr(self.absmax),
+    def struct(self, device=None) -> QloraNF4:
+        """The C struct, after checking every buffer against the sizes the
+        library needs for a d x k weight in this mode: dtype, byte size,
+        contiguity and device (``device``: the activations' device, when the
+        call has activations).  A short or misplaced buffer raises here instead
+        of being read or written past its end."""
+        mode = int(self.double_quant)
+        if mode not in (0, 1, 2):
+            raise ValueError(f"double_quant must be 0, 1 or 2, got {self.double_quant!r}")
+        sizes, _ = qlora_nf4_sizes(self.d, self.k, self.blocksize, mode)
+        dev = self.codes.device if device is None else torch.device(device)
+        want = [("codes", self.codes, sizes[0], (torch.uint8,)),
+                ("absmax", self.absmax, sizes[1], (torch.float32,)),
+                ("c2", self.c2, sizes[2], (torch.uint8,) if mode == 2 else (torch.int8,)),
+                ("c1", self.c1, sizes[3], (torch.float32,)),
+                ("mean", self.mean, sizes[4], (torch.float32,))]
+        for name, t, need, dtypes in want:
+            if need == 0:
+                continue
+            if t is None:
+                raise ValueError(f"NF4Weight.{name} is required for double_quant={mode}")
+            if t.dtype not in dtypes:
+                raise ValueError(f"NF4Weight.{name}: dtype {t.dtype}, expected {dtypes[0]}")
+            if not t.is_contiguous():
+                raise ValueError(f"NF4Weight.{name} must be contiguous")
+            if t.device != dev:
+                raise ValueError(f"NF4Weight.{name} is on {t.device}, the call runs on {dev}")
+            if _nbytes(t) < need:
+                raise ValueError(f"NF4Weight.{name}: {_nbytes(t)} bytes, a {self.d}x{self.k} weight needs {need}")
+        return QloraNF4(self.d, self.k, self.blocksize, mode, _ptr(self.codes), _ptr(self.absmax),
                         _ptr(self.c2), _ptr(self.c1), _ptr(self.mean))
 
     def nbytes(self) -> int:
@@ -179,7 +214,9 @@ def nf4_quantize(W0: torch.Tensor, double_quant: bool = True, out: Optional[NF4W
     _, ws_bytes = qlora_nf4_sizes(d, k, 64, q.double_quant)
     if workspace is None and ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=W0.device)
-    st = q.struct()
+    if workspace is not None and workspace.device != W0.device:
+        raise ValueError(f"workspace is on {workspace.device}, W0 on {W0.device}")
+    st = q.struct(W0.device)
     _check(lib().nf4_quantize(W0.data_ptr(), ctypes.byref(st), _ptr(workspace), _nbytes(workspace),
                               _stream(stream)))
     return q
@@ -197,7 +234,11 @@ def nf4_quantize_noalloc(W0: torch.Tensor, double_quant: bool = True, out: Optio
     assert W0.dtype == torch.bfloat16 and W0.dim() == 2 and W0.is_contiguous()
     d, k = W0.shape
     q = out or nf4_alloc(d, k, double_quant, W0.device)
-    st = q.struct()
+    if (q.d, q.k) != (d, k):
+        raise ValueError(f"out describes a {q.d}x{q.k} weight, W0 is {d}x{k}")
+    if int(q.double_quant) != int(double_quant):
+        raise ValueError(f"out holds double_quant={int(q.double_quant)} buffers, the call asks for {int(double_quant)}")
+    st = q.struct(W0.device)
     _check(lib().nf4_quantize_noalloc(W0.data_ptr(), ctypes.byref(st), _stream(stream)))
     return q
 
@@ -207,7 +248,7 @@ def nf4_dequantize(q: NF4Weight, out: Optional[torch.Tensor] = None, stream=None
     if out is None:
         out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device)
     _expect(out, "out", (q.d, q.k), torch.bfloat16)
-    st = q.struct()
+    st = q.struct(out.device)
     _check(lib().nf4_dequantize(ctypes.byref(st), out.data_ptr(), _stream(stream)))
     return out
 
@@ -221,7 +262,8 @@ def qlora_lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: floa
     _expect(A, "A", (r, q.k), torch.bfloat16)
     _expect(B, "B", (q.d, r), torch.bfloat16)
     _expect(out, "out", (q.d, q.k), torch.bfloat16)
-    st = q.struct()
+    _same_device(out.device, A=A, B=B)
+    st = q.struct(out.device)
     _check(lib().qlora_lora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha), out.data_ptr(),
                                   _stream(stream)))
     return out
@@ -256,7 +298,8 @@ def qlora_linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Te
     if workspace is None:
         n = qlora_linear_workspace_size(M, q.d, q.k, r, False)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
-    st = q.struct()
+    _same_device(dev, A=A, B=B, Y=Y, T_save=T_save, workspace=workspace)
+    st = q.struct(dev)
     _check(lib().qlora_linear_fwd(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha),
                                   Y.data_ptr(), _ptr(T_save), _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return Y, T_save
@@ -277,7 +320,7 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.T
     if dB is None:
         dB = torch.empty(q.d, r, dtype=torch.float32, device=dev)
     _expect(dY, "dY", (M, q.d), torch.bfloat16)
-    _expect(X, "X", (M, q.k), torch.bfloat16, required=False)
+    _expect(X, "X", (M, q.k), torch.bfloat16)
     _expect(A, "A", (r, q.k), torch.bfloat16)
     _expect(B, "B", (q.d, r), torch.bfloat16)
     _expect(T_save, "T_save", (M, qlora_rank_pad(r)), torch.bfloat16, required=False)
@@ -287,7 +330,8 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.T
     if workspace is None:
         n = qlora_linear_workspace_size(M, q.d, q.k, r, True)
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
-    st = q.struct()
+    _same_device(dev, X=X, A=A, B=B, T_save=T_save, dX=dX, dA=dA, dB=dB, workspace=workspace)
+    st = q.struct(dev)
     _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
                                   float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
                                   _ptr(workspace), _nbytes(workspace), _stream(stream)))

@@ -26,7 +26,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <mutex>
 
 #include <cuda_fp8.h>
 
@@ -597,9 +596,13 @@ cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cu
 // every GPU that loads the library until the process exits).
 //
 // Host code must not pass the array's name to a kernel: on the host that name
-// is only a stand-in, not a device address.  The first call on each device
-// (with that device current) asks the runtime for the real address with
-// cudaGetSymbolAddress and caches it.
+// is only a stand-in, not a device address.  Every call asks the runtime for
+// the real address with cudaGetSymbolAddress, with the call's device current.
+// That is a host-side lookup (it allocates nothing); the first one on a device
+// may load the library's device code there.  The address is not cached: after
+// the caller destroys and recreates the device's context (cudaDeviceReset, for
+// instance) the module is loaded again and the array may sit elsewhere, and a
+// cached address would then point at freed memory.
 // ----------------------------------------------------------------------------
 constexpr size_t noalloc_scratch_bytes() {
   return 256 * sizeof(unsigned long long) +
@@ -608,22 +611,11 @@ constexpr size_t noalloc_scratch_bytes() {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[noalloc_scratch_bytes()];
 
-static std::mutex g_noalloc_mu;
-static void* g_noalloc_addr[64] = {};
-
 cudaError_t noalloc_scratch(void** out, size_t* bytes) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_noalloc_addr[dev] = p;
-  }
-  *out = g_noalloc_addr[dev];
+  *out = p;
   *bytes = noalloc_scratch_bytes();
   return cudaSuccess;
 }

@@ -10,6 +10,7 @@
 
 #include <cstdint>
 
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include "qlora_device.cuh"
@@ -59,6 +60,15 @@ struct ScaleRecip {
   bool fast = false;
 };
 
+// c2 as the numerator: the int8 value, or the E4M3 byte decoded (exact).
+__device__ __forceinline__ float c2_numerator(int dq, int c2) {
+  if (dq == 2) {
+    const __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c2 & 0xFF), __NV_E4M3);
+    return __half2float(__half(h));
+  }
+  return static_cast<float>(c2);
+}
+
 __device__ __forceinline__ float scale_value(int dq, float mean, ScaleRaw r, ScaleRecip& rec) {
   if (!dq) return r.a;
   if (r.a != rec.c1) {
@@ -66,7 +76,7 @@ __device__ __forceinline__ float scale_value(int dq, float mean, ScaleRaw r, Sca
     rec.rc = __frcp_rn(r.a);
     rec.fast = (r.a >= 0x1p-60f) && (r.a <= 0x1p60f);
   }
-  const float w = static_cast<float>(r.b);
+  const float w = c2_numerator(dq, r.b);
   float q;
   if (rec.fast) {
     const float y = __fmul_rn(w, rec.rc);

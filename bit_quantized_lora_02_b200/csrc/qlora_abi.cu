@@ -207,14 +207,6 @@ int qlora_linear_workspace_size(int64_t M, int64_t d, int64_t k, int32_t r, int3
   return ok();
 }
 
-// E4M3 second-level constants are supported by quantisation and the standalone
-// dequantisation only; the fused kernels decode Int8 constants.
-static int check_dq_mode_fused(const qlora_nf4_t* q, const char* what) {
-  if (q->double_quant == 2)
-    return fail(QLORA_ERR_UNSUPPORTED, "%s: E4M3 second-level constants (double_quant = 2) are not supported", what);
-  return QLORA_OK;
-}
-
 // The tensor-core kernels read the packed codes with TMA: 16-byte alignment.
 static int check_codes_tma(const qlora_nf4_t* q) {
   if (!aligned(q->codes, 16)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 16-byte aligned for the linear layer");
@@ -233,7 +225,6 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const u
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
-  if ((rc = check_dq_mode_fused(q, "qlora_linear_fwd"))) return rc;
   if ((rc = check_linear_shape(M, q->d, q->k, r))) return rc;
   if (M == 0) return ok();
   if ((rc = check_codes_tma(q))) return rc;
@@ -261,7 +252,6 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlo
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
-  if ((rc = check_dq_mode_fused(q, "qlora_linear_bwd"))) return rc;
   if ((rc = check_linear_shape(M, q->d, q->k, r))) return rc;
   if ((rc = check_ptr16(dA, "dA", true)) || (rc = check_ptr16(dB, "dB", true))) return rc;
   if (M > 0 && (rc = check_codes_tma(q))) return rc;
@@ -290,7 +280,6 @@ int qlora_lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
-  if ((rc = check_dq_mode_fused(q, "qlora_lora_merge"))) return rc;
   if ((rc = check_linear_shape(0, q->d, q->k, r))) return rc;
   if (!aligned(q->codes, 16)) return fail(QLORA_ERR_ALIGNMENT, "codes must be 16-byte aligned for the merge");
   if ((rc = check_ptr16(A, "A", true)) || (rc = check_ptr16(B, "B", true)) || (rc = check_ptr16(W_out, "W_out", true)))

@@ -560,7 +560,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
       R.rc = __frcp_rn(R.c1);
       R.fast = (R.c1 >= 0x1p-60f) && (R.c1 <= 0x1p60f);
     }
-    const float w = static_cast<float>(c2v);
+    const float w = c2_numerator(p.sc.dq, c2v);
     float q;
     if (R.fast) {
       const float y = __fmul_rn(w, R.rc);

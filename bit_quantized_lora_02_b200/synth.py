@@ -16,8 +16,9 @@ tensor_id])``):
   pattern, and handed out as ``uint16`` bit arrays (or fp32 copies of them).
 
 Tensor ids: W0=0, A=1, B=2, X=3, dY=4, outlier mask=5, outlier values=6.
-Projections of one layer set use ``seed = base_seed * 1000 + projection
-index`` so every weight matrix is distinct.
+Projections of one layer set use their index as the seed (``seed = p``), so
+every weight matrix is distinct; rank rho of a data-parallel run draws its
+tokens X and dY with ``seed = p + 1000 * rho``.
 """
 from __future__ import annotations
 

@@ -86,9 +86,8 @@ typedef struct {
   int64_t k;
   int32_t blocksize;     /* weights per NF4 block; only 64 is supported       */
   int32_t double_quant;  /* 0: fp32 absmax per block; 1: int8 c2 + fp32 c1;   *
-                          * 2: E4M3 c2 + fp32 c1 (nf4_quantize, nf4_dequantize *
-                          * and the sizes query only; the linear layer and the *
-                          * merge return QLORA_ERR_UNSUPPORTED)                 */
+                          * 2: E4M3 c2 + fp32 c1.  Every entry point accepts   *
+                          * all three modes.                                   */
   uint8_t *codes;
   float *absmax;
   int8_t *c2;
@@ -139,8 +138,11 @@ int nf4_quantize(const uint16_t *W0, const qlora_nf4_t *q, void *workspace, size
  *   - d * k above QLORA_NOALLOC_MAX_WEIGHTS returns QLORA_ERR_UNSUPPORTED;
  *     use nf4_quantize with a workspace for larger weights.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, a host-side lookup that allocates nothing; it is
+ *     not cached, so a context destroyed and recreated by the caller is
+ *     handled).  The first call on a device may load the library's device
+ *     code there; make that first call before any stream capture.
  *   - All calls share the one array, and each call clears the part that must
  *     start at zero.  Calls whose kernels may overlap on the GPU (for instance
  *     on two streams without ordering) race on it and give wrong results. */

@@ -38,10 +38,19 @@ def test_default_step_flops():
 def test_traffic_counts_only_under_matching_source_hash(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "traffic_fwd_gemm.txt").write_text("# comment = ignored\nbytes_per_launch = 1234\nsource_hash = abc\n")
+    (prof / "traffic_fwd_gemm_wl.txt").write_text("# comment = ignored\nbytes_per_launch = 1234\nsource_hash = abc\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
-    assert bench.read_traffic("fwd_gemm") == 1234.0
+    assert bench.read_traffic("fwd_gemm", "wl") == 1234.0
+    assert bench.read_traffic("fwd_gemm", "other") is None   # another workload has its own file
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "def")
-    assert bench.read_traffic("fwd_gemm") is None
-    assert bench.read_traffic("bwd_gemm") is None   # no file
+    assert bench.read_traffic("fwd_gemm", "wl") is None
+    assert bench.read_traffic("bwd_gemm", "wl") is None   # no file
+
+
+def test_65b_step_flops():
+    from bit_quantized_lora_02_b200 import synth
+    work = synth.WORKLOADS["llama65b_block_m8192"]
+    M, r = work["m"], work["r"]
+    total = sum(bench.flops_fwd(M, d, k, r) + bench.flops_bwd(M, d, k, r) for _, d, k in work["proj"])
+    assert abs(total / 1e12 - 27.017) < 5e-3

@@ -25,7 +25,7 @@ def _layer(M, d, k, r, seed=0, a_std=None, b_zero=False, outliers=False):
 
 
 def _oracle_what(W0_bits, dq=True):
-    q = O.quantize_tensor(W0_bits.reshape(-1), double_quant=dq)
+    q = O.quantize_tensor(W0_bits.reshape(-1), double_quant=bool(dq), dq_fp8=(dq == 2))
     d, k = W0_bits.shape
     return O.dequantize_tensor(q).reshape(d, k)
 
@@ -143,3 +143,12 @@ def test_projection_full_size_sampled():
     _, dA_ref, dB_ref = O.qlora_backward(L["dY"], L["X"], Wh, L["A"], L["B"], alpha, r)
     assert_close(host_f32(out["dA"]), dA_ref, "dA")
     assert_close(host_f32(out["dB"]), dB_ref, "dB")
+
+
+@pytest.mark.parametrize("M,d,k,r", [(200, 520, 704, 16), (4, 1024, 2048, 16), (64, 768, 1024, 32)])
+def test_e4m3_constants(M, d, k, r):
+    """E4M3 second-level constants through every fused path: the paired GEMMs
+    (M > 128), the few-token path (M <= 16) and the swapped forward."""
+    L = _layer(M, d, k, r, seed=40 + M)
+    out = _run(L, 16.0, dq=2)
+    _check(L, out, 16.0, dq=2)

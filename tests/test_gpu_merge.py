@@ -97,3 +97,14 @@ def test_merge_full_size_sampled_rows():
     qo = O.quantize_tensor(W0[rows].reshape(-1), double_quant=False)
     Wh = O.dequantize_tensor(qo).reshape(len(rows), k)
     _check_merge(got, Wh, A, B[rows], 16.0, r, "merge 4096x4096 sampled rows")
+
+
+def test_merge_e4m3_constants():
+    d, k, r = 136, 576, 16
+    L = synth.layer(4, d, k, r, seed=31)
+    B = synth.lora_b(d, r, seed=32, std=0.5)
+    q = Q.nf4_quantize(dev_bf16(L["W0"]), double_quant=2)
+    Wm = Q.qlora_lora_merge(q, dev_bf16(L["A"]), dev_bf16(B), 16.0)
+    torch.cuda.synchronize()
+    Wh = O.dequantize_tensor(O.quantize_tensor(L["W0"].reshape(-1), double_quant=True, dq_fp8=True)).reshape(d, k)
+    _check_merge(host_bits(Wm), Wh, L["A"], B, 16.0, r, "merge with E4M3 constants")
