@@ -173,6 +173,7 @@ class OracleSample:
         from oracle import qlora_oracle as O
         self.O = O
         self.M, self.r, self.alpha = work["m"], work["r"], work["alpha"]
+        self.p = work.get("dropout", 0.0)
         self.frac = frac
         self.Ms = max(1, int(self.M * frac))
         self.prepared = []
@@ -194,10 +195,15 @@ class OracleSample:
         O, r, alpha = self.O, self.r, self.alpha
         t0 = time.perf_counter()
         flops = 0.0
-        for rows, k, W0q, What, X, dY, A, B in self.prepared:
+        for pi, (rows, k, W0q, What, X, dY, A, B) in enumerate(self.prepared):
             O.dequantize_tensor(O.quantize_tensor(W0q.reshape(-1), True))
-            O.qlora_forward(X, What, A, B, alpha, r)
-            O.qlora_backward(dY, X, What, A, B, alpha, r)
+            if self.p:
+                keep = O.dropout_keep(self.Ms, k, self.p, 1234, pi)
+                O.qlora_forward_dropout(X, What, A, B, alpha, r, keep, self.p)
+                O.qlora_backward_dropout(dY, X, What, A, B, alpha, r, keep, self.p)
+            else:
+                O.qlora_forward(X, What, A, B, alpha, r)
+                O.qlora_backward(dY, X, What, A, B, alpha, r)
             flops += flops_fwd(self.Ms, rows, k, r) + flops_bwd(self.Ms, rows, k, r)
         return time.perf_counter() - t0, flops
 
@@ -231,6 +237,8 @@ def run_ours(args, work, wl_name):
 
     M, r, alpha = work["m"], work["r"], work["alpha"]
     projs = work["proj"]
+    drop_p = work.get("dropout", 0.0)
+    step_no = [0]          # the dropout generator's offset: a new mask every step (and projection)
     # adapter gradients of every projection in one flat fp32 bucket (one all-reduce per step)
     bucket = GradBucket([s_ for _, d, k in projs for s_ in ((r, k), (d, r))], dev)
     bufs = []
@@ -252,7 +260,8 @@ def run_ours(args, work, wl_name):
         b["dX"] = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
         b["dA"] = bucket.views[2 * pi]
         b["dB"] = bucket.views[2 * pi + 1]
-        nws = max(Q.qlora_linear_workspace_size(M, d, k, r, False), Q.qlora_linear_workspace_size(M, d, k, r, True))
+        wsz = Q.qlora_linear_dropout_workspace_size if drop_p else Q.qlora_linear_workspace_size
+        nws = max(wsz(M, d, k, r, False), wsz(M, d, k, r, True))
         b["ws"] = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         for key in ("Y", "dX", "dA", "dB"):
             b["h_" + key] = torch.empty(b[key].shape, dtype=b[key].dtype, pin_memory=True)
@@ -262,12 +271,14 @@ def run_ours(args, work, wl_name):
     stream = torch.cuda.current_stream()
 
     def step():
-        for b in bufs:
+        for pi, b in enumerate(bufs):
+            drop = (drop_p, 1234 + rank, step_no[0] * len(bufs) + pi) if drop_p else None
             Q.nf4_quantize(b["W0"], True, out=b["q"], workspace=b["qws"], stream=stream)
             Q.qlora_linear_fwd(b["X"], b["q"], b["A"], b["B"], alpha, Y=b["Y"], T_save=b["T"], workspace=b["ws"],
-                               stream=stream)
+                               stream=stream, dropout=drop)
             Q.qlora_linear_bwd(b["dY"], b["X"], b["q"], b["A"], b["B"], alpha, T_save=b["T"], dX=b["dX"],
-                               dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream)
+                               dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream, dropout=drop)
+        step_no[0] += 1
         if world > 1:
             bucket.allreduce()
 
@@ -376,7 +387,8 @@ def run_ours(args, work, wl_name):
         "dtype": "bf16", "data": "synthetic (seeded numpy: W0~N(0,0.02), A~N(0,1/r), B~N(0,0.01), X,dY~N(0,1))",
         "config": {"workload": wl_name, "tokens_per_rank": M, "rank": r, "alpha": alpha,
                    "projections": [f"{n}:{d}x{k}" for n, d, k in projs], "nf4_blocksize": 64,
-                   "double_quant": True, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "double_quant": True, "lora_dropout": drop_p,
+                   "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "working set per step larger than L2 (no explicit flush)"},
         "breakdown_ms_per_step": {c: round(v / args.steps, 4) for c, v in kms.items()},
         "profiled_ms_per_step": round(ms_profiled / args.steps, 4),
@@ -575,6 +587,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="llama65b_block_m8192",
                     choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512",
+                             "llama7b_proj_set_m4096_dropout", "llama65b_block_m8192_dropout",
                              "decode_28672x8192", "quant_sweep", "merge_sweep"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

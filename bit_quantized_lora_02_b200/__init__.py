@@ -28,7 +28,9 @@ _STATUS = {0: "QLORA_OK", -1: "QLORA_ERR_INVALID_ARG", -2: "QLORA_ERR_UNSUPPORTE
 EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_lora_merge",
            "qlora_rank_pad", "qlora_linear_workspace_size",
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error",
-           "qlora_profile_enable", "qlora_profile_read")
+           "qlora_profile_enable", "qlora_profile_read",
+           "qlora_dropout_mask", "qlora_linear_dropout_workspace_size", "qlora_linear_fwd_dropout",
+           "qlora_linear_bwd_dropout", "qlora_selftest_wait_timeout")
 
 KERNEL_CLASSES = ("quant", "dq_const", "dequant", "fwd_gemm", "bwd_gemm", "lora_gemm", "aux")
 
@@ -44,6 +46,12 @@ class QloraNF4(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int64), ("k", ctypes.c_int64), ("blocksize", ctypes.c_int32),
                 ("double_quant", ctypes.c_int32), ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
                 ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mean", ctypes.c_void_p)]
+
+
+class QloraDropout(ctypes.Structure):
+    """Mirror of ``qlora_dropout_t``: adapter dropout probability p and the
+    generator's (seed, offset)."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
 
 
 _lib = None
@@ -72,13 +80,22 @@ def lib() -> ctypes.CDLL:
                                    vp, vp, vp, c_sz, vp]
     L.qlora_nf4_codebook.argtypes = [ctypes.POINTER(ctypes.c_float)]
     L.qlora_device_status.argtypes = [vp, ctypes.POINTER(c_i32)]
+    L.qlora_dropout_mask.argtypes = [c_i64, c_i64, ctypes.POINTER(QloraDropout), vp, vp]
+    L.qlora_linear_dropout_workspace_size.argtypes = [c_i64, c_i64, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz)]
+    L.qlora_linear_fwd_dropout.argtypes = [vp, c_i64, ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float,
+                                           ctypes.POINTER(QloraDropout), vp, vp, vp, c_sz, vp]
+    L.qlora_linear_bwd_dropout.argtypes = [vp, vp, c_i64, ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float,
+                                           ctypes.POINTER(QloraDropout), vp, vp, vp, vp, vp, c_sz, vp]
+    L.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, vp]
     L.qlora_last_error.restype = ctypes.c_char_p
     L.qlora_profile_enable.argtypes = [c_i32]
     L.qlora_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
     for name in ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequantize", "qlora_lora_merge",
                  "qlora_linear_workspace_size",
                  "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
-                 "qlora_profile_enable", "qlora_profile_read"):
+                 "qlora_profile_enable", "qlora_profile_read", "qlora_dropout_mask",
+                 "qlora_linear_dropout_workspace_size", "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout",
+                 "qlora_selftest_wait_timeout"):
         getattr(L, name).restype = c_i32
     _lib = L
     return L
@@ -279,10 +296,54 @@ def qlora_linear_workspace_size(M: int, d: int, k: int, r: int, backward: bool) 
     return n.value
 
 
+def _dropout_struct(dropout) -> Optional[QloraDropout]:
+    """(p, seed, offset) -> qlora_dropout_t, or None for no dropout."""
+    if dropout is None:
+        return None
+    p, seed, offset = dropout
+    if not (0.0 <= float(p) < 1.0):
+        raise ValueError(f"dropout probability {p} outside [0, 1)")
+    return QloraDropout(float(p), int(seed) & (2 ** 64 - 1), int(offset) & (2 ** 64 - 1))
+
+
+def qlora_linear_dropout_workspace_size(M: int, d: int, k: int, r: int, backward: bool) -> int:
+    n = ctypes.c_size_t()
+    _check(lib().qlora_linear_dropout_workspace_size(M, d, k, r, int(backward), ctypes.byref(n)))
+    return n.value
+
+
+def qlora_dropout_mask(M: int, k: int, p: float, seed: int, offset: int = 0, out: Optional[torch.Tensor] = None,
+                       device=None, stream=None) -> torch.Tensor:
+    """Keep bitmask of an M x k activation as int32 words (bit b of word w is
+    flat element 32 w + b; 1 = kept)."""
+    nw = (M * k + 31) // 32
+    if out is None:
+        device = device or torch.device("cuda", torch.cuda.current_device())
+        out = torch.empty(max(nw, 1), dtype=torch.int32, device=device)
+    if out.dtype != torch.int32 or out.numel() < nw or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous int32 tensor of at least {nw} words")
+    st = _dropout_struct((p, seed, offset))
+    _check(lib().qlora_dropout_mask(M, k, ctypes.byref(st), out.data_ptr() if nw else None, _stream(stream)))
+    return out
+
+
+def qlora_linear_fwd_dropout(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                             dropout, **kw):
+    """qlora_linear_fwd with adapter dropout; dropout = (p, seed, offset)."""
+    return qlora_linear_fwd(X, q, A, B, alpha, dropout=dropout, **kw)
+
+
+def qlora_linear_bwd_dropout(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor,
+                             alpha: float, dropout, **kw):
+    """qlora_linear_bwd for the dropout forward with the same (p, seed, offset)."""
+    return qlora_linear_bwd(dY, X, q, A, B, alpha, dropout=dropout, **kw)
+
+
 def qlora_linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
                      Y: Optional[torch.Tensor] = None, T_save: Optional[torch.Tensor] = None,
-                     workspace: Optional[torch.Tensor] = None, stream=None, save_T: bool = True):
-    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns (Y, T_save)."""
+                     workspace: Optional[torch.Tensor] = None, stream=None, save_T: bool = True, dropout=None):
+    """Y = X W^T + (alpha/r) (X A^T) B^T.  Returns (Y, T_save).  With
+    dropout = (p, seed, offset) the adapter sees drop(X) instead of X."""
     M, k = X.shape
     r = A.shape[0]
     dev = X.device
@@ -295,21 +356,30 @@ def qlora_linear_fwd(X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Te
     _expect(B, "B", (q.d, r), torch.bfloat16)
     _expect(Y, "Y", (M, q.d), torch.bfloat16)
     _expect(T_save, "T_save", (M, qlora_rank_pad(r)), torch.bfloat16, required=False)
+    drop = _dropout_struct(dropout)
     if workspace is None:
-        n = qlora_linear_workspace_size(M, q.d, q.k, r, False)
+        n = (qlora_linear_dropout_workspace_size(M, q.d, q.k, r, False) if drop is not None
+             else qlora_linear_workspace_size(M, q.d, q.k, r, False))
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
     _same_device(dev, A=A, B=B, Y=Y, T_save=T_save, workspace=workspace)
     st = q.struct(dev)
-    _check(lib().qlora_linear_fwd(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha),
-                                  Y.data_ptr(), _ptr(T_save), _ptr(workspace), _nbytes(workspace), _stream(stream)))
+    if drop is None:
+        _check(lib().qlora_linear_fwd(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha),
+                                      Y.data_ptr(), _ptr(T_save), _ptr(workspace), _nbytes(workspace),
+                                      _stream(stream)))
+    else:
+        _check(lib().qlora_linear_fwd_dropout(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
+                                              float(alpha), ctypes.byref(drop), Y.data_ptr(), _ptr(T_save),
+                                              _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return Y, T_save
 
 
 def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.Tensor, B: torch.Tensor,
                      alpha: float, T_save: Optional[torch.Tensor] = None, dX: Optional[torch.Tensor] = None,
                      dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
-                     workspace: Optional[torch.Tensor] = None, stream=None, need_dX: bool = True):
-    """Gradients for the adapters and the input; returns (dX, dA, dB)."""
+                     workspace: Optional[torch.Tensor] = None, stream=None, need_dX: bool = True, dropout=None):
+    """Gradients for the adapters and the input; returns (dX, dA, dB).  With
+    dropout = (p, seed, offset), the backward of the dropout forward."""
     M = dY.shape[0]
     r = A.shape[0]
     dev = dY.device
@@ -327,14 +397,22 @@ def qlora_linear_bwd(dY: torch.Tensor, X: torch.Tensor, q: NF4Weight, A: torch.T
     _expect(dX, "dX", (M, q.k), torch.bfloat16, required=False)
     _expect(dA, "dA", (r, q.k), torch.float32)
     _expect(dB, "dB", (q.d, r), torch.float32)
+    drop = _dropout_struct(dropout)
     if workspace is None:
-        n = qlora_linear_workspace_size(M, q.d, q.k, r, True)
+        n = (qlora_linear_dropout_workspace_size(M, q.d, q.k, r, True) if drop is not None
+             else qlora_linear_workspace_size(M, q.d, q.k, r, True))
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=dev) if n else None
     _same_device(dev, X=X, A=A, B=B, T_save=T_save, dX=dX, dA=dA, dB=dB, workspace=workspace)
     st = q.struct(dev)
-    _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
-                                  float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
-                                  _ptr(workspace), _nbytes(workspace), _stream(stream)))
+    if drop is None:
+        _check(lib().qlora_linear_bwd(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
+                                      float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
+                                      _ptr(workspace), _nbytes(workspace), _stream(stream)))
+    else:
+        _check(lib().qlora_linear_bwd_dropout(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(),
+                                              r, float(alpha), ctypes.byref(drop), _ptr(T_save), _ptr(dX),
+                                              dA.data_ptr(), dB.data_ptr(), _ptr(workspace), _nbytes(workspace),
+                                              _stream(stream)))
     return dX, dA, dB
 
 
@@ -351,6 +429,15 @@ def qlora_device_status(stream=None) -> int:
     if rc not in (QLORA_OK, -6):
         _check(rc)
     return s.value
+
+
+def qlora_selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
+    """Run the bounded-wait self-test (a wait nothing ends, given up after
+    limit_us); returns the kernel's result word (2: gave up and released its
+    TMEM).  The status word then holds code 7 until qlora_device_status()."""
+    res = torch.zeros(1, dtype=torch.int32, device=torch.device("cuda", torch.cuda.current_device()))
+    _check(lib().qlora_selftest_wait_timeout(int(limit_us), res.data_ptr(), _stream(stream)))
+    return int(res.item())
 
 
 def qlora_profile_enable(on: bool = True) -> None:

@@ -18,7 +18,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libqlora.so")
-SOURCES = ["qlora_abi.cu", "nf4_quant.cu", "qlora_gemm.cu", "qlora_fewtok.cu", "qlora_merge.cu", "qlora_prof.cu"]
+SOURCES = ["qlora_abi.cu", "nf4_quant.cu", "qlora_gemm.cu", "qlora_fewtok.cu", "qlora_merge.cu", "qlora_dropout.cu",
+           "qlora_prof.cu"]
 HEADERS = ["qlora_device.cuh", "qlora_internal.h", "nf4_table.h", "nf4_scale.cuh"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

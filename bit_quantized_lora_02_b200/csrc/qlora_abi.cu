@@ -13,6 +13,58 @@ namespace qlora {
 
 __device__ int g_status = 0;
 
+// Self-test of the failure path every kernel's waits share: one CTA takes 32
+// TMEM columns, then waits on an mbarrier that nothing ever arrives at with
+// the same bounded loop as mbar_wait but a caller-chosen limit.  When the
+// limit runs out it records DEV_WAIT_TIMEOUT_SELFTEST in the status word,
+// releases its TMEM like any kernel winding down after a failed wait, and
+// writes 2 to *result after the release (1 would mean the barrier completed,
+// which cannot happen).  No fault, trap or endless loop is involved.
+__global__ void k_selftest_wait_timeout(uint64_t limit_ns, int* result) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t slot;
+  __shared__ volatile int abort_flag;
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&slot, 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = slot;
+  int outcome = 0;
+  if (threadIdx.x == 0) {
+    const uint32_t a = smem_u32(&bar);
+    const uint64_t t0 = globaltimer_ns();
+    outcome = 2;
+    for (uint32_t it = 1;; ++it) {
+      if (mbar_try_wait(a, 0)) {
+        outcome = 1;
+        break;
+      }
+      if ((it & 63u) == 0 && globaltimer_ns() - t0 > limit_ns) {
+        report(DEV_WAIT_TIMEOUT_SELFTEST);
+        abort_flag = 1;
+        break;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) *result = outcome;
+}
+
 cudaError_t read_and_clear_status(int* out) {
   int zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(out, g_status, sizeof(int));
@@ -219,9 +271,31 @@ static int check_ptr16(const void* p, const char* name, bool required) {
   return ok();
 }
 
-int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
-                     int32_t r, float alpha, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
-                     qlora_stream_t stream) {
+}  // extern "C"
+
+// Adapter dropout arguments: p finite in [0, 1).  p == 0 (or no struct) is the
+// plain layer, bit for bit.
+static int check_dropout(const qlora_dropout_t* drop, DropoutArgs* out, bool* on) {
+  *on = false;
+  if (!drop) return QLORA_OK;
+  const float p = drop->p;
+  if (!(p >= 0.0f && p < 1.0f)) return fail(QLORA_ERR_INVALID_ARG, "dropout probability must lie in [0, 1)");
+  if (p == 0.0f) return QLORA_OK;
+  const float keep = 1.0f - p;   // RN32(1 - p)
+  out->p = p;
+  out->thr = dropout_threshold(p);
+  out->dscale = 1.0f / keep;     // RN32(1 / RN32(1 - p))
+  out->seed = drop->seed;
+  out->offset = drop->offset;
+  *on = true;
+  return QLORA_OK;
+}
+
+static int linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
+                      int32_t r, float alpha, const qlora_dropout_t* drop, uint16_t* Y, uint16_t* T_save,
+                      void* workspace, size_t workspace_bytes, qlora_stream_t stream, const char* name) {
+  DropoutArgs dargs{};
+  bool dropping = false;
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
@@ -231,7 +305,8 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const u
   if ((rc = check_ptr16(X, "X", true)) || (rc = check_ptr16(A, "A", true)) || (rc = check_ptr16(B, "B", true)) ||
       (rc = check_ptr16(Y, "Y", true)) || (rc = check_ptr16(T_save, "T_save", false)))
     return rc;
-  const size_t need = fwd_workspace_bytes(M, q->d, q->k, r);
+  if ((rc = check_dropout(drop, &dargs, &dropping))) return rc;
+  const size_t need = dropping ? dropout_workspace_bytes(M, q->d, q->k, r, false) : fwd_workspace_bytes(M, q->d, q->k, r);
   if (need && (!workspace || workspace_bytes < need))
     return fail(QLORA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : 0);
   if (workspace && (rc = check_ptr16(workspace, "workspace", false))) return rc;
@@ -240,15 +315,19 @@ int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const u
   a.X = X; a.M = M; a.d = q->d; a.k = q->k; a.q = q; a.A = A; a.B = B; a.r = r; a.rp = qlora_rank_pad(r);
   a.s = alpha / static_cast<float>(r);
   a.Y = Y; a.T = T_save; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  a.drop = dropping ? &dargs : nullptr;
   const char* why = "";
   rc = launch_linear_fwd(a, static_cast<cudaStream_t>(stream), &why);
-  if (rc) return fail(rc, "qlora_linear_fwd: %s", why);
+  if (rc) return fail(rc, "%s: %s", name, why);
   return ok();
 }
 
-int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A,
-                     const uint16_t* B, int32_t r, float alpha, const uint16_t* T_save, uint16_t* dX, float* dA,
-                     float* dB, void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+static int linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A,
+                      const uint16_t* B, int32_t r, float alpha, const qlora_dropout_t* drop, const uint16_t* T_save,
+                      uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                      qlora_stream_t stream, const char* name) {
+  DropoutArgs dargs{};
+  bool dropping = false;
   int64_t N = 0;
   int rc = check_nf4(q, &N);
   if (rc) return rc;
@@ -259,7 +338,8 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlo
       (rc = check_ptr16(B, "B", true)) || (rc = check_ptr16(dX, "dX", false)) ||
       (rc = check_ptr16(T_save, "T_save", false)))
     return rc;
-  const size_t need = bwd_workspace_bytes(M, q->d, q->k, r);
+  if ((rc = check_dropout(drop, &dargs, &dropping))) return rc;
+  const size_t need = dropping ? dropout_workspace_bytes(M, q->d, q->k, r, true) : bwd_workspace_bytes(M, q->d, q->k, r);
   if (need && (!workspace || workspace_bytes < need))
     return fail(QLORA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : 0);
   if (workspace && (rc = check_ptr16(workspace, "workspace", false))) return rc;
@@ -269,10 +349,73 @@ int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlo
   a.rp = qlora_rank_pad(r);
   a.s = alpha / static_cast<float>(r);
   a.Tin = T_save; a.dX = dX; a.dA = dA; a.dB = dB; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  a.drop = dropping ? &dargs : nullptr;
   const char* why = "";
   rc = launch_linear_bwd(a, static_cast<cudaStream_t>(stream), &why);
-  if (rc) return fail(rc, "qlora_linear_bwd: %s", why);
+  if (rc) return fail(rc, "%s: %s", name, why);
   return ok();
+}
+
+extern "C" {
+
+int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
+                     int32_t r, float alpha, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,
+                     qlora_stream_t stream) {
+  return linear_fwd(X, M, q, A, B, r, alpha, nullptr, Y, T_save, workspace, workspace_bytes, stream,
+                    "qlora_linear_fwd");
+}
+
+int qlora_linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A,
+                     const uint16_t* B, int32_t r, float alpha, const uint16_t* T_save, uint16_t* dX, float* dA,
+                     float* dB, void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  return linear_bwd(dY, X, M, q, A, B, r, alpha, nullptr, T_save, dX, dA, dB, workspace, workspace_bytes, stream,
+                    "qlora_linear_bwd");
+}
+
+int qlora_linear_fwd_dropout(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A,
+                             const uint16_t* B, int32_t r, float alpha, const qlora_dropout_t* drop, uint16_t* Y,
+                             uint16_t* T_save, void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  return linear_fwd(X, M, q, A, B, r, alpha, drop, Y, T_save, workspace, workspace_bytes, stream,
+                    "qlora_linear_fwd_dropout");
+}
+
+int qlora_linear_bwd_dropout(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_t* q,
+                             const uint16_t* A, const uint16_t* B, int32_t r, float alpha,
+                             const qlora_dropout_t* drop, const uint16_t* T_save, uint16_t* dX, float* dA, float* dB,
+                             void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  return linear_bwd(dY, X, M, q, A, B, r, alpha, drop, T_save, dX, dA, dB, workspace, workspace_bytes, stream,
+                    "qlora_linear_bwd_dropout");
+}
+
+int qlora_linear_dropout_workspace_size(int64_t M, int64_t d, int64_t k, int32_t r, int32_t backward,
+                                        size_t* bytes) {
+  if (!bytes) return fail(QLORA_ERR_INVALID_ARG, "bytes is NULL");
+  int rc = check_linear_shape(M, d, k, r);
+  if (rc) return rc;
+  *bytes = dropout_workspace_bytes(M, d, k, r, backward != 0);
+  return ok();
+}
+
+int qlora_dropout_mask(int64_t M, int64_t k, const qlora_dropout_t* drop, uint32_t* keep_bits,
+                       qlora_stream_t stream) {
+  if (!drop) return fail(QLORA_ERR_INVALID_ARG, "dropout descriptor is NULL");
+  int64_t n = 0;
+  if (!elem_count(M, k, &n)) return fail(QLORA_ERR_INVALID_ARG, "bad shape M=%lld k=%lld", (long long)M, (long long)k);
+  const float p = drop->p;
+  if (!(p >= 0.0f && p < 1.0f)) return fail(QLORA_ERR_INVALID_ARG, "dropout probability must lie in [0, 1)");
+  if (n == 0) return ok();
+  if (!keep_bits) return fail(QLORA_ERR_INVALID_ARG, "keep_bits is NULL");
+  if (!aligned(keep_bits, 4)) return fail(QLORA_ERR_ALIGNMENT, "keep_bits must be 4-byte aligned");
+  int rc = bind_device(keep_bits);
+  if (rc) return rc;
+  DropoutArgs dargs{};
+  dargs.p = p;
+  dargs.thr = dropout_threshold(p);
+  dargs.dscale = 1.0f / (1.0f - p);
+  dargs.seed = drop->seed;
+  dargs.offset = drop->offset;
+  return check_cuda(launch_dropout_bits(n, dargs, keep_bits, static_cast<cudaStream_t>(stream)),
+                    "qlora_dropout_mask launch");
 }
 
 int qlora_lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int32_t r, float alpha,
@@ -306,6 +449,16 @@ int qlora_device_status(qlora_stream_t stream, int32_t* status) {
   *status = s;
   if (s) return fail(QLORA_ERR_DEVICE, "a kernel reported failed check %d", s);
   return ok();
+}
+
+int qlora_selftest_wait_timeout(uint32_t limit_us, int32_t* result, qlora_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(QLORA_ERR_INVALID_ARG, "limit_us must lie in 1..1000000");
+  if (!result) return fail(QLORA_ERR_INVALID_ARG, "result is NULL");
+  if (!aligned(result, 4)) return fail(QLORA_ERR_ALIGNMENT, "result must be 4-byte aligned");
+  int rc = bind_device(result);
+  if (rc) return rc;
+  k_selftest_wait_timeout<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(1000ull * limit_us, result);
+  return check_cuda(cudaGetLastError(), "qlora_selftest_wait_timeout launch");
 }
 
 const char* qlora_last_error(void) { return t_err.c_str(); }

@@ -25,6 +25,7 @@ enum DeviceError : int {
   DEV_WAIT_TIMEOUT_EPILOGUE = 4,
   DEV_WAIT_TIMEOUT_DRAIN = 5,
   DEV_SMEM_LAYOUT = 6,           // the shared-memory window could not hold a kernel's layout
+  DEV_WAIT_TIMEOUT_SELFTEST = 7, // the self-test's wait on a barrier nothing arrives at ran out
 };
 
 extern __device__ int g_status;

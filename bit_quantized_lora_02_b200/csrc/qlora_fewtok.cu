@@ -230,10 +230,18 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p) { return *reinter
 // every 8th 16-column step of it, the warps' fragments are added in warp order
 // and CTA 0 adds the eight CTAs' sums in order through distributed shared
 // memory.  The last cluster also writes the zero columns r .. rp - 1.
+// With adapter dropout `keep` is the keep bitmask of X (bit b of word w <->
+// flat element 32 w + b) and dropped elements enter the products as zeros;
+// `s` then includes the 1 / (1 - p) of the kept ones.
 // ============================================================================
+// 32-bit lane mask of a bf16 pair from its two keep bits (bit 0: low element)
+__device__ __forceinline__ uint32_t pair_keep_mask(uint32_t two) {
+  return ((two & 1u) ? 0x0000FFFFu : 0u) | ((two & 2u) ? 0xFFFF0000u : 0u);
+}
+
 __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
     k_lora_down_fewtok(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int M, int64_t k, int r,
-                       int rp, float s, uint16_t* __restrict__ T) {
+                       int rp, float s, uint16_t* __restrict__ T, const uint32_t* __restrict__ keep) {
   griddep_launch_dependents();
   __shared__ float4 red[8][32];
   const uint32_t q = cluster_rank();
@@ -251,9 +259,25 @@ __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
 #pragma unroll 4
     for (int64_t st = s0 + warp; st < s1; st += 8) {
       const int64_t k0 = 16 * st;
-      const uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
-      const uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
+      uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
+      uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
       const uint32_t b0 = jv ? ld_pair(ar + k0) : 0u, b1 = jv ? ld_pair(ar + k0 + 8) : 0u;
+      if (keep) {
+        // keep bits of columns k0 .. k0 + 15 of rows g and g + 8 (k0 % 16 == 0,
+        // k % 64 == 0: the 16 bits sit in one word at bit 0 or 16)
+        if (ta) {
+          const int64_t e = static_cast<int64_t>(g) * k + k0;
+          const uint32_t w = __ldg(keep + (e >> 5)) >> (e & 31);
+          a0 &= pair_keep_mask(w >> (2 * c));
+          a2 &= pair_keep_mask(w >> (8 + 2 * c));
+        }
+        if (tb) {
+          const int64_t e = static_cast<int64_t>(g + 8) * k + k0;
+          const uint32_t w = __ldg(keep + (e >> 5)) >> (e & 31);
+          a1 &= pair_keep_mask(w >> (2 * c));
+          a3 &= pair_keep_mask(w >> (8 + 2 * c));
+        }
+      }
       mma16816(acc, a0, a1, a2, a3, b0, b1);
     }
   }
@@ -811,7 +835,7 @@ size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k) {
 
 template <int NTOK>
 static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm, uint16_t* T, float* part,
-                     cudaStream_t st, const char** why) {
+                     cudaStream_t st, const char** why, const uint32_t* keep) {
   CUtensorMap tx, tc2;
   if (!map_x(&tx, a.X, a.M, a.k, NTOK)) {
     *why = "tensor map encoding failed (few-token X)";
@@ -824,8 +848,9 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   if (!c2_tma) tc2 = tx;   // unused
   {
     ProfScope ps_(QLORA_KC_LORA_GEMM, st);
+    const float s_down = (keep && a.drop) ? a.s * a.drop->dscale : a.s;
     k_lora_down_fewtok<<<static_cast<unsigned>(kFtCluster * ceil_div(a.r, 8)), 256, 0, st>>>(
-        a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, a.s, T);
+        a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, s_down, T, keep);
   }
   if (cudaGetLastError() != cudaSuccess) {
     *why = "few-token down-projection launch";
@@ -889,12 +914,12 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
 }
 
 int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensorMap* tm_codes, cudaStream_t st,
-                      const char** why) {
+                      const char** why, const uint32_t* keep) {
   const FtPlan f = ft_plan(a.M, a.d, a.k);
   char* w = static_cast<char*>(ws);
   float* part = reinterpret_cast<float*>(w);
-  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, st, why)
-                     : ft_launch<16>(a, f, *tm_codes, T, part, st, why);
+  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, st, why, keep)
+                     : ft_launch<16>(a, f, *tm_codes, T, part, st, why, keep);
 }
 
 }  // namespace qlora

@@ -912,10 +912,38 @@ struct ThinParams {
   int32_t mode;          // ThinOut
   int32_t r;
   int64_t ld;            // THIN_DA: row stride of dA (= k)
-  float scale;
+  float scale;           // applied to every output (1 for a plain dA / dB)
   uint16_t* out16;
   float* outf;
+  // Adapter dropout on the A operand X (nullptr: none): keep bitmask of the
+  // M x k activations (bit b of word w <-> flat element 32 w + b).  Dropped
+  // elements are zeroed in shared memory before the tensor core reads them.
+  const uint32_t* keep;
+  int64_t keep_rows;     // M
+  int64_t keep_ld;       // k
 };
+
+// Zero the dropped elements of one 128-byte row (64 bf16) of a tile stored
+// with the 128-byte swizzle; bit e of `bits` keeps element e of the row.  A
+// mask byte becomes four 32-bit lane masks without a table: multiplying its
+// low (high) nibble by 2^7 + 2^14 + 2^21 + 2^28 moves bit i to bit 8 i + 7,
+// the sign bit of byte i (the partial products never overlap), and a byte
+// permute with sign replication widens each sign bit to 16 bits.
+__device__ __forceinline__ void mask_row_sw128(uint32_t tile, uint32_t r, uint64_t bits) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t b = static_cast<uint32_t>(bits >> (8 * c)) & 0xFFu;
+    if (b == 0xFFu) continue;
+    const uint32_t lo = (b & 0xFu) * 0x10204080u, hi = (b >> 4) * 0x10204080u;
+    const uint32_t addr = tile + sw128_offset(r, static_cast<uint32_t>(c));
+    uint4 v = lds128(addr);
+    v.x &= prmt(lo, 0u, 0x9988u);
+    v.y &= prmt(lo, 0u, 0xBBAAu);
+    v.z &= prmt(hi, 0u, 0x9988u);
+    v.w &= prmt(hi, 0u, 0xBBAAu);
+    sts128(addr, v);
+  }
+}
 
 struct ThinCfg {
   static constexpr int kStages = 4;
@@ -942,6 +970,7 @@ __global__ void __launch_bounds__(128, 2)
   uint64_t* tmem_full = bars + 2 * S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 2);
+  uint64_t* masked_bar = bars + 2 * S + 3;   // dropout: the stage's X tile has been masked
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -958,6 +987,7 @@ __global__ void __launch_bounds__(128, 2)
     for (int i = 0; i < S; ++i) {
       mbar_init(&full_bar[i], 1);
       mbar_init(&empty_bar[i], 1);
+      mbar_init(&masked_bar[i], 2);   // one arrival per masking warp
     }
     mbar_init(tmem_full, 1);
     *abort_flag = 0;
@@ -1010,10 +1040,11 @@ __global__ void __launch_bounds__(128, 2)
     }
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = make_idesc_bf16(128, static_cast<uint32_t>(rp), kAMN, kBMN);
+    uint64_t* ready = p.keep ? masked_bar : full_bar;
     for (int l = 0; l < n_local; ++l) {
       const int st = l % S;
       const uint32_t ph = (l / S) & 1;
-      if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
+      if (!mbar_wait(&ready[st], ph, abort_flag, p.keep ? DEV_WAIT_TIMEOUT_DEQUANT : DEV_WAIT_TIMEOUT_TMA)) break;
       tc_fence_after();
       const uint32_t aa = smem_u32(a_tile(st));
       const uint32_t bb = smem_u32(b_tile(st));
@@ -1028,6 +1059,51 @@ __global__ void __launch_bounds__(128, 2)
       umma_commit(&empty_bar[st]);
     }
     umma_commit(tmem_full);
+  } else if (warp >= 2 && p.keep) {
+    // adapter dropout: warps 2 and 3 zero the dropped activations of each
+    // stage's X tile before the MMA thread may read it.  The mask bits of a
+    // stage are fetched before its TMA wait, so their latency overlaps it.
+    const int t = static_cast<int>(threadIdx.x) - 64;   // 0..63
+    for (int l = 0; l < n_local; ++l) {
+      const int st = l % S;
+      const uint32_t ph = (l / S) & 1;
+      const int i = s_begin + l;
+      uint64_t bits[2] = {~0ull, ~0ull};
+      bool live[2] = {false, false};
+      const unsigned long long* kb = reinterpret_cast<const unsigned long long*>(p.keep);
+      if (!kAMN) {
+        // 128 token rows x 64 features (columns 64 i ..): rows t and t + 64
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t m = row0 + t + 64 * h;
+          live[h] = m < p.keep_rows;
+          if (live[h]) bits[h] = __ldg(kb + ((m * p.keep_ld + 64ll * i) >> 6));
+        }
+      } else {
+        // two halves of 64 token rows (64 i + t) x 64 features (row0 + 64 h ..)
+        const int64_t m = 64ll * i + t;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int64_t f = row0 + 64 * h;
+          live[h] = m < p.keep_rows && f < p.keep_ld;
+          if (live[h]) bits[h] = __ldg(kb + ((m * p.keep_ld + f) >> 6));
+        }
+      }
+      const bool okw = mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
+      if (!__all_sync(0xffffffffu, okw)) break;
+      const uint32_t at = smem_u32(a_tile(st));
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!live[h]) continue;   // rows past M or columns past k were filled with zeros by the copy
+        if (!kAMN)
+          mask_row_sw128(at, static_cast<uint32_t>(t + 64 * h), bits[h]);
+        else
+          mask_row_sw128(at + 8192u * h, static_cast<uint32_t>(t), bits[h]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&masked_bar[st]);
+    }
   }
   __syncwarp();
 
@@ -1098,7 +1174,7 @@ __global__ void __launch_bounds__(128, 2)
         o.y = pack_bf16x2(acc.z * p.scale, acc.w * p.scale);
         *reinterpret_cast<uint2*>(p.out16 + row * rp + j0) = o;
       } else {
-        const float e[4] = {acc.x, acc.y, acc.z, acc.w};
+        const float e[4] = {acc.x * p.scale, acc.y * p.scale, acc.z * p.scale, acc.w * p.scale};
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           if (j0 + u < p.r) {
@@ -1293,6 +1369,12 @@ size_t fwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
 size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r) {
   return make_plan(M, d, k, r, true, true).total;
 }
+size_t dropout_mask_offset(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd) {
+  return align_up(bwd ? bwd_workspace_bytes(M, d, k, r) : fwd_workspace_bytes(M, d, k, r), 256);
+}
+size_t dropout_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd) {
+  return dropout_mask_offset(M, d, k, r, bwd) + align_up(static_cast<size_t>((M * k + 31) / 32) * 4, 256);
+}
 
 static int grid1d(int64_t work, int per_block) {
   int64_t g = ceil_div(work, per_block);
@@ -1345,7 +1427,8 @@ static int launch_thin(const CUtensorMap& ta, const CUtensorMap& tb, ThinParams 
 // b_mn = true : bmat is (K x brows) row-major, read MN-major (B of the layer,
 //               K = d, N = r), which needs brows * 2 bytes to be a multiple of 16.
 static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uint16_t* bmat, int64_t brows,
-                            bool b_mn, int rp, float s, int splits, uint16_t* out, cudaStream_t st, const char** why) {
+                            bool b_mn, int rp, float s, int splits, uint16_t* out, cudaStream_t st, const char** why,
+                            const uint32_t* keep = nullptr) {
   CUtensorMap ta, tb;
   const bool okb = b_mn ? map_bf16(&tb, bmat, brows, K, 64, 64) : map_bf16(&tb, bmat, K, brows, 64, rp);
   if (!map_bf16(&ta, act, K, M, 64, 128) || !okb) {
@@ -1359,6 +1442,9 @@ static int run_lowrank_down(const uint16_t* act, int64_t M, int64_t K, const uin
   tp.mode = THIN_BF16;
   tp.scale = s;
   tp.out16 = out;
+  tp.keep = keep;
+  tp.keep_rows = M;
+  tp.keep_ld = K;
   return b_mn ? launch_thin<false, true>(ta, tb, tp, ceil_div(M, 128), splits, st, why)
               : launch_thin<false, false>(ta, tb, tp, ceil_div(M, 128), splits, st, why);
 }
@@ -1419,6 +1505,21 @@ static ScaleSrc scale_src(const qlora_nf4_t& q) {
   return s;
 }
 
+// Adapter dropout: the keep bitmask of X in the workspace (nullptr without
+// dropout), generated for this call from (seed, offset).
+static int dropout_mask(const LinearArgs& a, bool bwd, cudaStream_t st, const char** why, const uint32_t** keep) {
+  *keep = nullptr;
+  if (!a.drop) return 0;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(static_cast<char*>(a.ws) +
+                                               dropout_mask_offset(a.M, a.d, a.k, a.r, bwd));
+  if (launch_dropout_bits(a.M * a.k, *a.drop, bits, st) != cudaSuccess) {
+    *why = "dropout mask launch";
+    return QLORA_ERR_CUDA;
+  }
+  *keep = bits;
+  return 0;
+}
+
 int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   const int64_t M = a.M, d = a.d, k = a.k;
   const int rp = a.rp;
@@ -1426,6 +1527,11 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   Plan pl = make_plan(M, d, k, a.r, false, true);
   char* ws = static_cast<char*>(a.ws);
   uint16_t* T = own_T ? reinterpret_cast<uint16_t*>(ws + pl.off_T) : a.T;
+  const uint32_t* keep = nullptr;
+  int rc = dropout_mask(a, false, st, why, &keep);
+  if (rc) return rc;
+  // with dropout, T_s = BF16(s / (1 - p) * (X . keep) A^T)
+  const float s_down = a.drop ? a.s * a.drop->dscale : a.s;
   if (pl.fewtok) {
     CUtensorMap tm;
     if (!make_map(&tm, a.q->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, k / 2, d, k / 2, 128, 256,
@@ -1433,9 +1539,9 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
       *why = "tensor map encoding failed (few-token forward)";
       return QLORA_ERR_CUDA;
     }
-    return launch_fewtok_fwd(a, T, ws + pl.off_main, &tm, st, why);
+    return launch_fewtok_fwd(a, T, ws + pl.off_main, &tm, st, why, keep);
   }
-  int rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, a.s, pl.splits_T, T, st, why);
+  rc = run_lowrank_down(a.X, M, k, a.A, a.r, false, rp, s_down, pl.splits_T, T, st, why, keep);
   if (rc) return rc;
 
   const qlora_nf4_t& q = *a.q;
@@ -1510,11 +1616,16 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     cudaMemsetAsync(a.dB, 0, static_cast<size_t>(d) * r * 4, st);
     return 0;
   }
+  // adapter dropout: the same keep decisions as the forward, regenerated
+  const uint32_t* keep = nullptr;
+  rc = dropout_mask(a, true, st, why, &keep);
+  if (rc) return rc;
+  const float dscale = a.drop ? a.drop->dscale : 1.0f;
   // T_s (recompute when not saved)
   const uint16_t* T = a.Tin;
   if (!T) {
     uint16_t* Tw = reinterpret_cast<uint16_t*>(ws + pl.off_T);
-    rc = run_lowrank_down(a.X, M, k, a.A, r, false, rp, a.s, pl.splits_T, Tw, st, why);
+    rc = run_lowrank_down(a.X, M, k, a.A, r, false, rp, a.s * dscale, pl.splits_T, Tw, st, why, keep);
     if (rc) return rc;
     T = Tw;
   }
@@ -1545,7 +1656,9 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     mp.lora = a.A;
     mp.n_out = k;
     mp.steps_main = static_cast<int32_t>(ceil_div(d, 64));
-    mp.ext_steps = rp / 64;
+    // with dropout the adapter term is masked elementwise, so it cannot share
+    // the base accumulator: it is added afterwards by the dropout kernel
+    mp.ext_steps = keep ? 0 : rp / 64;
     mp.steps_per_split = static_cast<int32_t>(ceil_div(mp.steps_main, pl.main_splits));
     mp.splits = static_cast<int32_t>(ceil_div(mp.steps_main, mp.steps_per_split));
     mp.out = a.dX;
@@ -1571,6 +1684,10 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
       }
       QL_CHECK_LAUNCH("reduce launch (dX)");
     }
+    if (keep && launch_lora_up_dropout(U, rp, a.A, r, keep, dscale, M, k, a.dX, st) != cudaSuccess) {
+      *why = "dropout adapter-term launch (dX)";
+      return QLORA_ERR_CUDA;
+    }
   }
 
   // dA^T = X^T U_s  and  dB = dY^T T_s  (reduction over tokens, MN-major operands)
@@ -1588,6 +1705,10 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.r = r;
     tp.ld = k;
     tp.outf = a.dA;
+    tp.scale = dscale;          // dA = U_s^T (X . keep) / (1 - p)
+    tp.keep = keep;
+    tp.keep_rows = M;
+    tp.keep_ld = k;
     rc = launch_thin<true, true>(ta, tb, tp, ceil_div(k, 128), pl.splits_dA, st, why);
     if (rc) return rc;
   }
@@ -1604,6 +1725,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.mode = THIN_DB;
     tp.r = r;
     tp.outf = a.dB;
+    tp.scale = 1.0f;
     rc = launch_thin<true, true>(ta, tb, tp, ceil_div(d, 128), pl.splits_dB, st, why);
     if (rc) return rc;
   }

@@ -33,6 +33,20 @@ cudaError_t launch_lora_merge(const qlora_nf4_t& q, const uint16_t* A, const uin
 // device address and size of the library-owned quantisation scratch (current device)
 cudaError_t noalloc_scratch(void** out, size_t* bytes);
 
+// adapter dropout (qlora_dropout.cu)
+struct DropoutArgs {
+  float p;           // drop probability, 0 <= p < 1
+  uint32_t thr;      // ceil(p * 2^24): a 24-bit draw at or above it keeps the element
+  float dscale;      // RN32(1 / RN32(1 - p)), the scale of kept elements
+  uint64_t seed, offset;
+};
+uint32_t dropout_threshold(float p);
+// keep bitmask of n elements (bit b of word w <-> element 32 w + b) into bits[ceil(n / 32)]
+cudaError_t launch_dropout_bits(int64_t n, const DropoutArgs& d, uint32_t* bits, cudaStream_t st);
+// dX (M x k, bf16, in place) += dscale * keep . (U A), U = U_s (M x rp), A (r x k)
+cudaError_t launch_lora_up_dropout(const uint16_t* U, int rp, const uint16_t* A, int r, const uint32_t* keep,
+                                   float dscale, int64_t M, int64_t k, uint16_t* dX, cudaStream_t st);
+
 // linear layer (qlora_gemm.cu)
 struct LinearArgs {
   const uint16_t* X;    // M x k
@@ -51,10 +65,16 @@ struct LinearArgs {
   float* dB;            // d x r
   void* ws;
   size_t ws_bytes;
+  // adapter dropout (drop == nullptr: none).  The keep bitmask lives in the
+  // workspace past the plain layer's part, at dropout_mask_offset().
+  const DropoutArgs* drop;
 };
 
 size_t fwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r);
 size_t bwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r);
+// with adapter dropout: the plain layer's workspace, then the keep bitmask of X
+size_t dropout_mask_offset(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd);
+size_t dropout_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd);
 // Returns 0 on success, a negative qlora_status otherwise; `why` names the failure.
 int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why);
 int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why);
@@ -66,7 +86,7 @@ constexpr int kFewTokMax = 16;
 bool fewtok_eligible(int64_t M, int64_t d, int64_t k);
 size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k);
 int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensorMap* tm_codes, cudaStream_t st,
-                      const char** why);
+                      const char** why, const uint32_t* keep);
 
 // Raise a kernel's dynamic shared-memory limit once per (kernel, device); the
 // attribute call costs host time on every launch otherwise.  Instantiations of

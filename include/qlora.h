@@ -216,6 +216,55 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t M, const qlo
                      const uint16_t *T_save, uint16_t *dX, float *dA, float *dB,
                      void *workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* Adapter dropout ("LoRA and QLoRA: Efficient Fine-Tuning of Large Language
+ * Models" (fromzero2ai.dev), "Python Implementation: Fine-Tuning with PEFT and
+ * BitsAndBytes", step 4: lora_dropout = 0.05).  Dropout acts on the adapter's
+ * input only; the frozen base path sees X unchanged:
+ *     Y = X W^T + s (drop(X) A^T) B^T,   drop(X) = X . keep / (1 - p).
+ * The keep decision of element i = m * k + j of X comes from the counter-based
+ * generator Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as
+ * 1, 2, 3", SC 2011): output word i % 4 at counter (i / 4 low 32 bits, i / 4
+ * high 32 bits, offset low, offset high) under key (seed low, seed high);
+ * with u = (word >> 8) * 2^-24 the element is kept when u >= p.  Kept values
+ * are scaled by RN32(1 / RN32(1 - p)).  The backward regenerates the same
+ * decisions from (seed, offset), so no mask is stored between the calls; use
+ * a new offset (or seed) for every training step. */
+typedef struct {
+  float p;           /* drop probability, 0 <= p < 1 (0: the plain layer, bit for bit) */
+  uint64_t seed;     /* generator key                                                  */
+  uint64_t offset;   /* generator counter offset                                       */
+} qlora_dropout_t;
+
+/* Writes the keep bitmask of an M x k activation: bit b of keep_bits[w] is the
+ * decision for flat element 32 w + b (1 = kept); ceil(M * k / 32) words,
+ * bits past M * k are 0.  keep_bits: device, 4-byte aligned. */
+int qlora_dropout_mask(int64_t M, int64_t k, const qlora_dropout_t *drop, uint32_t *keep_bits,
+                       qlora_stream_t stream);
+
+/* Workspace bytes of qlora_linear_fwd_dropout (backward == 0) or
+ * qlora_linear_bwd_dropout (backward == 1): the plain layer's workspace plus
+ * the keep bitmask of X (M * k / 8 bytes, rounded up to 256).  Host-only. */
+int qlora_linear_dropout_workspace_size(int64_t M, int64_t d, int64_t k, int32_t r, int32_t backward,
+                                        size_t *bytes);
+
+/* qlora_linear_fwd with adapter dropout `drop` (NULL or p == 0: no dropout).
+ * T_save receives BF16(s * drop(X) * A^T).  Other arguments and requirements
+ * as for qlora_linear_fwd; workspace from qlora_linear_dropout_workspace_size.
+ * A probability outside [0, 1) returns QLORA_ERR_INVALID_ARG. */
+int qlora_linear_fwd_dropout(const uint16_t *X, int64_t M, const qlora_nf4_t *q, const uint16_t *A,
+                             const uint16_t *B, int32_t r, float alpha, const qlora_dropout_t *drop, uint16_t *Y,
+                             uint16_t *T_save, void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* qlora_linear_bwd for the dropout forward with the same `drop`:
+ *     U  = s dY B,   dX = dY W + (U A) . keep / (1 - p),
+ *     dA = U^T drop(X),   dB = s dY^T (drop(X) A^T).
+ * T_save: the buffer the dropout forward filled (NULL recomputes it with the
+ * same mask).  Workspace from qlora_linear_dropout_workspace_size. */
+int qlora_linear_bwd_dropout(const uint16_t *dY, const uint16_t *X, int64_t M, const qlora_nf4_t *q,
+                             const uint16_t *A, const uint16_t *B, int32_t r, float alpha,
+                             const qlora_dropout_t *drop, const uint16_t *T_save, uint16_t *dX, float *dA, float *dB,
+                             void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
 /* The library's NF4 table C[0..15] (fp32, ascending) copied to host memory. */
 int qlora_nf4_codebook(float out[16]);
 
@@ -224,6 +273,17 @@ int qlora_nf4_codebook(float out[16]);
  * read, otherwise the code of the first failure.  Returns QLORA_ERR_DEVICE
  * when *status != 0. */
 int qlora_device_status(qlora_stream_t stream, int32_t *status);
+
+/* Self-test of the device-side failure path (not a paper operation).  Every
+ * wait inside the library's kernels is bounded; when one runs out the kernel
+ * records a code in the status word, releases what it holds (TMEM) and
+ * returns, so the context stays usable.  This call exercises exactly that path
+ * without any fault: one CTA takes 32 TMEM columns and waits on a barrier that
+ * nothing arrives at, for limit_us microseconds (1 .. 1000000).  It then
+ * records code 7 in the status word, frees the TMEM and writes 2 to *result
+ * (device int32, 4-byte aligned).  qlora_device_status afterwards returns
+ * QLORA_ERR_DEVICE with status 7 and clears it. */
+int qlora_selftest_wait_timeout(uint32_t limit_us, int32_t *result, qlora_stream_t stream);
 
 /* Tracing: every kernel launch of the library belongs to one class. */
 enum {

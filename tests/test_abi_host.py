@@ -133,3 +133,43 @@ def test_param_count_matches_buffer_shapes(golden):
     g = golden("lora_param_count.json")
     # A is r x k and B is d x r: the entries the backward writes
     assert g["r"] * g["k"] + g["d"] * g["r"] == g["trainable"]
+
+
+def test_dropout_validation_without_gpu(L):
+    """Adapter dropout entry points: the probability must lie in [0, 1), the
+    workspace grows by the keep bitmask (M k / 8 bytes rounded up to 256), and
+    every refusal happens before any device work (fake aligned pointers)."""
+    n, nd = ctypes.c_size_t(), ctypes.c_size_t()
+    for bwd in (0, 1):
+        assert L.qlora_linear_workspace_size(200, 520, 704, 16, bwd, ctypes.byref(n)) == 0
+        assert L.qlora_linear_dropout_workspace_size(200, 520, 704, 16, bwd, ctypes.byref(nd)) == 0
+        mask = -(-200 * 704 // 32) * 4
+        assert nd.value == -(-n.value // 256) * 256 + -(-mask // 256) * 256
+    assert L.qlora_linear_dropout_workspace_size(16, 512, 500, 8, 0, ctypes.byref(nd)) == -2   # k % 64
+    st = Q.QloraNF4(512, 512, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+    for p in (1.0, 1.5, -0.1, float("nan")):
+        drop = Q.QloraDropout(p, 1, 2)
+        rc = L.qlora_linear_fwd_dropout(0x10000, 16, ctypes.byref(st), 0x10000, 0x20000, 8, 16.0, ctypes.byref(drop),
+                                        0x30000, None, 0x40000, 1 << 30, None)
+        assert rc == -1 and b"[0, 1)" in L.qlora_last_error(), p
+        rc = L.qlora_linear_bwd_dropout(0x10000, 0x10000, 16, ctypes.byref(st), 0x10000, 0x20000, 8, 16.0,
+                                        ctypes.byref(drop), None, 0x30000, 0x40000, 0x50000, 0x60000, 1 << 30, None)
+        assert rc == -1, p
+        assert L.qlora_dropout_mask(4, 64, ctypes.byref(drop), 0x10000, None) == -1
+    drop = Q.QloraDropout(0.05, 1, 2)
+    # a workspace sized for the plain layer is too small once the mask is needed
+    L.qlora_linear_workspace_size(16, 512, 512, 8, 0, ctypes.byref(n))
+    rc = L.qlora_linear_fwd_dropout(0x10000, 16, ctypes.byref(st), 0x10000, 0x20000, 8, 16.0, ctypes.byref(drop),
+                                    0x30000, None, 0x40000, n.value, None)
+    assert rc == -4
+    assert L.qlora_dropout_mask(4, 64, None, 0x10000, None) == -1
+    assert L.qlora_dropout_mask(4, 64, ctypes.byref(drop), None, None) == -1
+    assert L.qlora_dropout_mask(4, 64, ctypes.byref(drop), 0x10002, None) == -3       # 4-byte alignment
+    assert L.qlora_dropout_mask(0, 64, ctypes.byref(drop), None, None) == 0            # nothing to do
+
+
+def test_selftest_validation_without_gpu(L):
+    assert L.qlora_selftest_wait_timeout(0, 0x10000, None) == -1
+    assert L.qlora_selftest_wait_timeout(1000001, 0x10000, None) == -1
+    assert L.qlora_selftest_wait_timeout(100, None, None) == -1
+    assert L.qlora_selftest_wait_timeout(100, 0x10002, None) == -3
