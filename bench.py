@@ -239,29 +239,52 @@ def run_ours(args, work, wl_name):
     projs = work["proj"]
     drop_p = work.get("dropout", 0.0)
     step_no = [0]          # the dropout generator's offset: a new mask every step (and projection)
+    # Units of the step: a single projection, or (grouped workloads) the
+    # projections that share X (q, k, v; gate, up), run as one grouped layer.
+    units = work.get("groups") or [[pi] for pi in range(len(projs))]
     # adapter gradients of every projection in one flat fp32 bucket (one all-reduce per step)
-    bucket = GradBucket([s_ for _, d, k in projs for s_ in ((r, k), (d, r))], dev)
+    shapes = []
+    for u in units:
+        k = projs[u[0]][2]
+        shapes += [(len(u) * r, k), (sum(projs[pi][1] for pi in u), r)]
+    bucket = GradBucket(shapes, dev)
     bufs = []
     h2d_bytes = d2h_bytes = 0
-    for pi, (name, d, k) in enumerate(projs):
-        tok_seed = pi + 1000 * rank         # each rank has its own token batch
-        host = {"W0": synth.weight(d, k, seed=pi), "A": synth.lora_a(r, k, seed=pi), "B": synth.lora_b(d, r, seed=pi),
+    for ui, u in enumerate(units):
+        p0 = u[0]
+        ds = [projs[pi][1] for pi in u]
+        d, k = sum(ds), projs[p0][2]
+        tok_seed = p0 + 1000 * rank         # each rank has its own token batch
+        host = {"A": np.concatenate([synth.lora_a(r, k, seed=pi) for pi in u]),
+                "B": np.concatenate([synth.lora_b(projs[pi][1], r, seed=pi) for pi in u]),
                 "X": synth.activations(M, k, seed=tok_seed), "dY": synth.grad_output(M, d, seed=tok_seed)}
-        b = {"d": d, "k": k, "name": name}
+        for j, pi in enumerate(u):
+            host[f"W0_{j}"] = synth.weight(projs[pi][1], k, seed=pi)
+        b = {"d": d, "k": k, "name": "+".join(projs[pi][0] for pi in u), "n": len(u)}
         for key, arr in host.items():
             pinned = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).pin_memory()
             b["h_" + key] = pinned
             b[key] = pinned.to(dev, non_blocking=True)
             h2d_bytes += pinned.numel() * 2
-        b["q"] = Q.nf4_alloc(d, k, True, dev)
-        b["qws"] = torch.empty(max(Q.qlora_nf4_sizes(d, k, 64, True)[1], 16), dtype=torch.uint8, device=dev)
+        if len(u) > 1:
+            b["g"] = Q.nf4_alloc_group(ds, k, True, dev)
+            b["qparts"] = b["g"].parts
+        else:
+            b["q"] = Q.nf4_alloc(d, k, True, dev)
+            b["qparts"] = [b["q"]]
+        b["qws"] = torch.empty(max(max(Q.qlora_nf4_sizes(x, k, 64, True)[1] for x in ds), 16), dtype=torch.uint8,
+                               device=dev)
         b["Y"] = torch.empty(M, d, dtype=torch.bfloat16, device=dev)
-        b["T"] = torch.empty(M, Q.qlora_rank_pad(r), dtype=torch.bfloat16, device=dev)
+        b["T"] = torch.empty(M, Q.qlora_rank_pad(len(u) * r), dtype=torch.bfloat16, device=dev)
         b["dX"] = torch.empty(M, k, dtype=torch.bfloat16, device=dev)
-        b["dA"] = bucket.views[2 * pi]
-        b["dB"] = bucket.views[2 * pi + 1]
-        wsz = Q.qlora_linear_dropout_workspace_size if drop_p else Q.qlora_linear_workspace_size
-        nws = max(wsz(M, d, k, r, False), wsz(M, d, k, r, True))
+        b["dA"] = bucket.views[2 * ui]
+        b["dB"] = bucket.views[2 * ui + 1]
+        if len(u) > 1:
+            nws = max(Q.qlora_grouped_workspace_size(M, b["g"], r, False),
+                      Q.qlora_grouped_workspace_size(M, b["g"], r, True))
+        else:
+            wsz = Q.qlora_linear_dropout_workspace_size if drop_p else Q.qlora_linear_workspace_size
+            nws = max(wsz(M, d, k, r, False), wsz(M, d, k, r, True))
         b["ws"] = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         for key in ("Y", "dX", "dA", "dB"):
             b["h_" + key] = torch.empty(b[key].shape, dtype=b[key].dtype, pin_memory=True)
@@ -271,21 +294,29 @@ def run_ours(args, work, wl_name):
     stream = torch.cuda.current_stream()
 
     def step():
-        for pi, b in enumerate(bufs):
-            drop = (drop_p, 1234 + rank, step_no[0] * len(bufs) + pi) if drop_p else None
-            Q.nf4_quantize(b["W0"], True, out=b["q"], workspace=b["qws"], stream=stream)
-            Q.qlora_linear_fwd(b["X"], b["q"], b["A"], b["B"], alpha, Y=b["Y"], T_save=b["T"], workspace=b["ws"],
-                               stream=stream, dropout=drop)
-            Q.qlora_linear_bwd(b["dY"], b["X"], b["q"], b["A"], b["B"], alpha, T_save=b["T"], dX=b["dX"],
-                               dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream, dropout=drop)
+        for ui, b in enumerate(bufs):
+            drop = (drop_p, 1234 + rank, step_no[0] * len(bufs) + ui) if drop_p else None
+            for j, part in enumerate(b["qparts"]):
+                Q.nf4_quantize(b[f"W0_{j}"], True, out=part, workspace=b["qws"], stream=stream)
+            if b["n"] > 1:
+                Q.qlora_linear_fwd_grouped(b["X"], b["g"], b["A"], b["B"], alpha, r=r, Y=b["Y"], T_save=b["T"],
+                                           workspace=b["ws"], stream=stream)
+                Q.qlora_linear_bwd_grouped(b["dY"], b["X"], b["g"], b["A"], b["B"], alpha, r=r, T_save=b["T"],
+                                           dX=b["dX"], dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream)
+            else:
+                Q.qlora_linear_fwd(b["X"], b["q"], b["A"], b["B"], alpha, Y=b["Y"], T_save=b["T"],
+                                   workspace=b["ws"], stream=stream, dropout=drop)
+                Q.qlora_linear_bwd(b["dY"], b["X"], b["q"], b["A"], b["B"], alpha, T_save=b["T"], dX=b["dX"],
+                                   dA=b["dA"], dB=b["dB"], workspace=b["ws"], stream=stream, dropout=drop)
         step_no[0] += 1
         if world > 1:
             bucket.allreduce()
 
     def h2d():
         for b in bufs:
-            for key in ("W0", "A", "B", "X", "dY"):
-                b[key].copy_(b["h_" + key], non_blocking=True)
+            for key in b:
+                if key.startswith("h_") and key[2:] in ("A", "B", "X", "dY") or key.startswith("h_W0_"):
+                    b[key[2:]].copy_(b[key], non_blocking=True)
 
     def d2h():
         for b in bufs:
@@ -388,6 +419,7 @@ def run_ours(args, work, wl_name):
         "config": {"workload": wl_name, "tokens_per_rank": M, "rank": r, "alpha": alpha,
                    "projections": [f"{n}:{d}x{k}" for n, d, k in projs], "nf4_blocksize": 64,
                    "double_quant": True, "lora_dropout": drop_p,
+                   "grouped": [[projs[pi][0] for pi in u] for u in units if len(u) > 1],
                    "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": "working set per step larger than L2 (no explicit flush)"},
         "breakdown_ms_per_step": {c: round(v / args.steps, 4) for c, v in kms.items()},
@@ -588,6 +620,7 @@ def main():
     ap.add_argument("--workload", default="llama65b_block_m8192",
                     choices=("llama7b_proj_set_m4096", "llama65b_block_m8192", "proj_q_4096", "tiny_512",
                              "llama7b_proj_set_m4096_dropout", "llama65b_block_m8192_dropout",
+                             "llama7b_proj_set_m4096_grouped", "llama65b_block_m8192_grouped",
                              "decode_28672x8192", "quant_sweep", "merge_sweep"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

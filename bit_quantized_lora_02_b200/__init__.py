@@ -30,7 +30,8 @@ EXPORTS = ("qlora_nf4_sizes", "nf4_quantize", "nf4_quantize_noalloc", "nf4_dequa
            "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status", "qlora_last_error",
            "qlora_profile_enable", "qlora_profile_read",
            "qlora_dropout_mask", "qlora_linear_dropout_workspace_size", "qlora_linear_fwd_dropout",
-           "qlora_linear_bwd_dropout", "qlora_selftest_wait_timeout")
+           "qlora_linear_bwd_dropout", "qlora_selftest_wait_timeout", "qlora_grouped_workspace_size",
+           "qlora_linear_fwd_grouped", "qlora_linear_bwd_grouped")
 
 KERNEL_CLASSES = ("quant", "dq_const", "dequant", "fwd_gemm", "bwd_gemm", "lora_gemm", "aux")
 
@@ -46,6 +47,14 @@ class QloraNF4(ctypes.Structure):
     _fields_ = [("d", ctypes.c_int64), ("k", ctypes.c_int64), ("blocksize", ctypes.c_int32),
                 ("double_quant", ctypes.c_int32), ("codes", ctypes.c_void_p), ("absmax", ctypes.c_void_p),
                 ("c2", ctypes.c_void_p), ("c1", ctypes.c_void_p), ("mean", ctypes.c_void_p)]
+
+
+MAX_GROUP = 4
+
+
+class QloraNF4Group(ctypes.Structure):
+    """Mirror of ``qlora_nf4_group_t``."""
+    _fields_ = [("n", ctypes.c_int32), ("d", ctypes.c_int64 * MAX_GROUP), ("w", QloraNF4)]
 
 
 class QloraDropout(ctypes.Structure):
@@ -87,6 +96,11 @@ def lib() -> ctypes.CDLL:
     L.qlora_linear_bwd_dropout.argtypes = [vp, vp, c_i64, ctypes.POINTER(QloraNF4), vp, vp, c_i32, ctypes.c_float,
                                            ctypes.POINTER(QloraDropout), vp, vp, vp, vp, vp, c_sz, vp]
     L.qlora_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp, vp]
+    G = ctypes.POINTER(QloraNF4Group)
+    L.qlora_grouped_workspace_size.argtypes = [c_i64, G, c_i32, c_i32, ctypes.POINTER(c_sz)]
+    L.qlora_linear_fwd_grouped.argtypes = [vp, c_i64, G, vp, vp, c_i32, ctypes.c_float, vp, vp, vp, c_sz, vp]
+    L.qlora_linear_bwd_grouped.argtypes = [vp, vp, c_i64, G, vp, vp, c_i32, ctypes.c_float, vp, vp, vp, vp, vp,
+                                           c_sz, vp]
     L.qlora_last_error.restype = ctypes.c_char_p
     L.qlora_profile_enable.argtypes = [c_i32]
     L.qlora_profile_read.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]
@@ -95,7 +109,8 @@ def lib() -> ctypes.CDLL:
                  "qlora_linear_fwd", "qlora_linear_bwd", "qlora_nf4_codebook", "qlora_device_status",
                  "qlora_profile_enable", "qlora_profile_read", "qlora_dropout_mask",
                  "qlora_linear_dropout_workspace_size", "qlora_linear_fwd_dropout", "qlora_linear_bwd_dropout",
-                 "qlora_selftest_wait_timeout"):
+                 "qlora_selftest_wait_timeout", "qlora_grouped_workspace_size", "qlora_linear_fwd_grouped",
+                 "qlora_linear_bwd_grouped"):
         getattr(L, name).restype = c_i32
     _lib = L
     return L
@@ -284,6 +299,145 @@ def qlora_lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: floa
     _check(lib().qlora_lora_merge(ctypes.byref(st), A.data_ptr(), B.data_ptr(), r, float(alpha), out.data_ptr(),
                                   _stream(stream)))
     return out
+
+
+# ---------------------------------------------------------------------------
+# grouped projections (several weights that share their input X)
+# ---------------------------------------------------------------------------
+@dataclass
+class NF4Group:
+    """Stacked NF4 buffers of n projections that share X (layout of
+    ``qlora_nf4_group_t``): `w` describes all rows together and `parts[i]` is
+    the slice of projection i (quantise W_i into it with nf4_quantize)."""
+    ds: tuple
+    w: NF4Weight
+    parts: list
+
+    def struct(self, device=None) -> QloraNF4Group:
+        n = len(self.ds)
+        st = QloraNF4Group()
+        st.n = n
+        for i in range(MAX_GROUP):
+            st.d[i] = int(self.ds[i]) if i < n else 0
+        st.w = self.w.struct(device)
+        if self.w.double_quant and _nbytes(self.w.mean) < 4 * n:
+            raise ValueError(f"the group's mean buffer holds {_nbytes(self.w.mean)} bytes, {n} means need {4 * n}")
+        return st
+
+
+def nf4_alloc_group(ds, k: int, double_quant: bool = True, device=None) -> NF4Group:
+    """Stacked buffers for projections of ds[i] x k rows (ds[i] % 256 == 0 for
+    all but the last) and per-projection slice descriptors."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    ds = tuple(int(x) for x in ds)
+    if not 1 <= len(ds) <= MAX_GROUP:
+        raise ValueError(f"1..{MAX_GROUP} projections, got {len(ds)}")
+    if any(x % 256 for x in ds[:-1]):
+        raise ValueError("every projection but the last needs a multiple of 256 rows")
+    mode = int(double_quant)
+    per = [qlora_nf4_sizes(d, k, 64, mode)[0] for d in ds]
+    tot = [sum(sz[j] for sz in per) for j in range(5)]
+
+    def buf(nbytes, dtype, esize):
+        return torch.empty(max(nbytes // esize, 1) + 16 // esize, dtype=dtype, device=device)
+    codes = buf(tot[0], torch.uint8, 1)
+    c2_dtype = torch.uint8 if mode == 2 else torch.int8
+    absmax = buf(tot[1], torch.float32, 4) if not mode else None
+    c2 = buf(tot[2], c2_dtype, 1) if mode else None
+    c1 = buf(tot[3], torch.float32, 4) if mode else None
+    mean = buf(4 * len(ds), torch.float32, 4) if mode else None
+    w = NF4Weight(sum(ds), k, mode, codes, absmax, c2, c1, mean)
+    parts, off = [], [0] * 5
+    for i, (d, sz) in enumerate(zip(ds, per)):
+        def sl(t, j, esize):
+            return None if t is None else t[off[j] // esize: (off[j] + sz[j]) // esize]
+        parts.append(NF4Weight(d, k, mode, sl(codes, 0, 1), sl(absmax, 1, 4), sl(c2, 2, 1), sl(c1, 3, 4),
+                               None if mean is None else mean[i:i + 1]))
+        off = [o + x for o, x in zip(off, sz)]
+    return NF4Group(ds, w, parts)
+
+
+def nf4_quantize_group(Ws, double_quant: bool = True, out: Optional[NF4Group] = None, stream=None) -> NF4Group:
+    """Quantise each W_i (d_i x k bf16) on its own into the group's stacked buffers."""
+    k = Ws[0].shape[1]
+    g = out or nf4_alloc_group([W.shape[0] for W in Ws], k, double_quant, Ws[0].device)
+    for W, part in zip(Ws, g.parts):
+        nf4_quantize(W, double_quant=part.double_quant, out=part, stream=stream)
+    return g
+
+
+def qlora_grouped_workspace_size(M: int, g: NF4Group, r: int, backward: bool) -> int:
+    n = ctypes.c_size_t()
+    st = g.struct()
+    _check(lib().qlora_grouped_workspace_size(M, ctypes.byref(st), r, int(backward), ctypes.byref(n)))
+    return n.value
+
+
+def qlora_linear_fwd_grouped(X: torch.Tensor, g: NF4Group, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                             r: Optional[int] = None, Y: Optional[torch.Tensor] = None,
+                             T_save: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                             stream=None, save_T: bool = True):
+    """Y = [Y_0 | Y_1 | ...], Y_i = X W_i^T + (alpha/r) (X A_i^T) B_i^T with
+    A = stacked A_i ((n r) x k) and B = stacked B_i (sum d_i x r)."""
+    n = len(g.ds)
+    M, k = X.shape
+    r = A.shape[0] // n if r is None else r
+    dev = X.device
+    dt = g.w.d
+    if Y is None:
+        Y = torch.empty(M, dt, dtype=torch.bfloat16, device=dev)
+    if T_save is None and save_T:
+        T_save = torch.empty(M, qlora_rank_pad(n * r), dtype=torch.bfloat16, device=dev)
+    _expect(X, "X", (M, g.w.k), torch.bfloat16)
+    _expect(A, "A", (n * r, g.w.k), torch.bfloat16)
+    _expect(B, "B", (dt, r), torch.bfloat16)
+    _expect(Y, "Y", (M, dt), torch.bfloat16)
+    _expect(T_save, "T_save", (M, qlora_rank_pad(n * r)), torch.bfloat16, required=False)
+    if workspace is None:
+        nws = qlora_grouped_workspace_size(M, g, r, False)
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev) if nws else None
+    _same_device(dev, A=A, B=B, Y=Y, T_save=T_save, workspace=workspace)
+    st = g.struct(dev)
+    _check(lib().qlora_linear_fwd_grouped(X.data_ptr(), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
+                                          float(alpha), Y.data_ptr(), _ptr(T_save), _ptr(workspace),
+                                          _nbytes(workspace), _stream(stream)))
+    return Y, T_save
+
+
+def qlora_linear_bwd_grouped(dY: torch.Tensor, X: torch.Tensor, g: NF4Group, A: torch.Tensor, B: torch.Tensor,
+                             alpha: float, r: Optional[int] = None, T_save: Optional[torch.Tensor] = None,
+                             dX: Optional[torch.Tensor] = None, dA: Optional[torch.Tensor] = None,
+                             dB: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                             stream=None, need_dX: bool = True):
+    """Backward of qlora_linear_fwd_grouped; returns (dX, dA stacked, dB stacked)."""
+    n = len(g.ds)
+    M = dY.shape[0]
+    r = A.shape[0] // n if r is None else r
+    dev = dY.device
+    dt = g.w.d
+    if dX is None and need_dX:
+        dX = torch.empty(M, g.w.k, dtype=torch.bfloat16, device=dev)
+    if dA is None:
+        dA = torch.empty(n * r, g.w.k, dtype=torch.float32, device=dev)
+    if dB is None:
+        dB = torch.empty(dt, r, dtype=torch.float32, device=dev)
+    _expect(dY, "dY", (M, dt), torch.bfloat16)
+    _expect(X, "X", (M, g.w.k), torch.bfloat16)
+    _expect(A, "A", (n * r, g.w.k), torch.bfloat16)
+    _expect(B, "B", (dt, r), torch.bfloat16)
+    _expect(T_save, "T_save", (M, qlora_rank_pad(n * r)), torch.bfloat16, required=False)
+    _expect(dX, "dX", (M, g.w.k), torch.bfloat16, required=False)
+    _expect(dA, "dA", (n * r, g.w.k), torch.float32)
+    _expect(dB, "dB", (dt, r), torch.float32)
+    if workspace is None:
+        nws = qlora_grouped_workspace_size(M, g, r, True)
+        workspace = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev) if nws else None
+    _same_device(dev, X=X, A=A, B=B, T_save=T_save, dX=dX, dA=dA, dB=dB, workspace=workspace)
+    st = g.struct(dev)
+    _check(lib().qlora_linear_bwd_grouped(_ptr(dY), _ptr(X), M, ctypes.byref(st), A.data_ptr(), B.data_ptr(), r,
+                                          float(alpha), _ptr(T_save), _ptr(dX), dA.data_ptr(), dB.data_ptr(),
+                                          _ptr(workspace), _nbytes(workspace), _stream(stream)))
+    return dX, dA, dB
 
 
 def qlora_rank_pad(r: int) -> int:

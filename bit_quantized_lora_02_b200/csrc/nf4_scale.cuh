@@ -18,13 +18,33 @@
 namespace qlora {
 
 // Block scale s^ for NF4 block `blk`.
+//
+// A grouped weight stacks the NF4 buffers of up to four projections that share
+// their input (q, k, v or gate, up), each quantised on its own: codes, c2 (or
+// absmax) and c1 are laid out back to back, and each projection keeps its own
+// mean.  Rows from gstart[i] on belong to projection i + 1; a plain weight has
+// ngrp <= 1 and reads mean[0].
 struct ScaleSrc {
   const float* absmax;   // DQ off
   const int8_t* c2;      // DQ on
   const float* c1;
-  const float* mean;     // device scalar, DQ on
+  const float* mean;     // device, one per projection, DQ on
   int dq;
+  int ngrp;              // projections stacked in the weight (0 or 1: a plain weight)
+  int64_t gstart[3];     // first row of projections 1, 2, 3
 };
+
+// Projection that weight row `row` belongs to.
+__host__ __device__ __forceinline__ int group_of(const ScaleSrc& s, int64_t row) {
+  int g = 0;
+#pragma unroll
+  for (int j = 0; j < 3; ++j) g += (j + 1 < s.ngrp && row >= s.gstart[j]) ? 1 : 0;
+  return g;
+}
+
+__device__ __forceinline__ float group_mean(const ScaleSrc& s, int64_t row) {
+  return s.dq ? __ldg(s.mean + group_of(s, row)) : 0.0f;
+}
 
 struct ScaleRaw {
   float a;   // absmax (DQ off) or c1 (DQ on)

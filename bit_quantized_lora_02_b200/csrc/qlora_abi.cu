@@ -356,7 +356,112 @@ static int linear_bwd(const uint16_t* dY, const uint16_t* X, int64_t M, const ql
   return ok();
 }
 
+// Grouped projections: n projections that share X, their NF4 buffers stacked.
+// Checks the group and fills the grouping fields of `a`; *d_total and *r_all
+// are the stacked weight's rows and the projections' ranks together.
+static int check_group(const qlora_nf4_group_t* g, int32_t r, LinearArgs* a) {
+  if (!g) return fail(QLORA_ERR_INVALID_ARG, "group descriptor is NULL");
+  if (g->n < 1 || g->n > QLORA_MAX_GROUP) return fail(QLORA_ERR_INVALID_ARG, "group of %d projections (1..4)", g->n);
+  int64_t total = 0;
+  for (int i = 0; i < g->n; ++i) {
+    if (g->d[i] <= 0) return fail(QLORA_ERR_INVALID_ARG, "projection %d has %lld rows", i, (long long)g->d[i]);
+    if (i + 1 < g->n && g->d[i] % 256)
+      return fail(QLORA_ERR_UNSUPPORTED, "projection %d: rows %lld not a multiple of 256 (all but the last must be)",
+                  i, (long long)g->d[i]);
+    total += g->d[i];
+  }
+  if (total != g->w.d)
+    return fail(QLORA_ERR_INVALID_ARG, "stacked weight has %lld rows, the projections %lld", (long long)g->w.d,
+                (long long)total);
+  if (g->n > 1 && r % 8) return fail(QLORA_ERR_UNSUPPORTED, "grouped projections need r %% 8 == 0 (r=%d)", r);
+  if (static_cast<int64_t>(g->n) * r > 256)
+    return fail(QLORA_ERR_UNSUPPORTED, "n * r = %lld above 256", static_cast<long long>(g->n) * r);
+  a->ngrp = g->n;
+  a->r_group = r;
+  int64_t row = 0;
+  for (int i = 0; i < 3; ++i) {
+    row += (i < g->n) ? g->d[i] : 0;
+    a->gstart[i] = row;
+  }
+  return QLORA_OK;
+}
+
 extern "C" {
+
+int qlora_grouped_workspace_size(int64_t M, const qlora_nf4_group_t* g, int32_t r, int32_t backward,
+                                 size_t* bytes) {
+  if (!bytes) return fail(QLORA_ERR_INVALID_ARG, "bytes is NULL");
+  LinearArgs a{};
+  int rc = check_group(g, r, &a);
+  if (rc) return rc;
+  const int32_t rall = g->n * r;
+  if ((rc = check_linear_shape(M, g->w.d, g->w.k, rall))) return rc;
+  *bytes = backward ? bwd_workspace_bytes(M, g->w.d, g->w.k, rall) : fwd_workspace_bytes(M, g->w.d, g->w.k, rall);
+  return ok();
+}
+
+int qlora_linear_fwd_grouped(const uint16_t* X, int64_t M, const qlora_nf4_group_t* g, const uint16_t* A,
+                             const uint16_t* B, int32_t r, float alpha, uint16_t* Y, uint16_t* T_save,
+                             void* workspace, size_t workspace_bytes, qlora_stream_t stream) {
+  LinearArgs a{};
+  int rc = check_group(g, r, &a);
+  if (rc) return rc;
+  const qlora_nf4_t* q = &g->w;
+  const int32_t rall = g->n * r;
+  int64_t N = 0;
+  if ((rc = check_nf4(q, &N))) return rc;
+  if ((rc = check_linear_shape(M, q->d, q->k, rall))) return rc;
+  if (M == 0) return ok();
+  if ((rc = check_codes_tma(q))) return rc;
+  if ((rc = check_ptr16(X, "X", true)) || (rc = check_ptr16(A, "A", true)) || (rc = check_ptr16(B, "B", true)) ||
+      (rc = check_ptr16(Y, "Y", true)) || (rc = check_ptr16(T_save, "T_save", false)))
+    return rc;
+  const size_t need = fwd_workspace_bytes(M, q->d, q->k, rall);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(QLORA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : 0);
+  if (workspace && (rc = check_ptr16(workspace, "workspace", false))) return rc;
+  if ((rc = bind_device(X))) return rc;
+  a.X = X; a.M = M; a.d = q->d; a.k = q->k; a.q = q; a.A = A; a.B = B; a.r = rall; a.rp = qlora_rank_pad(rall);
+  a.s = alpha / static_cast<float>(r);
+  a.Y = Y; a.T = T_save; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  const char* why = "";
+  rc = launch_linear_fwd(a, static_cast<cudaStream_t>(stream), &why);
+  if (rc) return fail(rc, "qlora_linear_fwd_grouped: %s", why);
+  return ok();
+}
+
+int qlora_linear_bwd_grouped(const uint16_t* dY, const uint16_t* X, int64_t M, const qlora_nf4_group_t* g,
+                             const uint16_t* A, const uint16_t* B, int32_t r, float alpha, const uint16_t* T_save,
+                             uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+                             qlora_stream_t stream) {
+  LinearArgs a{};
+  int rc = check_group(g, r, &a);
+  if (rc) return rc;
+  const qlora_nf4_t* q = &g->w;
+  const int32_t rall = g->n * r;
+  int64_t N = 0;
+  if ((rc = check_nf4(q, &N))) return rc;
+  if ((rc = check_linear_shape(M, q->d, q->k, rall))) return rc;
+  if ((rc = check_ptr16(dA, "dA", true)) || (rc = check_ptr16(dB, "dB", true))) return rc;
+  if (M > 0 && (rc = check_codes_tma(q))) return rc;
+  if ((rc = check_ptr16(dY, "dY", M > 0)) || (rc = check_ptr16(X, "X", M > 0)) || (rc = check_ptr16(A, "A", true)) ||
+      (rc = check_ptr16(B, "B", true)) || (rc = check_ptr16(dX, "dX", false)) ||
+      (rc = check_ptr16(T_save, "T_save", false)))
+    return rc;
+  const size_t need = bwd_workspace_bytes(M, q->d, q->k, rall);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(QLORA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need, workspace ? workspace_bytes : 0);
+  if (workspace && (rc = check_ptr16(workspace, "workspace", false))) return rc;
+  if ((rc = bind_device(dA))) return rc;
+  a.dY = dY; a.X = X; a.M = M; a.d = q->d; a.k = q->k; a.q = q; a.A = A; a.B = B; a.r = rall;
+  a.rp = qlora_rank_pad(rall);
+  a.s = alpha / static_cast<float>(r);
+  a.Tin = T_save; a.dX = dX; a.dA = dA; a.dB = dB; a.ws = workspace; a.ws_bytes = workspace_bytes;
+  const char* why = "";
+  rc = launch_linear_bwd(a, static_cast<cudaStream_t>(stream), &why);
+  if (rc) return fail(rc, "qlora_linear_bwd_grouped: %s", why);
+  return ok();
+}
 
 int qlora_linear_fwd(const uint16_t* X, int64_t M, const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B,
                      int32_t r, float alpha, uint16_t* Y, uint16_t* T_save, void* workspace, size_t workspace_bytes,

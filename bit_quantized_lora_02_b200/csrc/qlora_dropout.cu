@@ -44,8 +44,11 @@ namespace {
 __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int i = 0; i < 10; ++i) {
-    const uint32_t lo0 = c.x * 0xD2511F53u, hi0 = __umulhi(c.x, 0xD2511F53u);
-    const uint32_t lo1 = c.z * 0xCD9E8D57u, hi1 = __umulhi(c.z, 0xCD9E8D57u);
+    // one widening multiply gives both halves of each product
+    const uint64_t p0 = static_cast<uint64_t>(c.x) * 0xD2511F53u;
+    const uint64_t p1 = static_cast<uint64_t>(c.z) * 0xCD9E8D57u;
+    const uint32_t lo0 = static_cast<uint32_t>(p0), hi0 = static_cast<uint32_t>(p0 >> 32);
+    const uint32_t lo1 = static_cast<uint32_t>(p1), hi1 = static_cast<uint32_t>(p1 >> 32);
     c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
     k0 += 0x9E3779B9u;
     k1 += 0xBB67AE85u;
@@ -61,6 +64,9 @@ __global__ void __launch_bounds__(256) k_dropout_bits(int64_t n, uint32_t thr, u
   griddep_launch_dependents();
   const int64_t w = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nw = (n + 31) >> 5;
+  // (word >> 8) >= thr  <=>  word >= thr * 2^8 (thr <= 2^24; thr == 2^24 would
+  // drop everything and needs p = 1, which is refused)
+  const uint32_t thr8 = thr << 8;
   uint32_t word = 0;
   if (w < nw) {
 #pragma unroll
@@ -68,13 +74,14 @@ __global__ void __launch_bounds__(256) k_dropout_bits(int64_t n, uint32_t thr, u
       const uint64_t q = static_cast<uint64_t>(w) * 8u + static_cast<uint64_t>(t);
       const uint4 r = philox4x32_10(
           make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32), off_lo, off_hi), seed_lo, seed_hi);
-      const uint32_t v[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t e = 32 * w + 4 * t + i;
-        if ((v[i] >> 8) >= thr && e < n) word |= 1u << (4 * t + i);
-      }
+      word |= (r.x >= thr8 ? 1u : 0u) << (4 * t);
+      word |= (r.y >= thr8 ? 1u : 0u) << (4 * t + 1);
+      word |= (r.z >= thr8 ? 1u : 0u) << (4 * t + 2);
+      word |= (r.w >= thr8 ? 1u : 0u) << (4 * t + 3);
     }
+    // elements past n (a ragged last word) are not kept
+    const int64_t valid = n - 32 * w;
+    if (valid < 32) word &= (1u << valid) - 1u;
   }
   griddep_wait();   // the previous kernel may still read an earlier mask in the same workspace
   if (w < nw) bits[w] = word;

@@ -80,9 +80,9 @@ struct FtCfg {
 struct FtParams {
   int64_t M, d, k;
   int32_t kpb;          // NF4 blocks per weight row
-  int32_t r, rp;
-  ScaleSrc sc;
-  const uint16_t* B;    // d x r
+  int32_t r, rp;         // r: the rank of one projection (B's row length); rp: T_s's row length
+  ScaleSrc sc;            // grouped weights: rows from sc.gstart[i] on belong to projection i + 1
+  const uint16_t* B;    // d x r (projections' rows stacked)
   const uint16_t* T;    // M x rp, T_s (written by the down kernel)
   uint16_t* Y;          // M x d
   float* partial;       // [G][segmax][NTOK][256]
@@ -418,8 +418,10 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
 #pragma unroll
         for (int e = 0; e < 4; ++e) v[t][e] += pv[u][t][e];
   }
-  // LoRA term: rows of B are the A operand, T_s^T the B operand.
+  // LoRA term: rows of B are the A operand, T_s^T the B operand.  The row
+  // block's projection g uses T_s columns [g r, (g + 1) r).
   const bool even = (p.r & 1) == 0;
+  const int toff = group_of(p.sc, static_cast<int64_t>(rb) * kFtRows) * p.r;
   auto bpair = [&](int64_t n, int j) -> uint32_t {
     if (n >= p.d || j >= p.r) return 0u;
     const uint16_t* src = p.B + n * p.r + j;
@@ -440,9 +442,10 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
         const int tok = 8 * t + g;
-        const uint16_t* trow = p.T + static_cast<int64_t>(tok) * p.rp;
-        bf[u][t][0] = (ok && tok < p.M) ? ld_pair(trow + j0) : 0u;
-        bf[u][t][1] = (ok && tok < p.M) ? ld_pair(trow + j0 + 8) : 0u;
+        const uint16_t* trow = p.T + static_cast<int64_t>(tok) * p.rp + toff;
+        // columns past this projection's r meet zero rows of B; keep the reads inside T_s
+        bf[u][t][0] = (ok && tok < p.M && toff + j0 + 1 < p.rp) ? ld_pair(trow + j0) : 0u;
+        bf[u][t][1] = (ok && tok < p.M && toff + j0 + 9 < p.rp) ? ld_pair(trow + j0 + 8) : 0u;
       }
     }
 #pragma unroll
@@ -535,7 +538,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   const uint32_t x_off = kFtCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
   const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
   float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
-  const float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;
+  float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;   // of the current row block's projection
 
   // ---- TMA issue of item j into stage sj: the code tile, the item's 256
   // columns of X and, at the first item of a group of four, the group's c2
@@ -569,6 +572,8 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   RowConst rw[2];
   auto set_rows = [&](int rbx) {
     const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
+    // a 256-row block lies in one projection of a grouped weight
+    if (dq && p.sc.ngrp > 1) mean = group_mean(p.sc, static_cast<int64_t>(rbx) * kFtRows);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       rw[h].valid = r0 + 8 * h < p.d;
@@ -865,9 +870,11 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   p.d = a.d;
   p.k = a.k;
   p.kpb = static_cast<int32_t>(a.k / 64);
-  p.r = a.r;
+  p.r = a.r_group > 0 ? a.r_group : a.r;
   p.rp = a.rp;
   p.sc.dq = a.q->double_quant;
+  p.sc.ngrp = a.ngrp;
+  for (int i = 0; i < 3; ++i) p.sc.gstart[i] = a.gstart[i];
   p.sc.absmax = a.q->absmax;
   p.sc.c2 = a.q->c2;
   p.sc.c1 = a.q->c1;

@@ -137,10 +137,11 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 // ============================================================================
 struct MainParams {
   int64_t M, d, k;
-  int32_t r, rp;
+  int32_t r, rp;            // adapter rank (all projections of a group together) and r padded to 64
+  int32_t r_group;          // rank of one projection (== r for a plain weight)
   int32_t kpb;              // NF4 blocks per weight row (k / 64)
   ScaleSrc sc;
-  const uint16_t* lora;     // forward: B (d x r); backward: A (r x k)
+  const uint16_t* lora;     // forward: B (d x r_group, projections stacked); backward: A (r x k)
   uint16_t* out;            // bf16 output (splits == 1)
   float* partial;           // fp32 [splits][M][n_out] (splits > 1)
   int64_t n_out;            // output columns: d (forward) or k (backward)
@@ -150,6 +151,28 @@ struct MainParams {
   int32_t splits;
   int32_t ncp;              // paired kernel: 256-column pairs across the output
 };
+
+// Forward LoRA extension steps of the output rows starting at `row0` (all in
+// one projection): T_s columns [g r_group, (g + 1) r_group) of projection g
+// meet that projection's rows of B, so only the 64-wide steps overlapping that
+// window are run.  A plain weight has g = 0 and runs steps [0, rp / 64).
+struct ExtWindow {
+  int e_lo, n;    // first extension step and their count
+  int g;          // projection
+};
+__device__ __forceinline__ ExtWindow ext_window(const MainParams& p, int64_t row0) {
+  ExtWindow w;
+  w.g = group_of(p.sc, row0);
+  const int lo = w.g * p.r_group, hi = lo + p.r_group;
+  w.e_lo = lo / 64;
+  w.n = (hi + 63) / 64 - w.e_lo;
+  return w;
+}
+// bf16 bits of B[n][j] for T_s column j (0 outside the row's projection window)
+__device__ __forceinline__ uint32_t ext_b(const MainParams& p, const ExtWindow& w, int64_t n, int64_t j) {
+  const int64_t jl = j - static_cast<int64_t>(w.g) * p.r_group;
+  return (n < p.d && jl >= 0 && jl < p.r_group) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r_group + jl)) : 0u;
+}
 
 // ============================================================================
 // Swapped forward (17..128 tokens): the weight rows are the MMA's M side (128
@@ -210,7 +233,8 @@ __global__ void __launch_bounds__(576, 1)
   const int s_begin = split * p.steps_per_split;
   const int s_end = min(p.steps_main, s_begin + p.steps_per_split);
   const int n_main = max(0, s_end - s_begin);
-  const int n_local = n_main + (split == 0 ? p.ext_steps : 0);
+  const ExtWindow xw = ext_window(p, n0);
+  const int n_local = n_main + (split == 0 ? xw.n : 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -258,7 +282,7 @@ __global__ void __launch_bounds__(576, 1)
           tma_load_2d(act_tile(st) + Cfg::kActAtomBytes, &tm_act, &full_bar[st], 128 * i + 64, 0);
           tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 64 * i, static_cast<int>(n0));
         } else {
-          const int e = l - n_main;
+          const int e = xw.e_lo + l - n_main;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActAtomBytes);
           tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, 0);
         }
@@ -314,7 +338,7 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
     for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
-    const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
+    const float mean = group_mean(sc, n0);   // the tile's 128 rows lie in one projection
     // row = W row (0..127), sub = which of the step's two blocks
     const int row = tg & 127;
     const int sub = tg >> 7;
@@ -381,19 +405,16 @@ __global__ void __launch_bounds__(576, 1)
           for (int c = 0; c < 8; ++c) sts128(wt + sw128_offset(row, c), make_uint4(0, 0, 0, 0));
         }
       } else if (sub == 0) {
-        // LoRA extension step (64 wide): B (d x r) row n, columns 64e + [0, 64)
+        // LoRA extension step (64 wide): B row n against T_s columns 64e + [0, 64)
         // into the first K atom
-        const int e = l - n_main;
+        const int e = xw.e_lo + l - n_main;
         const int64_t n = n0 + row;
         const uint32_t wt0 = smem_u32(w_tile(sw));
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint32_t h[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int64_t j = 64ll * e + 8 * c + q;
-            h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
-          }
+          for (int q = 0; q < 8; ++q) h[q] = ext_b(p, xw, n, 64ll * e + 8 * c + q);
           sts128(wt0 + sw128_offset(row, c),
                  make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
         }
@@ -604,7 +625,18 @@ __global__ void __launch_bounds__(576, 1)
   const int s_begin = split * p.steps_per_split;
   const int s_end = min(p.steps_main, s_begin + p.steps_per_split);
   const int n_main = max(0, s_end - s_begin);
-  const int n_local = n_main + (split == 0 ? p.ext_steps : 0);
+  // forward: the pair's 256 output rows lie in one projection (same window in
+  // both CTAs); backward: every projection's adapter term reaches every dX
+  // column, so all extension steps run
+  ExtWindow xw;
+  if (BWD) {
+    xw.g = 0;
+    xw.e_lo = 0;
+    xw.n = p.ext_steps;
+  } else {
+    xw = ext_window(p, n0);
+  }
+  const int n_local = n_main + (split == 0 ? xw.n : 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -657,7 +689,7 @@ __global__ void __launch_bounds__(576, 1)
           else
             tma_load_2d(code_tile(st), &tm_codes, &full_bar[st], 32 * i, static_cast<int>(h0));
         } else {
-          const int e = l - n_main;
+          const int e = xw.e_lo + l - n_main;
           mbar_arrive_expect_tx(&full_bar[st], Cfg::kActBytes);
           tma_load_2d(act_tile(st), &tm_ext, &full_bar[st], 64 * e, static_cast<int>(m0));
         }
@@ -714,7 +746,10 @@ __global__ void __launch_bounds__(576, 1)
 #pragma unroll
     for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
     const ScaleSrc sc = p.sc;
-    const float mean = sc.dq ? __ldg(sc.mean) : 0.0f;
+    // forward: the CTA's 128 weight rows lie in one projection; backward: a K
+    // step's 64 weight rows do (the mean is re-read per step for a grouped weight)
+    const float mean = group_mean(sc, BWD ? 64ll * s_begin : h0);
+    const bool step_mean = BWD && sc.ngrp > 1;
     //   Fwd: row = W row of this CTA's half (0..127)
     //   Bwd: row = W row within the 64-row K step, sub = 64-column chunk of this CTA's half
     const int row = BWD ? (tg & 63) : tg;
@@ -778,7 +813,8 @@ __global__ void __launch_bounds__(576, 1)
           w8[4 * h + 3] = cw.w;
         }
         if (cur_valid) {
-          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur, recip), C);
+          const float mean_l = step_mean ? group_mean(sc, 64ll * (s_begin + l)) : mean;
+          const Nf4Tab tab = make_tab(scale_value(sc.dq, mean_l, cur, recip), C);
 #pragma unroll
           for (int c = 0; c < CPT; ++c) sts128(wt + sw128_offset(row, c_first + c), dq8(w8[c], tab));
         } else {
@@ -787,7 +823,7 @@ __global__ void __launch_bounds__(576, 1)
         }
       } else {
         // LoRA extension step (64 wide): this CTA's half of the adapter into the W tile
-        const int e = l - n_main;
+        const int e = xw.e_lo + l - n_main;
         if (BWD) {
           // A (r x k): K row j = 64e + row, N columns h0 + 64 sub + [0, 64)
           const int64_t j = 64ll * e + row;
@@ -801,16 +837,13 @@ __global__ void __launch_bounds__(576, 1)
             sts128(wt + sw128_offset(row, c), val);
           }
         } else {
-          // B (d x r): row n, columns 64e + [0, 64)
+          // B row n against T_s columns 64e + [0, 64)
           const int64_t n = h0 + row;
 #pragma unroll
           for (int c = c_first; c < c_first + CPT; ++c) {
             uint32_t h[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int64_t j = 64ll * e + 8 * c + q;
-              h[q] = (n < p.d && j < p.r) ? static_cast<uint32_t>(__ldg(p.lora + n * p.r + j)) : 0u;
-            }
+            for (int q = 0; q < 8; ++q) h[q] = ext_b(p, xw, n, 64ll * e + 8 * c + q);
             sts128(wt + sw128_offset(row, c),
                    make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
           }
@@ -921,6 +954,12 @@ struct ThinParams {
   const uint32_t* keep;
   int64_t keep_rows;     // M
   int64_t keep_ld;       // k
+  // THIN_DB of a grouped weight: output rows from gstart[i] on belong to
+  // projection i + 1, whose dB takes columns [g r_group, (g + 1) r_group) of
+  // the tile (a plain weight: ngrp <= 1, r_group = r)
+  int32_t ngrp;
+  int32_t r_group;
+  int64_t gstart[3];
 };
 
 // Zero the dropped elements of one 128-byte row (64 bf16) of a tile stored
@@ -1175,14 +1214,18 @@ __global__ void __launch_bounds__(128, 2)
         *reinterpret_cast<uint2*>(p.out16 + row * rp + j0) = o;
       } else {
         const float e[4] = {acc.x * p.scale, acc.y * p.scale, acc.z * p.scale, acc.w * p.scale};
+        if (p.mode == THIN_DA) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (j0 + u < p.r) {
-            if (p.mode == THIN_DA)
-              p.outf[static_cast<int64_t>(j0 + u) * p.ld + row] = e[u];
-            else
-              p.outf[row * p.r + j0 + u] = e[u];
-          }
+          for (int u = 0; u < 4; ++u)
+            if (j0 + u < p.r) p.outf[static_cast<int64_t>(j0 + u) * p.ld + row] = e[u];
+        } else {
+          int g = 0;   // projection of this output row (128-row tiles never straddle two)
+#pragma unroll
+          for (int jg = 0; jg < 3; ++jg) g += (jg + 1 < p.ngrp && row0 >= p.gstart[jg]) ? 1 : 0;
+          const int lo = g * p.r_group;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (j0 + u >= lo && j0 + u < lo + p.r_group) p.outf[row * p.r_group + (j0 + u - lo)] = e[u];
         }
       }
     }
@@ -1222,6 +1265,33 @@ __global__ void k_reduce_bf16(const float* __restrict__ partial, int splits, int
 }
 
 // Bt[j][n] = B[n][j] for j < r, 0 for r <= j < rp
+// B' (d x r, bf16) block diagonal from the stacked B (d x r_group): row n of
+// projection g holds its B row in columns [g r_group, (g + 1) r_group), zeros
+// elsewhere.  Eight columns per thread (r % 8 == 0 for grouped weights).
+struct BlockDiag {
+  int64_t d;
+  int32_t r_group, r, ngrp;
+  int64_t gstart[3];
+};
+__global__ void k_blockdiag_B(const uint16_t* __restrict__ B, const BlockDiag bd, uint16_t* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();   // a previous call's kernels may still read the workspace
+  const int64_t n8 = bd.d * bd.r / 8;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = (8 * i) / bd.r;
+    const int j0 = static_cast<int>(8 * i - n * bd.r);
+    int g = 0;
+#pragma unroll
+    for (int jg = 0; jg < 3; ++jg) g += (jg + 1 < bd.ngrp && n >= bd.gstart[jg]) ? 1 : 0;
+    const int lo = g * bd.r_group;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (j0 >= lo && j0 < lo + bd.r_group)   // r_group % 8 == 0: the 8 columns lie in the window together
+      v = __ldg(reinterpret_cast<const uint4*>(B + n * bd.r_group + (j0 - lo)));
+    *reinterpret_cast<uint4*>(out + 8 * i) = v;
+  }
+}
+
 __global__ void k_transpose_B(const uint16_t* __restrict__ B, int64_t d, int r, int rp, uint16_t* __restrict__ Bt) {
   __shared__ uint16_t tile[32][34];
   griddep_launch_dependents();
@@ -1495,15 +1565,19 @@ static int launch_pair(const CUtensorMap& ta, const CUtensorMap& tc, const CUten
   return 0;
 }
 
-static ScaleSrc scale_src(const qlora_nf4_t& q) {
+static ScaleSrc scale_src(const qlora_nf4_t& q, const LinearArgs& a) {
   ScaleSrc s{};
   s.dq = q.double_quant;
   s.absmax = q.absmax;
   s.c2 = q.c2;
   s.c1 = q.c1;
   s.mean = q.mean;
+  s.ngrp = a.ngrp;
+  for (int i = 0; i < 3; ++i) s.gstart[i] = a.gstart[i];
   return s;
 }
+
+static int32_t rank_group(const LinearArgs& a) { return a.r_group > 0 ? a.r_group : a.r; }
 
 // Adapter dropout: the keep bitmask of X in the workspace (nullptr without
 // dropout), generated for this call from (seed, offset).
@@ -1548,7 +1622,8 @@ int launch_linear_fwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   MainParams mp{};
   mp.M = M; mp.d = d; mp.k = k; mp.r = a.r; mp.rp = rp;
   mp.kpb = static_cast<int32_t>(k / 64);
-  mp.sc = scale_src(q);
+  mp.sc = scale_src(q, a);
+  mp.r_group = rank_group(a);
   mp.lora = a.B;
   mp.n_out = d;
   mp.steps_main = static_cast<int32_t>(pl.nt ? ceil_div(k, 128) : k / 64);   // the swapped kernel steps 128 wide
@@ -1613,7 +1688,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   int rc;
   if (M == 0) {
     cudaMemsetAsync(a.dA, 0, static_cast<size_t>(r) * k * 4, st);
-    cudaMemsetAsync(a.dB, 0, static_cast<size_t>(d) * r * 4, st);
+    cudaMemsetAsync(a.dB, 0, static_cast<size_t>(d) * rank_group(a) * 4, st);
     return 0;
   }
   // adapter dropout: the same keep decisions as the forward, regenerated
@@ -1633,7 +1708,24 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
   // its row-major storage when its rows are 16-byte multiples; otherwise a
   // K-major copy B^T (rp x d) is made first.
   uint16_t* U = reinterpret_cast<uint16_t*>(ws + pl.off_U);
-  if (r % 8 == 0) {
+  if (a.ngrp > 1) {
+    // grouped: U_s = s dY B' with B' (d x r) block diagonal, projection i's B
+    // in columns [i r_group, (i + 1) r_group); one pass over dY for all
+    uint16_t* Bd = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
+    BlockDiag bd{};
+    bd.d = d;
+    bd.r_group = rank_group(a);
+    bd.r = r;
+    bd.ngrp = a.ngrp;
+    for (int i = 0; i < 3; ++i) bd.gstart[i] = a.gstart[i];
+    {
+      ProfScope ps_(QLORA_KC_AUX, st);
+      (void)launch_pdl(k_blockdiag_B, dim3(static_cast<unsigned>(grid1d(d * r / 8, 256))), dim3(256), 0, st, nullptr,
+                       a.B, bd, Bd);
+    }
+    QL_CHECK_LAUNCH("block-diagonal B launch");
+    rc = run_lowrank_down(a.dY, M, d, Bd, r, true, rp, a.s, pl.splits_U, U, st, why);
+  } else if (r % 8 == 0) {
     rc = run_lowrank_down(a.dY, M, d, a.B, r, true, rp, a.s, pl.splits_U, U, st, why);
   } else {
     uint16_t* Bt = reinterpret_cast<uint16_t*>(ws + pl.off_Bt);
@@ -1652,7 +1744,8 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     MainParams mp{};
     mp.M = M; mp.d = d; mp.k = k; mp.r = r; mp.rp = rp;
     mp.kpb = static_cast<int32_t>(k / 64);
-    mp.sc = scale_src(q);
+    mp.sc = scale_src(q, a);
+    mp.r_group = rank_group(a);
     mp.lora = a.A;
     mp.n_out = k;
     mp.steps_main = static_cast<int32_t>(ceil_div(d, 64));
@@ -1726,6 +1819,9 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why) {
     tp.r = r;
     tp.outf = a.dB;
     tp.scale = 1.0f;
+    tp.ngrp = a.ngrp;
+    tp.r_group = rank_group(a);
+    for (int i = 0; i < 3; ++i) tp.gstart[i] = a.gstart[i];
     rc = launch_thin<true, true>(ta, tb, tp, ceil_div(d, 128), pl.splits_dB, st, why);
     if (rc) return rc;
   }

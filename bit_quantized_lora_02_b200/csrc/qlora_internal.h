@@ -68,6 +68,14 @@ struct LinearArgs {
   // adapter dropout (drop == nullptr: none).  The keep bitmask lives in the
   // workspace past the plain layer's part, at dropout_mask_offset().
   const DropoutArgs* drop;
+  // Grouped projections sharing X: q stacks ngrp projections (rows from
+  // gstart[i] on belong to projection i + 1, each with its own mean); r is the
+  // rank of all of them together (A, T_s, U_s, dA stack the projections'
+  // ranks), r_group the rank of one; B and dB are (d x r_group) with the
+  // projections' rows stacked.  A plain layer has ngrp = 0 and r_group = r.
+  int32_t r_group;
+  int32_t ngrp;
+  int64_t gstart[3];
 };
 
 size_t fwd_workspace_bytes(int64_t M, int64_t d, int64_t k, int32_t r);

@@ -98,6 +98,11 @@ WORKLOADS = {
     "decode_28672x8192": dict(proj=[("up", 28672, 8192), ("down", 8192, 28672)], m=(1, 8, 32, 128),
                               r=16, alpha=32.0, a_std=None, bwd=False),
     "llama65b_block_m8192": dict(proj=PROJ_65B, m=8192, r=64, alpha=16.0, a_std=None, bwd=True),
+    # the same sets with q, k, v and gate, up grouped: each group reads one X
+    "llama7b_proj_set_m4096_grouped": dict(proj=PROJ_7B, m=4096, r=64, alpha=16.0, a_std=None, bwd=True,
+                                           groups=[[0, 1, 2], [3], [4, 5], [6]]),
+    "llama65b_block_m8192_grouped": dict(proj=PROJ_65B, m=8192, r=64, alpha=16.0, a_std=None, bwd=True,
+                                         groups=[[0, 1, 2], [3], [4, 5], [6]]),
     # the same sets with adapter dropout p = 0.05 (the lora_dropout of the PEFT configuration)
     "llama7b_proj_set_m4096_dropout": dict(proj=PROJ_7B, m=4096, r=64, alpha=16.0, a_std=None, bwd=True,
                                            dropout=0.05),

@@ -216,6 +216,52 @@ int qlora_linear_bwd(const uint16_t *dY, const uint16_t *X, int64_t M, const qlo
                      const uint16_t *T_save, uint16_t *dX, float *dA, float *dB,
                      void *workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* Grouped projections ("LoRA and QLoRA: Efficient Fine-Tuning of Large
+ * Language Models" (fromzero2ai.dev), "4. Define LoRA Target Modules and
+ * Config": q_proj, k_proj, v_proj and o_proj carry adapters; q, k and v read
+ * the same input, as gate and up do in the MLP).  Projections that share X
+ * run as one layer over their stacked rows, so X is read once per pass
+ * instead of once per projection:
+ *     Y_i = X W_i^T + s (X A_i^T) B_i^T,   i = 0 .. n-1,
+ * each W_i quantised on its own (own blocks, groups and mean; bit for bit what
+ * nf4_quantize gives for W_i alone), each with its own adapter of rank r.
+ *
+ * Layout (all row-major, projections in order i = 0 .. n-1):
+ *   w      : the stacked weight, w.d = d[0] + ... + d[n-1]; codes, c2 (or
+ *            absmax) and c1 hold the projections' buffers back to back (quantise
+ *            W_i with nf4_quantize into its slice: codes + (rows before i) * k / 2,
+ *            c2 + (rows before i) * k / 64, c1 + (rows before i) * k / 16384);
+ *            w.mean points to n means, one per projection.
+ *   A      : (n r) x k, the A_i stacked.        B : w.d x r, the B_i stacked.
+ *   Y, dY  : M x w.d, Y_i in columns [rows before i, + d[i]).
+ *   T_save : M x qlora_rank_pad(n r), T_i = BF16(s X A_i^T) in columns [i r, (i+1) r).
+ *   dA     : (n r) x k (fp32), the dA_i stacked.   dB : w.d x r (fp32), the dB_i stacked.
+ *   dX     : M x k, the sum over the projections.
+ * Requirements: 1 <= n <= 4; d[i] a multiple of 256 for i < n - 1; n r <= 256;
+ * r % 8 == 0 when n > 1; otherwise as for qlora_linear_fwd / _bwd. */
+#define QLORA_MAX_GROUP 4
+typedef struct {
+  int32_t n;                   /* projections sharing the input, 1..4 */
+  int64_t d[QLORA_MAX_GROUP];  /* output rows of each                 */
+  qlora_nf4_t w;               /* the stacked weight                  */
+} qlora_nf4_group_t;
+
+/* Workspace bytes of the grouped forward (backward == 0) or backward. */
+int qlora_grouped_workspace_size(int64_t M, const qlora_nf4_group_t *g, int32_t r, int32_t backward,
+                                 size_t *bytes);
+
+/* Forward of n projections sharing X (layout above); s = RN32(alpha / r). */
+int qlora_linear_fwd_grouped(const uint16_t *X, int64_t M, const qlora_nf4_group_t *g, const uint16_t *A,
+                             const uint16_t *B, int32_t r, float alpha, uint16_t *Y, uint16_t *T_save,
+                             void *workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/* Backward of the grouped forward: dX = sum_i (dY_i W_i + s (dY_i B_i) A_i),
+ * dA_i = s (dY_i B_i)^T X, dB_i = s dY_i^T (X A_i^T). */
+int qlora_linear_bwd_grouped(const uint16_t *dY, const uint16_t *X, int64_t M, const qlora_nf4_group_t *g,
+                             const uint16_t *A, const uint16_t *B, int32_t r, float alpha, const uint16_t *T_save,
+                             uint16_t *dX, float *dA, float *dB, void *workspace, size_t workspace_bytes,
+                             qlora_stream_t stream);
+
 /* Adapter dropout ("LoRA and QLoRA: Efficient Fine-Tuning of Large Language
  * Models" (fromzero2ai.dev), "Python Implementation: Fine-Tuning with PEFT and
  * BitsAndBytes", step 4: lora_dropout = 0.05).  Dropout acts on the adapter's

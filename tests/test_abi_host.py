@@ -173,3 +173,54 @@ def test_selftest_validation_without_gpu(L):
     assert L.qlora_selftest_wait_timeout(1000001, 0x10000, None) == -1
     assert L.qlora_selftest_wait_timeout(100, None, None) == -1
     assert L.qlora_selftest_wait_timeout(100, 0x10002, None) == -3
+
+
+def test_grouped_validation_without_gpu(L):
+    """Grouped projections: 1..4 projections, all but the last a multiple of
+    256 rows summing to the stacked weight, n r <= 256 and r % 8 == 0; the
+    workspace equals the plain layer's for the stacked rows and ranks."""
+    def group(ds, k=512, total=None):
+        g = Q.QloraNF4Group()
+        g.n = len(ds)
+        for i, x in enumerate(ds):
+            g.d[i] = x
+        g.w = Q.QloraNF4(sum(ds) if total is None else total, k, 64, 1, 0x1000, None, 0x2000, 0x3000, 0x4000)
+        return g
+    n, n1 = ctypes.c_size_t(), ctypes.c_size_t()
+    g = group([256, 256, 520])
+    for bwd in (0, 1):
+        assert L.qlora_grouped_workspace_size(300, ctypes.byref(g), 16, bwd, ctypes.byref(n)) == 0
+        assert L.qlora_linear_workspace_size(300, 1032, 512, 48, bwd, ctypes.byref(n1)) == 0
+        assert n.value == n1.value
+    assert L.qlora_grouped_workspace_size(300, ctypes.byref(group([200, 256])), 16, 0, ctypes.byref(n)) == -2
+    assert L.qlora_grouped_workspace_size(300, ctypes.byref(group([256, 256], total=768)), 16, 0,
+                                          ctypes.byref(n)) == -1
+    assert L.qlora_grouped_workspace_size(300, ctypes.byref(group([256, 256, 256])), 96, 0, ctypes.byref(n)) == -2
+    assert L.qlora_grouped_workspace_size(300, ctypes.byref(group([256, 256])), 12, 0, ctypes.byref(n)) == -2
+    assert L.qlora_grouped_workspace_size(300, ctypes.byref(group([])), 16, 0, ctypes.byref(n)) == -1
+    assert L.qlora_grouped_workspace_size(300, None, 16, 0, ctypes.byref(n)) == -1
+    g = group([256, 256])
+    rc = L.qlora_linear_fwd_grouped(0x10000, 300, ctypes.byref(g), 0x10000, 0x20000, 16, 16.0, 0x30000, None, None,
+                                    0, None)
+    assert rc == -4                                   # workspace missing, before any device work
+    rc = L.qlora_linear_bwd_grouped(0x10000, 0x10000, 300, ctypes.byref(g), 0x10000, 0x20000, 16, 16.0, None,
+                                    None, 0x30000, 0x40000, None, 0, None)
+    assert rc == -4
+
+
+def test_group_buffers_are_slices_of_the_stack():
+    """The binding's stacked allocation: slice i starts where the earlier
+    projections' buffers end (codes, c2, c1) and holds projection i's mean."""
+    import torch
+    ds, k = (256, 512, 264), 1024
+    sizes = [Q.qlora_nf4_sizes(d, k, 64, 1)[0] for d in ds]
+    codes = torch.zeros(sum(s[0] for s in sizes) + 16, dtype=torch.uint8)
+    off = 0
+    for d, s in zip(ds, sizes):
+        assert s[0] == d * k // 2 and s[2] == d * k // 64
+        off += s[0]
+    assert off == sum(ds) * k // 2
+    assert all(s[3] == d * k // 64 // 256 * 4 for d, s in zip(ds[:-1], sizes[:-1]))
+    st = Q.qlora_nf4_sizes(sum(ds), k, 64, 1)[0]
+    assert st[0] == off and st[2] == sum(s[2] for s in sizes) and st[3] == sum(s[3] for s in sizes)
+    del codes
