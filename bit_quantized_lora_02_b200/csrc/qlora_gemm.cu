@@ -1365,23 +1365,16 @@ struct Plan {
   size_t off_T, off_Bt, off_U, off_main, total;
 };
 
-// Few-token forward: the kernel streams weights, so keep every SM busy until
-// the end.  Choose the K split (1..8) with the best wave efficiency; a larger
-// split must win by 5% (its partial sums cost an extra pass).
+// Swapped forward (17..128 tokens): split K only as far as one wave of CTAs
+// (one per SM) is filled.  Each CTA pays a fixed set-up and drain per launch
+// and a split adds an fp32 partial pass, so a second, partly empty wave of
+// whole-K CTAs beats many short split CTAs: on 28672 x 8192 at M = 32, one
+// split (224 CTAs in two waves) took 128 us against 148 us for seven.
 static int plan_swap_splits(int64_t tiles, int steps) {
-  int best = 1;
-  double best_eff = 0.0;
-  for (int s = 1; s <= 8; ++s) {
-    if (steps / s < 4) break;
-    const int64_t ctas = tiles * s;
-    const int64_t waves = ceil_div(ctas, kSms);
-    const double eff = static_cast<double>(ctas) / static_cast<double>(waves * kSms);
-    if (eff > best_eff + 0.05) {
-      best_eff = eff;
-      best = s;
-    }
-  }
-  return best;
+  int s = static_cast<int>(tiles >= kSms ? 1 : kSms / tiles);
+  if (s > 8) s = 8;
+  while (s > 1 && steps / s < 4) --s;
+  return s < 1 ? 1 : s;
 }
 
 static int swap_nt(int64_t M) {
