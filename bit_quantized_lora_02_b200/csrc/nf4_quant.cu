@@ -29,6 +29,7 @@
 
 #include <cuda_fp8.h>
 
+#include "nf4_scale.cuh"
 #include "nf4_table.h"
 #include "qlora_device.cuh"
 #include "qlora_internal.h"
@@ -450,58 +451,68 @@ __global__ void __launch_bounds__(256) k_dq_groups(const uint16_t* __restrict__ 
 
 // ----------------------------------------------------------------------------
 // Standalone double dequantisation: W_out[i] = BF16(RN32(C[q_i] * s^_j)).
+//
+// One thread per 64-weight block: its 32 code bytes are loaded first (two
+// 16-byte loads when the codes are 16-byte aligned, else eight 4-byte loads),
+// so every thread keeps 32 bytes in flight; s^ is computed once per block;
+// the block's 16 values T[j] = BF16(RN32(C[j] * s^)) are built in registers
+// and each 4-bit code is resolved with byte permutes (the GEMMs' expansion,
+// bit-identical to the per-weight formula); the block's 128 bytes go out as
+// eight 16-byte stores.  A ragged last block (N % 64 != 0) is expanded element
+// by element.
 // ----------------------------------------------------------------------------
 // kDQ: 0 = fp32 absmax per block, 1 = Int8 c2, 2 = E4M3 c2.
 template <int kDQ>
-__global__ void __launch_bounds__(256) k_nf4_dequant(const uint8_t* __restrict__ codes, int64_t N,
+__device__ __forceinline__ float dequant_scale(int64_t blk, const float* __restrict__ absmax,
+                                               const int8_t* __restrict__ c2, const float* __restrict__ c1, float mu) {
+  if (kDQ == 1) return __fadd_rn(__fdiv_rn(static_cast<float>(__ldg(c2 + blk)), __ldg(c1 + (blk >> 8))), mu);
+  if (kDQ == 2) {
+    const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(__ldg(c2 + blk)), __NV_E4M3);
+    return __fadd_rn(__fdiv_rn(__half2float(__half(hr)), __ldg(c1 + (blk >> 8))), mu);   // E4M3 -> fp32 is exact
+  }
+  return __ldg(absmax + blk);
+}
+
+template <int kDQ, bool kVec16>
+__global__ void __launch_bounds__(256, 4) k_nf4_dequant(const uint8_t* __restrict__ codes, int64_t N,
                                                      const float* __restrict__ absmax, const int8_t* __restrict__ c2,
                                                      const float* __restrict__ c1, const float* __restrict__ mean,
                                                      uint16_t* __restrict__ out) {
-  __shared__ float s_C[16];
   constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
-  if (threadIdx.x == 0) {
+  float C[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) s_C[j] = __uint_as_float(kCB[j]);
-  }
-  __syncthreads();
+  for (int j = 0; j < 16; ++j) C[j] = __uint_as_float(kCB[j]);
   griddep_launch_dependents();
   griddep_wait();
-  const float mu = kDQ ? *mean : 0.0f;
-  const int64_t ngroups = (N + 7) >> 3;
+  const float mu = kDQ ? __ldg(mean) : 0.0f;
+  const int64_t nfull = N >> 6;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups; g += stride) {
-    const int64_t e0 = g << 3;
-    const int64_t blk = e0 >> 6;
-    float sh;
-    if (kDQ == 1) {
-      sh = __fadd_rn(__fdiv_rn(static_cast<float>(c2[blk]), c1[blk >> 8]), mu);
-    } else if (kDQ == 2) {
-      const __half_raw hr = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(c2[blk]), __NV_E4M3);
-      sh = __fadd_rn(__fdiv_rn(__half2float(__half(hr)), c1[blk >> 8]), mu);   // E4M3 -> fp32 is exact
+  for (int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; blk < nfull; blk += stride) {
+    const uint8_t* src = codes + (blk << 5);
+    uint32_t cw[8];
+    if (kVec16) {
+      const uint4 a = ldg_nc_v4(src), b = ldg_nc_v4(src + 16);
+      cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+      cw[4] = b.x; cw[5] = b.y; cw[6] = b.z; cw[7] = b.w;
     } else {
-      sh = absmax[blk];
-    }
-    const bool full = (e0 + 8 <= N);
-    uint32_t cw;
-    if (full) {
-      cw = __ldg(reinterpret_cast<const unsigned int*>(codes + (e0 >> 1)));
-    } else {
-      cw = 0;
-      const int nbytes = static_cast<int>((N - e0 + 1) >> 1);
-      for (int b = 0; b < nbytes; ++b) cw |= static_cast<uint32_t>(codes[(e0 >> 1) + b]) << (8 * b);
-    }
-    uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float a = __fmul_rn(s_C[(cw >> (8 * i)) & 15u], sh);
-      const float b = __fmul_rn(s_C[(cw >> (8 * i + 4)) & 15u], sh);
-      o[i] = pack_bf16x2(a, b);
+      for (int i = 0; i < 8; ++i) cw[i] = __ldg(reinterpret_cast<const unsigned int*>(src) + i);
     }
-    if (full) {
-      *reinterpret_cast<uint4*>(out + e0) = make_uint4(o[0], o[1], o[2], o[3]);
-    } else {
-      for (int i = 0; e0 + i < N; ++i) out[e0 + i] = static_cast<uint16_t>(o[i >> 1] >> (16 * (i & 1)));
-    }
+    const Nf4Tab tab = make_tab(dequant_scale<kDQ>(blk, absmax, c2, c1, mu), C);
+    uint4* dst = reinterpret_cast<uint4*>(out + (blk << 6));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = dq8(cw[i], tab);
+  }
+  // ragged last block: the elements past 64 * nfull, eight per thread of CTA 0
+  const int64_t e0 = (nfull << 6) + 8 * static_cast<int64_t>(threadIdx.x);
+  if (blockIdx.x == 0 && threadIdx.x < 8 && e0 < N) {
+    const Nf4Tab tab = make_tab(dequant_scale<kDQ>(nfull, absmax, c2, c1, mu), C);
+    uint32_t cw = 0;
+    for (int64_t b = e0 >> 1; b < ((N + 1) >> 1) && b < (e0 >> 1) + 4; ++b)
+      cw |= static_cast<uint32_t>(codes[b]) << (8 * (b - (e0 >> 1)));
+    const uint4 v = dq8(cw, tab);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 8 && e0 + i < N; ++i) out[e0 + i] = static_cast<uint16_t>(w[i >> 1] >> (16 * (i & 1)));
   }
 }
 
@@ -565,19 +576,25 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t N, const qlora_nf4_t& q, 
   return cudaGetLastError();
 }
 
+template <int kDQ>
+static cudaError_t launch_dequant_mode(const qlora_nf4_t& q, int64_t N, uint16_t* out, int grid, cudaStream_t st) {
+  const float* absmax = kDQ ? nullptr : q.absmax;
+  const int8_t* c2 = kDQ ? q.c2 : nullptr;
+  const float* c1 = kDQ ? q.c1 : nullptr;
+  const float* mean = kDQ ? q.mean : nullptr;
+  const bool vec16 = (reinterpret_cast<uintptr_t>(q.codes) & 15u) == 0;
+  return vec16 ? launch_pdl(k_nf4_dequant<kDQ, true>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, absmax, c2,
+                            c1, mean, out)
+               : launch_pdl(k_nf4_dequant<kDQ, false>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, absmax, c2,
+                            c1, mean, out);
+}
+
 cudaError_t launch_dequantize(const qlora_nf4_t& q, int64_t N, uint16_t* out, cudaStream_t st) {
-  const int grid = grid_for((N + 7) / 8);
+  const int grid = grid_for(N >> 6 > 0 ? N >> 6 : 1);   // one thread per complete 64-weight block
   ProfScope ps_(QLORA_KC_DEQUANT, st);
-  const cudaError_t e =
-      q.double_quant == 2
-          ? launch_pdl(k_nf4_dequant<2>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
-                       static_cast<const float*>(nullptr), q.c2, q.c1, q.mean, out)
-      : q.double_quant
-          ? launch_pdl(k_nf4_dequant<1>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N,
-                       static_cast<const float*>(nullptr), q.c2, q.c1, q.mean, out)
-          : launch_pdl(k_nf4_dequant<0>, dim3(grid), dim3(256), 0, st, nullptr, q.codes, N, q.absmax,
-                       static_cast<const int8_t*>(nullptr), static_cast<const float*>(nullptr),
-                       static_cast<const float*>(nullptr), out);
+  const cudaError_t e = q.double_quant == 2 ? launch_dequant_mode<2>(q, N, out, grid, st)
+                        : q.double_quant    ? launch_dequant_mode<1>(q, N, out, grid, st)
+                                            : launch_dequant_mode<0>(q, N, out, grid, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
