@@ -700,7 +700,46 @@ __global__ void __launch_bounds__(kFtThreads, 1)
         sm1 = bv && rw[1].valid ? cur_ab1 : 0.0f;
       }
     }
-    // four independent accumulation chains (one per 16-row group)
+    if constexpr (TG == 2) {
+      // 16 tokens: the two token groups give each row group two independent
+      // chains, so the row groups go one after another and only one row
+      // group's partial sums are live (no register spills at 128 registers)
+#pragma unroll
+      for (int rg = 0; rg < 4; ++rg) {
+        float tmq[TG][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
+          const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
+          const uint32_t w0 = (j < 2) ? cw[rg][0].x : cw[rg][0].y;
+          const uint32_t w1 = (j < 2) ? cw[rg][1].x : cw[rg][1].y;
+          const uint32_t a0 = lds32_const(prmt(w0, lanebase, sa));
+          const uint32_t a2 = lds32_const(prmt(w0, lanebase, sb));
+          const uint32_t a1 = lds32_const(prmt(w1, lanebase, sa));
+          const uint32_t a3 = lds32_const(prmt(w1, lanebase, sb));
+#pragma unroll
+          for (int t = 0; t < TG; ++t) {
+            const uint4 xq = xv[t][j >> 1];
+            const uint32_t b0 = (j & 1) ? xq.z : xq.x;
+            const uint32_t b1 = (j & 1) ? xq.w : xq.y;
+            if (j == 0)
+              mma16816_first(tmq[t], a0, a1, a2, a3, b0, b1);
+            else
+              mma16816(tmq[t], a0, a1, a2, a3, b0, b1);
+          }
+        }
+        const float s0 = __shfl_sync(0xffffffffu, sm0, 4 * g + rg);
+        const float s1 = __shfl_sync(0xffffffffu, sm1, 4 * g + rg);
+#pragma unroll
+        for (int t = 0; t < TG; ++t) {
+          acc[rg][t][0] = fmaf(tmq[t][0], s0, acc[rg][t][0]);
+          acc[rg][t][1] = fmaf(tmq[t][1], s0, acc[rg][t][1]);
+          acc[rg][t][2] = fmaf(tmq[t][2], s1, acc[rg][t][2]);
+          acc[rg][t][3] = fmaf(tmq[t][3], s1, acc[rg][t][3]);
+        }
+      }
+    } else {
+    // 8 tokens: four independent accumulation chains (one per 16-row group)
     float tmp[4][TG][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -740,6 +779,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
         acc[rg][t][2] = fmaf(tmp[rg][t][2], s1, acc[rg][t][2]);
         acc[rg][t][3] = fmaf(tmp[rg][t][3], s1, acc[rg][t][3]);
       }
+    }
     }
     // leaving the row block (the next item starts another one, or the range ends)
     if (++kc == p.KC || i + 1 == n_items) {
