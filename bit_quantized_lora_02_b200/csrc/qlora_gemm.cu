@@ -185,19 +185,26 @@ struct SwapCfg {
   static constexpr int kWRows = 128;                                   // W rows per K step
   static constexpr uint32_t kActAtomBytes = NT * 128;                  // one 64-wide K atom of the activations
   static constexpr uint32_t kActBytes = kActAtomBytes * (kStepK / 64);
-  static constexpr uint32_t kWBytes = kWRows * kStepK * 2;
   static constexpr uint32_t kCodeBytes = kWRows * kStepK / 2;
-  // Two rings: TMA stages (activations + packed codes, small) and dequantized
-  // W-tile buffers (large, written by the dequant warps).  Decoupling them lets
-  // many more code tiles be in flight than W tiles.
+  // Two rings: TMA stages in shared memory (activations + packed codes) and
+  // dequantized W tiles in tensor memory, written by the dequant warps with
+  // tcgen05.st and read by the MMA as its A operand, so the expanded weights
+  // never pass through shared memory (with few tokens the shared-memory
+  // round trip of every weight was the limit).
   static constexpr uint32_t kStageBytes = kActBytes + kCodeBytes;     // one TMA stage
-  static constexpr int kWBufs = 3;   // W tiles being written or waiting + one the MMAs read
-  static constexpr int kStagesRaw = static_cast<int>((218u * 1024u - kWBufs * kWBytes) / kStageBytes);
+  static constexpr int kWBufs = 4;   // W tiles being written or waiting + one the MMAs read
+  static constexpr int kStagesRaw = static_cast<int>((200u * 1024u) / kStageBytes);
   static constexpr int kStages = kStagesRaw > 12 ? 12 : kStagesRaw;
-  static constexpr uint32_t kTmemCols = NT <= 32 ? 32u : (NT <= 64 ? 64u : 128u);
-  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + kWBufs * kWBytes + 1024 /*align*/ + 512 /*barriers*/;
+  // TMEM: the fp32 accumulator in columns [0, 128), W tile sw (128 rows x 128
+  // K, two bf16 per 32-bit column) in columns [128 + 64 sw, 192 + 64 sw)
+  static constexpr uint32_t kAccCols = 128;
+  static constexpr uint32_t kWCols = kStepK / 2;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kAccCols + kWBufs * kWCols <= kTmemCols, "TMEM holds the accumulator and the W ring");
+  static constexpr uint32_t kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*barriers*/;
   // two groups of 8 dequant warps take alternate steps; every thread expands
-  // one whole block (the dequant rate is what matters with few tokens)
+  // one whole block into its TMEM lane (the dequant rate is what matters with
+  // few tokens)
   static constexpr int kGroups = 2;
   static constexpr int kGroupThreads = 256;
   static constexpr int kThreads = 64 + kGroups * kGroupThreads;
@@ -215,8 +222,7 @@ __global__ void __launch_bounds__(576, 1)
   const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_addr - raw_addr);
   constexpr int SW = Cfg::kWBufs;
-  uint8_t* wbase = base + S * Cfg::kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(wbase + SW * Cfg::kWBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + S * Cfg::kStageBytes);
   uint64_t* full_bar = bars;                // TMA data landed (act + codes)
   uint64_t* empty_bar = bars + S;           // MMAs reading the TMA stage completed
   uint64_t* wready_bar = bars + 2 * S;      // a dequant group filled the W buffer
@@ -265,7 +271,7 @@ __global__ void __launch_bounds__(576, 1)
 
   auto act_tile = [&](int st) { return base + st * Cfg::kStageBytes; };
   auto code_tile = [&](int st) { return base + st * Cfg::kStageBytes + Cfg::kActBytes; };
-  auto w_tile = [&](int sw) { return wbase + sw * Cfg::kWBytes; };
+  auto w_col = [&](int sw) { return Cfg::kAccCols + static_cast<uint32_t>(sw) * Cfg::kWCols; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -310,14 +316,19 @@ __global__ void __launch_bounds__(576, 1)
         if (!mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA)) break;
         if (!mbar_wait(&wready_bar[sw], phw, abort_flag, DEV_WAIT_TIMEOUT_DEQUANT)) break;
         tc_fence_after();
-        const uint32_t a_act = smem_u32(act_tile(st));
-        const uint32_t a_w = smem_u32(w_tile(sw));
-        const int slices = (l < n_main) ? Cfg::kStepK / 16 : 4;   // LoRA steps are 64 wide
-        for (int kk = 0; kk < slices; ++kk) {
-          const uint32_t atom = static_cast<uint32_t>(kk >> 2), kq = static_cast<uint32_t>(kk & 3);
-          const uint64_t da = make_sdesc_sw128(a_w + 16384u * atom + 32u * kq, 16u, 1024u);
-          const uint64_t db = make_sdesc_sw128(a_act + Cfg::kActAtomBytes * atom + 32u * kq, 16u, 1024u);
-          umma_bf16(tmem_base, da, db, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t db0 = make_sdesc_sw128(smem_u32(act_tile(st)), 16u, 1024u);
+        const uint32_t a_w = tmem_base + w_col(sw);
+        if (l < n_main) {
+#pragma unroll
+          for (int kk = 0; kk < Cfg::kStepK / 16; ++kk) {
+            // K slice kk: 8 TMEM columns of W; 32 bytes into the 128-byte-swizzled activation atom
+            const uint64_t ob = (Cfg::kActAtomBytes * static_cast<uint32_t>(kk >> 2) + 32u * (kk & 3)) >> 4;
+            umma_bf16_ta(tmem_base, a_w + 8u * kk, db0 + ob, Cfg::kIdesc, (l > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // LoRA steps are 64 wide
+            umma_bf16_ta(tmem_base, a_w + 8u * kk, db0 + ((32u * kk) >> 4), Cfg::kIdesc, 1u);
         }
         umma_commit(&empty_bar[st]);
         umma_commit(&wfree_bar[sw]);
@@ -331,7 +342,11 @@ __global__ void __launch_bounds__(576, 1)
     constexpr int G = Cfg::kGroups;
     const int t = threadIdx.x - 64;            // 0..511
     const int grp = t / Cfg::kGroupThreads;
-    const int tg = t % Cfg::kGroupThreads;     // block of the step
+    // A warp may only address its own 32-lane quarter of TMEM (warp % 4), and
+    // TMEM lane = W row: warp wl of a group (0..7) takes rows 32 (warp % 4) ..
+    // + 31 and block `sub` = wl / 4 of the step's two blocks per row.
+    const int wl = (warp - 2) & 7;
+    const uint32_t quarter = static_cast<uint32_t>(warp & 3);
     // the codebook as register immediates (no memory traffic)
     constexpr uint32_t kCB[16] = {QLORA_NF4_TABLE_BITS};
     float C[16];
@@ -340,9 +355,9 @@ __global__ void __launch_bounds__(576, 1)
     const ScaleSrc sc = p.sc;
     const float mean = group_mean(sc, n0);   // the tile's 128 rows lie in one projection
     // row = W row (0..127), sub = which of the step's two blocks
-    const int row = tg & 127;
-    const int sub = tg >> 7;
-    const uint32_t w_off = 16384u * sub;
+    const int row = 32 * static_cast<int>(quarter) + lane;
+    const int sub = wl >> 2;
+    const uint32_t lane_addr = quarter << 21;   // TMEM lane 32 * quarter in bits 16..31
     // Code tile rows are 64 B with the TMA 64-byte swizzle: 16-byte chunk j of
     // row r sits at j ^ ((r >> 1) & 3), which spreads a quarter-warp's reads
     // over all banks.
@@ -376,7 +391,8 @@ __global__ void __launch_bounds__(576, 1)
       bool okw = mbar_wait(&wfree_bar[sw], phw ^ 1, abort_flag, DEV_WAIT_TIMEOUT_MMA);
       okw = okw && mbar_wait(&full_bar[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
       if (!__all_sync(0xffffffffu, okw)) break;
-      const uint32_t wt = smem_u32(w_tile(sw)) + w_off;
+      tc_fence_after();   // the MMAs that read this W buffer have completed
+      const uint32_t wt = tmem_base + lane_addr + w_col(sw) + 32u * static_cast<uint32_t>(sub);
       if (l < n_main) {
         const ScaleRaw cur = pre0;
         const bool cur_valid = pre0_valid;
@@ -396,30 +412,37 @@ __global__ void __launch_bounds__(576, 1)
           w8[4 * h + 2] = cw.z;
           w8[4 * h + 3] = cw.w;
         }
+        // the block's 64 weights as 32 bf16 pairs, weight 2i in the low half
+        // of column i (K order), into this thread's TMEM lane
+        uint32_t v[32];
         if (cur_valid) {
           const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, cur, recip), C);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) sts128(wt + sw128_offset(row, c), dq8(w8[c], tab));
+          for (int c = 0; c < 8; ++c) {
+            const uint4 o = dq8(w8[c], tab);
+            v[4 * c] = o.x;
+            v[4 * c + 1] = o.y;
+            v[4 * c + 2] = o.z;
+            v[4 * c + 3] = o.w;
+          }
         } else {
 #pragma unroll
-          for (int c = 0; c < 8; ++c) sts128(wt + sw128_offset(row, c), make_uint4(0, 0, 0, 0));
+          for (int c = 0; c < 32; ++c) v[c] = 0u;
         }
+        tmem_st32(wt, v);
       } else if (sub == 0) {
         // LoRA extension step (64 wide): B row n against T_s columns 64e + [0, 64)
-        // into the first K atom
+        // into the first 32 columns of the W buffer
         const int e = xw.e_lo + l - n_main;
         const int64_t n = n0 + row;
-        const uint32_t wt0 = smem_u32(w_tile(sw));
+        uint32_t v[32];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint32_t h[8];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) h[q] = ext_b(p, xw, n, 64ll * e + 8 * c + q);
-          sts128(wt0 + sw128_offset(row, c),
-                 make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16)));
-        }
+        for (int c = 0; c < 32; ++c)
+          v[c] = ext_b(p, xw, n, 64ll * e + 2 * c) | (ext_b(p, xw, n, 64ll * e + 2 * c + 1) << 16);
+        tmem_st32(wt, v);
       }
-      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&wready_bar[sw]);
     }
