@@ -73,13 +73,22 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(src):
+    """Source text without comments and blank or trailing space, so that a
+    comment edit does not count as a kernel change."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash():
-    """Hash of the sources the many-token GEMM kernels are built from (the
+    """Hash of the code the many-token GEMM kernels are built from (the
     kernels whose DRAM traffic profiles/traffic_*.txt records)."""
     h = hashlib.sha256()
     for name in ("qlora_gemm.cu", "qlora_device.cuh", "qlora_internal.h", "nf4_scale.cuh", "nf4_table.h"):
-        with open(os.path.join(ROOT, "bit_quantized_lora_02_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "bit_quantized_lora_02_b200", "csrc", name)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

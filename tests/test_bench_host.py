@@ -54,3 +54,9 @@ def test_65b_step_flops():
     M, r = work["m"], work["r"]
     total = sum(bench.flops_fwd(M, d, k, r) + bench.flops_bwd(M, d, k, r) for _, d, k in work["proj"])
     assert abs(total / 1e12 - 27.017) < 5e-3
+
+
+def test_source_hash_ignores_comments():
+    src = "int f(int a) {  // add one\n  /* body */ return a + 1;\n}\n"
+    assert bench._code_only(src) == bench._code_only("int f(int a) {\n   return a + 1;\n}\n")
+    assert bench._code_only(src) != bench._code_only("int f(int a) {\n  return a + 2;\n}\n")
