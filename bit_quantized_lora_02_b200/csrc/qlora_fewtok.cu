@@ -474,7 +474,12 @@ __global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) 
   ft_finish<NTOK>(p, blockIdx.x, threadIdx.x >> 5, threadIdx.x & 31);
 }
 
-template <int NTOK>
+// CM selects how the block constants arrive: 0 = any mode (c2 loaded one item
+// ahead, or absmax without double quantisation, or c2 through TMA), 1 = Int8
+// c2 through TMA, 2 = E4M3 c2 through TMA.  Modes 1 and 2 carry no per-item
+// branches on the mode and check a row's c1 group only when its block index
+// reaches the next group boundary.
+template <int NTOK, int CM>
 __global__ void __launch_bounds__(kFtThreads, 1)
     k_qlora_fewtok(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_c2, const FtParams p) {
@@ -565,11 +570,12 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // blocks and its constant c1 with the correctly rounded reciprocal (s^ =
   // RN(RN(c2 / c1) + mean) through one residual correction; see nf4_scale.cuh).
   struct RowConst {
-    int64_t base, grp;
+    int32_t base, grp;   // 32-bit: the launcher requires every row's block indices below 2^31
     float c1, rc;
     bool fast, valid;
   };
   RowConst rw[2];
+  int32_t nxt = 0;       // (CM != 0) the block index at which a row of this lane enters another group
   auto set_rows = [&](int rbx) {
     const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
     // a 256-row block lies in one projection of a grouped weight
@@ -577,12 +583,35 @@ __global__ void __launch_bounds__(kFtThreads, 1)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       rw[h].valid = r0 + 8 * h < p.d;
-      rw[h].base = (r0 + 8 * h) * p.kpb;
+      rw[h].base = static_cast<int32_t>((r0 + 8 * h) * p.kpb);
       rw[h].grp = -1;
+      // rows past d: finite placeholders (their sums are never written)
+      rw[h].c1 = 1.0f;
+      rw[h].rc = 1.0f;
+      rw[h].fast = true;
+    }
+    nxt = 0;
+  };
+  // (CM != 0) reload c1 where a row's group changed at block blk (clamped to
+  // the row's last block in a ragged tail) and find the next boundary
+  auto refresh = [&](int32_t blk) {
+    const int32_t bq = blk < p.kpb ? blk : p.kpb - 1;
+    nxt = INT32_MAX;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (!rw[h].valid) continue;
+      const int32_t gq = (rw[h].base + bq) >> 8;
+      if (gq != rw[h].grp) {
+        rw[h].grp = gq;
+        rw[h].c1 = __ldg(p.sc.c1 + gq);
+        rw[h].rc = __frcp_rn(rw[h].c1);
+        rw[h].fast = (rw[h].c1 >= 0x1p-60f) && (rw[h].c1 <= 0x1p60f);
+      }
+      nxt = min(nxt, ((gq + 1) << 8) - rw[h].base);
     }
   };
-  auto row_scale = [&](RowConst& R, int64_t blk, int c2v) -> float {
-    const int64_t gq = (R.base + blk) >> 8;
+  auto row_scale = [&](RowConst& R, int32_t blk, int c2v) -> float {
+    const int32_t gq = (R.base + blk) >> 8;
     if (gq != R.grp) {
       R.grp = gq;
       R.c1 = __ldg(p.sc.c1 + gq);
@@ -641,7 +670,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   int pst = 0;        // stage and parity of the previous item
   uint32_t pph = 0;
   uint32_t c2w0 = 0, c2w1 = 0;   // c2 of this lane's two rows for the four items of the group
-  const bool loaded_consts = !(dq && c2_tma);
+  const bool loaded_consts = CM == 0 && !(dq && c2_tma);
   for (int i = 0; i < n_items; ++i) {
     const uint32_t cur_c2 = nc2;
     const float cur_ab0 = nab0, cur_ab1 = nab1;
@@ -649,7 +678,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
 
     mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
     const uint32_t sb = stage(st);
-    if (p.c2_tma && (i == 0 || (kc & 3) == 0)) {
+    if ((CM != 0 || p.c2_tma) && (i == 0 || (kc & 3) == 0)) {
       // first item of a group of four: the group's c2, row 16 c + g (+8) of the
       // row set; byte 4 t + bk is block bk of item t of the group
       const uint32_t cb = L.c2 + (((it0 + i) >> 2) & 1) * kFtC2Box + static_cast<uint32_t>(64 * rs + 16 * c + g) * 16u;
@@ -687,8 +716,30 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     }
 
     float sm0 = 0.0f, sm1 = 0.0f;
-    {
-      const int64_t blk = 4ll * kc + bk;
+    if constexpr (CM != 0) {
+      // s^ = RN(RN(c2 / c1) + mean) for this lane's two rows; the quotient
+      // through the reciprocal and one residual step (exact for c1 in
+      // [2^-60, 2^60], else the IEEE division)
+      const int32_t blk = 4 * kc + bk;
+      if (blk >= nxt) refresh(blk);
+      const int sh = 8 * (kc & 3);
+      auto numer = [&](uint32_t word) -> float {
+        return c2_numerator(CM, static_cast<int>(static_cast<int8_t>(static_cast<uint8_t>(word >> sh))));
+      };
+      const float w0 = numer(c2w0), w1 = numer(c2w1);
+      const float y0 = __fmul_rn(w0, rw[0].rc), y1 = __fmul_rn(w1, rw[1].rc);
+      float q0 = __fmaf_rn(__fmaf_rn(-rw[0].c1, y0, w0), rw[0].rc, y0);
+      float q1 = __fmaf_rn(__fmaf_rn(-rw[1].c1, y1, w1), rw[1].rc, y1);
+      if (!(rw[0].fast && rw[1].fast)) {
+        if (!rw[0].fast) q0 = __fdiv_rn(w0, rw[0].c1);
+        if (!rw[1].fast) q1 = __fdiv_rn(w1, rw[1].c1);
+      }
+      // blocks past the row's end (ragged K) contribute nothing; keep their scale finite
+      const bool bv = blk < p.kpb;
+      sm0 = bv ? __fadd_rn(q0, mean) : 0.0f;
+      sm1 = bv ? __fadd_rn(q1, mean) : 0.0f;
+    } else {
+      const int32_t blk = 4 * kc + bk;
       const bool bv = blk < p.kpb;
       if (dq) {
         const uint32_t c2p = c2_tma ? (((c2w0 >> (8 * (kc & 3))) & 0xFFu) | (((c2w1 >> (8 * (kc & 3))) & 0xFFu) << 8))
@@ -870,7 +921,9 @@ bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d) {
 }  // namespace
 
 bool fewtok_eligible(int64_t M, int64_t d, int64_t k) {
-  return M >= 1 && M <= kFewTokMax && d >= 1 && k >= 64 && k % 64 == 0;
+  // block indices of every row of every row block (rows past d included) fit in 31 bits
+  return M >= 1 && M <= kFewTokMax && d >= 1 && k >= 64 && k % 64 == 0 &&
+         ceil_div(d, kFtRows) * kFtRows * (k / 64) < (int64_t{1} << 31);
 }
 
 size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k) {
@@ -901,7 +954,10 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
     *why = "few-token down-projection launch";
     return QLORA_ERR_CUDA;
   }
-  if (set_smem(k_qlora_fewtok<NTOK>, kFtSmemBytes) != cudaSuccess) {
+  // Int8 or E4M3 c2 through TMA take the kernels without per-item mode branches
+  auto kern = !c2_tma ? k_qlora_fewtok<NTOK, 0> : a.q->double_quant == 2 ? k_qlora_fewtok<NTOK, 2>
+                                                                         : k_qlora_fewtok<NTOK, 1>;
+  if (set_smem(kern, kFtSmemBytes) != cudaSuccess) {
     *why = "smem attribute (few-token)";
     return QLORA_ERR_CUDA;
   }
@@ -941,7 +997,7 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   cudaError_t e;
   {
     ProfScope ps_(QLORA_KC_FWD_GEMM, st);
-    e = cudaLaunchKernelEx(&cfg, k_qlora_fewtok<NTOK>, tm, tx, tc2, p);
+    e = cudaLaunchKernelEx(&cfg, kern, tm, tx, tc2, p);
   }
   if (e != cudaSuccess || cudaGetLastError() != cudaSuccess) {
     *why = "few-token forward launch";
