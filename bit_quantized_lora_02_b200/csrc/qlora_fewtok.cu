@@ -73,7 +73,7 @@ struct FtCfg {
   static constexpr int kTG = NTOK / 8;                            // token groups of 8 (MMA N)
   static constexpr uint32_t kXBox = NTOK * 128u;                   // 64 columns of X for NTOK tokens
   static constexpr uint32_t kStageBytes = kFtCodeBytes + 4u * kXBox;
-  static constexpr uint32_t kScratch = 4u * 32u * 16u * kTG * 4u;  // [row set][lane][16 TG floats]
+  static constexpr uint32_t kScratch = 4u * 4u * kTG * 32u * 16u;  // [row set][row group, token group][lane] float4
   static constexpr uint32_t kMisc = 128;                           // barriers and flags
 };
 
@@ -324,11 +324,13 @@ __global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
 // Combine the four warps that share a 64-row set (one per 64-column block of
 // the item) and write the CTA's partial sums of the row block it leaves: in
 // three rounds the warps of block b = 1, 2, 3 park their sums in shared memory
-// (one slot per row set and lane) and the block-0 warp adds them in order.
+// (slot [row set][row group, token group][lane] of 16 bytes, so that a warp's
+// stores and loads cover consecutive banks) and the block-0 warp adds them in
+// order.  MMA row g of row group rg is weight row 16 rg + pg (and + 8).
 template <int TG>
 __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch, float* part, int rs, int bk,
-                                         int lane) {
-  float* scr = scratch + (rs * 32 + lane) * 16 * TG;
+                                         int lane, int pg) {
+  float4* scr = reinterpret_cast<float4*>(scratch) + rs * 4 * TG * 32 + lane;
   for (int b = 1; b < 4; ++b) {
     __syncthreads();   // the slot is free (block-0 warps have read the previous round)
     if (bk == b) {
@@ -336,8 +338,7 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
       for (int rg = 0; rg < 4; ++rg)
 #pragma unroll
         for (int t = 0; t < TG; ++t)
-          *reinterpret_cast<float4*>(scr + (rg * TG + t) * 4) =
-              make_float4(acc[rg][t][0], acc[rg][t][1], acc[rg][t][2], acc[rg][t][3]);
+          scr[(rg * TG + t) * 32] = make_float4(acc[rg][t][0], acc[rg][t][1], acc[rg][t][2], acc[rg][t][3]);
     }
     __syncthreads();
     if (bk == 0) {
@@ -345,7 +346,7 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
       for (int rg = 0; rg < 4; ++rg)
 #pragma unroll
         for (int t = 0; t < TG; ++t) {
-          const float4 v = *reinterpret_cast<const float4*>(scr + (rg * TG + t) * 4);
+          const float4 v = scr[(rg * TG + t) * 32];
           acc[rg][t][0] += v.x;
           acc[rg][t][1] += v.y;
           acc[rg][t][2] += v.z;
@@ -354,12 +355,12 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
     }
   }
   if (bk == 0) {
-    const int g = lane >> 2, c = lane & 3;
+    const int c = lane & 3;
 #pragma unroll
     for (int rg = 0; rg < 4; ++rg)
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
-        const int row = 64 * rs + 16 * rg + g;
+        const int row = 64 * rs + 16 * rg + pg;
         const int tok = 8 * t + 2 * c;
         part[tok * kFtRows + row] = acc[rg][t][0];
         part[(tok + 1) * kFtRows + row] = acc[rg][t][1];
@@ -536,9 +537,13 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   const int rs = warp & 3, bk = warp >> 2;
   const int g = lane >> 2, c = lane & 3;
   const uint32_t lanebase = L.table + static_cast<uint32_t>(lane) * 4u;
-  // this lane's 8 code bytes of row 64 rs + g in the 128-byte-swizzled tile
-  const uint32_t code_off = static_cast<uint32_t>(64 * rs + g) * 128u +
-                            16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ g) + 8u * static_cast<uint32_t>(c & 1);
+  // MMA row g (and g + 8) of a 16-row group is weight row pg (and pg + 8) of
+  // it, pg = 0, 2, 4, 6, 1, 3, 5, 7 for g = 0..7: the rows' 128-byte swizzle
+  // then spreads the 8-byte code loads of each half-warp over all 32 banks
+  const int pg = ((g & 3) << 1) | (g >> 2);
+  // this lane's 8 code bytes of row 64 rs + pg in the 128-byte-swizzled tile
+  const uint32_t code_off = static_cast<uint32_t>(64 * rs + pg) * 128u +
+                            16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ pg) + 8u * static_cast<uint32_t>(c & 1);
   // this lane's 16 columns of X (token 8 t + g) in the 128-byte-swizzled X chunk of block bk
   const uint32_t x_off = kFtCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
   const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
@@ -563,8 +568,8 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   if (threadIdx.x == 0)
     for (int j = 0; j < n_items && j < S; ++j) issue_item(j, j);
 
-  // ---- block constants.  This lane computes s^ for rows 16 c + g and +8 of its
-  // row set and block bk of each item.
+  // ---- block constants.  This lane computes s^ for rows lane and lane + 32 of
+  // its row set and block bk of each item.
   const bool dq = p.sc.dq != 0, c2_tma = p.c2_tma != 0;
   // Per row: flat index of block 0 of the row, the current group of 256
   // blocks and its constant c1 with the correctly rounded reciprocal (s^ =
@@ -577,13 +582,13 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   RowConst rw[2];
   int32_t nxt = 0;       // (CM != 0) the block index at which a row of this lane enters another group
   auto set_rows = [&](int rbx) {
-    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
+    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + lane;
     // a 256-row block lies in one projection of a grouped weight
     if (dq && p.sc.ngrp > 1) mean = group_mean(p.sc, static_cast<int64_t>(rbx) * kFtRows);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      rw[h].valid = r0 + 8 * h < p.d;
-      rw[h].base = static_cast<int32_t>((r0 + 8 * h) * p.kpb);
+      rw[h].valid = r0 + 32 * h < p.d;
+      rw[h].base = static_cast<int32_t>((r0 + 32 * h) * p.kpb);
       rw[h].grp = -1;
       // rows past d: finite placeholders (their sums are never written)
       rw[h].c1 = 1.0f;
@@ -635,15 +640,15 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   auto prefetch = [&](int rbx, int kcx) {
     if (dq && c2_tma) return;
     const int64_t blk = 4ll * kcx + bk;
-    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + 16 * c + g;
+    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + lane;
     const bool bv = blk < p.kpb;
     if (dq) {
       const uint32_t a = (bv && r0 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + r0 * p.kpb + blk)) : 0u;
-      const uint32_t b = (bv && r0 + 8 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + (r0 + 8) * p.kpb + blk)) : 0u;
+      const uint32_t b = (bv && r0 + 32 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + (r0 + 32) * p.kpb + blk)) : 0u;
       nc2 = a | (b << 8);
     } else {
       nab0 = (bv && r0 < p.d) ? __ldg(p.sc.absmax + r0 * p.kpb + blk) : 0.0f;
-      nab1 = (bv && r0 + 8 < p.d) ? __ldg(p.sc.absmax + (r0 + 8) * p.kpb + blk) : 0.0f;
+      nab1 = (bv && r0 + 32 < p.d) ? __ldg(p.sc.absmax + (r0 + 32) * p.kpb + blk) : 0.0f;
     }
   };
   set_rows(it0 / p.KC);
@@ -661,7 +666,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   int seg = 0;
   auto leave_block = [&](int) {
     ft_flush<TG>(acc, scratch, p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * kFtRows, rs,
-                 bk, lane);
+                 bk, lane, pg);
     ++seg;
   };
 
@@ -679,10 +684,10 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
     const uint32_t sb = stage(st);
     if ((CM != 0 || p.c2_tma) && (i == 0 || (kc & 3) == 0)) {
-      // first item of a group of four: the group's c2, row 16 c + g (+8) of the
-      // row set; byte 4 t + bk is block bk of item t of the group
-      const uint32_t cb = L.c2 + (((it0 + i) >> 2) & 1) * kFtC2Box + static_cast<uint32_t>(64 * rs + 16 * c + g) * 16u;
-      const uint4 ra = lds128(cb), rb8 = lds128(cb + 8u * 16u);
+      // first item of a group of four: the group's c2, rows lane and lane + 32
+      // of the row set; byte 4 t + bk is block bk of item t of the group
+      const uint32_t cb = L.c2 + (((it0 + i) >> 2) & 1) * kFtC2Box + static_cast<uint32_t>(64 * rs + lane) * 16u;
+      const uint4 ra = lds128(cb), rb8 = lds128(cb + 32u * 16u);
       const uint32_t sel = 0x40u + 0x11u * static_cast<uint32_t>(bk);   // byte bk of each word
       c2w0 = prmt(prmt(ra.x, ra.y, sel), prmt(ra.z, ra.w, sel), 0x5410u);
       c2w1 = prmt(prmt(rb8.x, rb8.y, sel), prmt(rb8.z, rb8.w, sel), 0x5410u);
@@ -751,56 +756,20 @@ __global__ void __launch_bounds__(kFtThreads, 1)
         sm1 = bv && rw[1].valid ? cur_ab1 : 0.0f;
       }
     }
-    if constexpr (TG == 2) {
-      // 16 tokens: the two token groups give each row group two independent
-      // chains, so the row groups go one after another and only one row
-      // group's partial sums are live (no register spills at 128 registers)
+    // The row groups go one after another, so only one row group's block sums
+    // are live.  MMA step j takes this lane's weights 4j .. 4j+3: code bytes 2j
+    // and 2j + 1, i.e. bytes 2 (j & 1) and 2 (j & 1) + 1 of word j >> 1; the
+    // byte permute puts the code byte into bits 8-15 of the lane's table
+    // address.  Row group rg's scales: weight rows 16 rg + pg and + 8 of the
+    // row set, computed by lanes (16 rg + pg) mod 32 and + 8 (s^ of rows 0..31
+    // in sm0, of rows 32..63 in sm1).
 #pragma unroll
-      for (int rg = 0; rg < 4; ++rg) {
-        float tmq[TG][4];
+    for (int rg = 0; rg < 4; ++rg) {
+      float tmq[TG][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
-          const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
-          const uint32_t w0 = (j < 2) ? cw[rg][0].x : cw[rg][0].y;
-          const uint32_t w1 = (j < 2) ? cw[rg][1].x : cw[rg][1].y;
-          const uint32_t a0 = lds32_const(prmt(w0, lanebase, sa));
-          const uint32_t a2 = lds32_const(prmt(w0, lanebase, sb));
-          const uint32_t a1 = lds32_const(prmt(w1, lanebase, sa));
-          const uint32_t a3 = lds32_const(prmt(w1, lanebase, sb));
-#pragma unroll
-          for (int t = 0; t < TG; ++t) {
-            const uint4 xq = xv[t][j >> 1];
-            const uint32_t b0 = (j & 1) ? xq.z : xq.x;
-            const uint32_t b1 = (j & 1) ? xq.w : xq.y;
-            if (j == 0)
-              mma16816_first(tmq[t], a0, a1, a2, a3, b0, b1);
-            else
-              mma16816(tmq[t], a0, a1, a2, a3, b0, b1);
-          }
-        }
-        const float s0 = __shfl_sync(0xffffffffu, sm0, 4 * g + rg);
-        const float s1 = __shfl_sync(0xffffffffu, sm1, 4 * g + rg);
-#pragma unroll
-        for (int t = 0; t < TG; ++t) {
-          acc[rg][t][0] = fmaf(tmq[t][0], s0, acc[rg][t][0]);
-          acc[rg][t][1] = fmaf(tmq[t][1], s0, acc[rg][t][1]);
-          acc[rg][t][2] = fmaf(tmq[t][2], s1, acc[rg][t][2]);
-          acc[rg][t][3] = fmaf(tmq[t][3], s1, acc[rg][t][3]);
-        }
-      }
-    } else {
-    // 8 tokens: four independent accumulation chains (one per 16-row group)
-    float tmp[4][TG][4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      // MMA step j takes this lane's weights 4j .. 4j+3: code bytes 2j and
-      // 2j + 1, i.e. bytes b = 2 (j & 1) and b + 1 of word j >> 1.  The byte
-      // permute puts the code byte into bits 8-15 of the lane's table address.
-      const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
-      const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
-#pragma unroll
-      for (int rg = 0; rg < 4; ++rg) {
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t sa = 0x7604u | ((2u * (j & 1)) << 4);
+        const uint32_t sb = 0x7604u | ((2u * (j & 1) + 1u) << 4);
         const uint32_t w0 = (j < 2) ? cw[rg][0].x : cw[rg][0].y;
         const uint32_t w1 = (j < 2) ? cw[rg][1].x : cw[rg][1].y;
         const uint32_t a0 = lds32_const(prmt(w0, lanebase, sa));
@@ -813,24 +782,21 @@ __global__ void __launch_bounds__(kFtThreads, 1)
           const uint32_t b0 = (j & 1) ? xq.z : xq.x;
           const uint32_t b1 = (j & 1) ? xq.w : xq.y;
           if (j == 0)
-            mma16816_first(tmp[rg][t], a0, a1, a2, a3, b0, b1);
+            mma16816_first(tmq[t], a0, a1, a2, a3, b0, b1);
           else
-            mma16816(tmp[rg][t], a0, a1, a2, a3, b0, b1);
+            mma16816(tmq[t], a0, a1, a2, a3, b0, b1);
         }
       }
-    }
-#pragma unroll
-    for (int rg = 0; rg < 4; ++rg) {
-      const float s0 = __shfl_sync(0xffffffffu, sm0, 4 * g + rg);
-      const float s1 = __shfl_sync(0xffffffffu, sm1, 4 * g + rg);
+      const float smr = rg < 2 ? sm0 : sm1;
+      const float s0 = __shfl_sync(0xffffffffu, smr, 16 * (rg & 1) + pg);
+      const float s1 = __shfl_sync(0xffffffffu, smr, 16 * (rg & 1) + 8 + pg);
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
-        acc[rg][t][0] = fmaf(tmp[rg][t][0], s0, acc[rg][t][0]);
-        acc[rg][t][1] = fmaf(tmp[rg][t][1], s0, acc[rg][t][1]);
-        acc[rg][t][2] = fmaf(tmp[rg][t][2], s1, acc[rg][t][2]);
-        acc[rg][t][3] = fmaf(tmp[rg][t][3], s1, acc[rg][t][3]);
+        acc[rg][t][0] = fmaf(tmq[t][0], s0, acc[rg][t][0]);
+        acc[rg][t][1] = fmaf(tmq[t][1], s0, acc[rg][t][1]);
+        acc[rg][t][2] = fmaf(tmq[t][2], s1, acc[rg][t][2]);
+        acc[rg][t][3] = fmaf(tmq[t][3], s1, acc[rg][t][3]);
       }
-    }
     }
     // leaving the row block (the next item starts another one, or the range ends)
     if (++kc == p.KC || i + 1 == n_items) {
