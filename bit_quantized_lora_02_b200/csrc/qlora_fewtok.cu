@@ -37,14 +37,17 @@
 //     multiplied by its scale s^ in fp32.  C[q] in bf16 times s^ carries the
 //     same bound, 2^-9 relative, as the bf16 weight BF16(C[q] s^) that the
 //     dequantisation produces.
-//   * When a CTA leaves a row block it writes its partial sums.  A third
+//   * When a CTA leaves a row block it writes its partial sums.  A second
 //     kernel, k_fewtok_finish, adds each row block's partial sums in CTA
 //     order, adds the LoRA term T_s B^T (mma.sync) and writes Y.
+//   * The down projection T_s = BF16(s X A^T) costs no launch of its own: the
+//     first 32 CTAs of the main kernel prefetch 32 shares of K of X and A
+//     into L2 when they start and compute their partial sums of X A^T after
+//     their last item; the finish kernel adds the 32 in order (every CTA for
+//     its row block's columns, and all CTAs together for the saved T_s).
 //
-// The three kernels are chained by programmatic dependent launch:
-// k_lora_down_fewtok computes T_s = BF16(s X A^T) (a cluster kernel), the main
-// kernel streams the weights while it runs and waits for it only before
-// exiting, and the finish kernel launches while the main kernel drains.
+// The finish kernel is launched with programmatic dependent launch, so it is
+// resident as soon as the main kernel's CTAs drain.
 #include <cstdio>
 
 #include "nf4_scale.cuh"
@@ -64,7 +67,6 @@ constexpr uint32_t kFtCodeBytes = kFtRows * kFtK / 2;       // 32 KB of codes pe
 constexpr int kFtMaxStages = 5;
 constexpr uint32_t kFtTableBytes = 65536;
 constexpr uint32_t kFtSmemBytes = 227u * 1024u;             // the whole window; placed in the kernel
-constexpr int kFtCluster = 8;                               // CTAs of one down-projection cluster
 constexpr uint32_t kFtC2Box = 16u * kFtRows;                // c2 of 16 blocks x 256 rows (four items)
 constexpr int kFtC2Slots = 2;
 
@@ -77,16 +79,24 @@ struct FtCfg {
   static constexpr uint32_t kMisc = 128;                           // barriers and flags
 };
 
+constexpr int kFtTProd = 32;   // CTAs of the main kernel that compute partial sums of X A^T
+
 struct FtParams {
   int64_t M, d, k;
   int32_t kpb;          // NF4 blocks per weight row
   int32_t r, rp;         // r: the rank of one projection (B's row length); rp: T_s's row length
+  int32_t rA;            // rows of A (every projection's r rows, stacked)
   ScaleSrc sc;            // grouped weights: rows from sc.gstart[i] on belong to projection i + 1
+  const uint16_t* X;    // M x k
+  const uint16_t* A;    // rA x k
+  const uint32_t* keep;  // adapter dropout: keep bits of X (bit b of word w <-> element 32 w + b), or null
+  float s_down;         // s, times 1 / (1 - p) of the kept elements with adapter dropout
   const uint16_t* B;    // d x r (projections' rows stacked)
-  const uint16_t* T;    // M x rp, T_s (written by the down kernel)
+  uint16_t* T;          // M x rp, T_s (written by the finish kernel)
   uint16_t* Y;          // M x d
   float* partial;       // [G][segmax][NTOK][256]
-  int32_t items, KC, G, segmax;
+  float* tpart;         // [tprod][16][rp]: each producer CTA's sums of X A^T over its share of K
+  int32_t items, KC, G, segmax, tprod;
   int32_t c2_tma;       // c2 arrives through the TMA ring (double quantisation, kpb % 16 == 0)
 };
 
@@ -193,23 +203,6 @@ __device__ __forceinline__ void mma16816_first(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ float ld_cluster_f32(const void* local, uint32_t rank) {
-  uint32_t remote;
-  float v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_u32(local)), "r"(rank));
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
-
-
 // The CTA whose item range holds item i (ranges: [c I / G, (c+1) I / G)).
 __device__ __forceinline__ int cta_of_item(int64_t i, int items, int G) {
   return static_cast<int>(((i + 1) * G + items - 1) / items) - 1;
@@ -224,98 +217,124 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p) { return *reinter
 }  // namespace
 
 // ============================================================================
-// T_s = BF16(s X A^T) for M <= 16 tokens on mma.sync: tokens are the M side
-// (16 rows), 8 ranks the N side.  One cluster of 8 CTAs per group of 8 ranks
-// below r; CTA q of the cluster covers the q-th eighth of K, its 8 warps take
-// every 8th 16-column step of it, the warps' fragments are added in warp order
-// and CTA 0 adds the eight CTAs' sums in order through distributed shared
-// memory.  The last cluster also writes the zero columns r .. rp - 1.
-// With adapter dropout `keep` is the keep bitmask of X (bit b of word w <->
-// flat element 32 w + b) and dropped elements enter the products as zeros;
-// `s` then includes the 1 / (1 - p) of the kept ones.
+// Partial sums of X A^T for M <= 16 tokens on mma.sync, computed by the first
+// tprod CTAs of the main kernel after their last item (their shares of X and A
+// were prefetched into L2 at the start): tokens are the M side (16 rows), 8
+// ranks the N side.  Producer q
+// takes the 16-column steps [n16 q / tprod, n16 (q + 1) / tprod) of K; its
+// warps split the rank groups of 8 and, within one, the steps; the warps of a
+// rank group add their sums in warp order through shared memory and write
+// tpart[q][token][rank].  The finish kernel adds the producers' sums in order,
+// so T_s = BF16(s X A^T) is the same on every run.
+// With adapter dropout `keep` is the keep bitmask of X and dropped elements
+// enter the products as zeros; s_down then includes the 1 / (1 - p).
 // ============================================================================
 // 32-bit lane mask of a bf16 pair from its two keep bits (bit 0: low element)
 __device__ __forceinline__ uint32_t pair_keep_mask(uint32_t two) {
   return ((two & 1u) ? 0x0000FFFFu : 0u) | ((two & 2u) ? 0xFFFF0000u : 0u);
 }
 
-__global__ void __cluster_dims__(kFtCluster, 1, 1) __launch_bounds__(256)
-    k_lora_down_fewtok(const uint16_t* __restrict__ X, const uint16_t* __restrict__ A, int M, int64_t k, int r,
-                       int rp, float s, uint16_t* __restrict__ T, const uint32_t* __restrict__ keep) {
-  griddep_launch_dependents();
-  __shared__ float4 red[8][32];
-  const uint32_t q = cluster_rank();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+// L2 prefetch of producer q's columns of X and A (one bulk prefetch per row:
+// 32 bytes per 16-column step, 16-byte aligned since k % 64 == 0)
+__device__ __forceinline__ void ft_down_prefetch(const FtParams& p, int q) {
+  const int64_t n16 = p.k >> 4;
+  const int64_t q0 = n16 * q / p.tprod, q1 = n16 * (q + 1) / p.tprod;
+  const uint32_t bytes = static_cast<uint32_t>(32 * (q1 - q0));
+  if (bytes == 0) return;
+  for (int row = threadIdx.x; row < p.M + p.rA; row += blockDim.x) {
+    const uint16_t* src = (row < p.M ? p.X + static_cast<int64_t>(row) * p.k
+                                     : p.A + static_cast<int64_t>(row - p.M) * p.k) + 16 * q0;
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+  }
+}
+
+__device__ __noinline__ void ft_down_part(const FtParams& p, int q, float4* red, int warp, int lane) {
   const int g = lane >> 2, c = lane & 3;
-  const int j0 = static_cast<int>(blockIdx.x / kFtCluster) * 8;
+  const int64_t k = p.k;
+  const int nrg = (p.rA + 7) >> 3;                        // rank groups of 8
+  const int wpg = nrg >= kFtWarps ? 1 : kFtWarps / nrg;   // warps per rank group
+  const int per_pass = kFtWarps / wpg;                    // rank groups per pass
+  const int sub = warp % wpg, slot = warp / wpg;
   const int64_t n16 = k >> 4;
-  const int64_t s0 = n16 * q / kFtCluster, s1 = n16 * (q + 1) / kFtCluster;
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  if (j0 < r) {
-    const bool ta = g < M, tb = g + 8 < M, jv = j0 + g < r;
-    const uint16_t* xa = X + static_cast<int64_t>(g) * k + 2 * c;
-    const uint16_t* xb = X + static_cast<int64_t>(g + 8) * k + 2 * c;
-    const uint16_t* ar = A + static_cast<int64_t>(j0 + g) * k + 2 * c;
-#pragma unroll 4
-    for (int64_t st = s0 + warp; st < s1; st += 8) {
-      const int64_t k0 = 16 * st;
-      uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
-      uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
-      const uint32_t b0 = jv ? ld_pair(ar + k0) : 0u, b1 = jv ? ld_pair(ar + k0 + 8) : 0u;
-      if (keep) {
-        // keep bits of columns k0 .. k0 + 15 of rows g and g + 8 (k0 % 16 == 0,
-        // k % 64 == 0: the 16 bits sit in one word at bit 0 or 16)
-        if (ta) {
-          const int64_t e = static_cast<int64_t>(g) * k + k0;
-          const uint32_t w = __ldg(keep + (e >> 5)) >> (e & 31);
-          a0 &= pair_keep_mask(w >> (2 * c));
-          a2 &= pair_keep_mask(w >> (8 + 2 * c));
+  const int64_t q0 = n16 * q / p.tprod, q1 = n16 * (q + 1) / p.tprod;
+  const int64_t s0 = q0 + (q1 - q0) * sub / wpg, s1 = q0 + (q1 - q0) * (sub + 1) / wpg;
+  const bool ta = g < p.M, tb = g + 8 < p.M;
+  const uint16_t* xa = p.X + static_cast<int64_t>(g) * k + 2 * c;
+  const uint16_t* xb = p.X + static_cast<int64_t>(g + 8) * k + 2 * c;
+  for (int rg0 = 0; rg0 < nrg; rg0 += per_pass) {
+    const int rgi = rg0 + slot;
+    const bool active = slot < per_pass && rgi < nrg;
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (active) {
+      const int j0 = 8 * rgi;
+      const bool jv = j0 + g < p.rA;
+      const uint16_t* ar = p.A + static_cast<int64_t>(j0 + g) * k + 2 * c;
+#pragma unroll 8
+      for (int64_t st = s0; st < s1; ++st) {
+        const int64_t k0 = 16 * st;
+        uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
+        uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
+        const uint32_t b0 = jv ? ld_pair(ar + k0) : 0u, b1 = jv ? ld_pair(ar + k0 + 8) : 0u;
+        if (p.keep) {
+          // keep bits of columns k0 .. k0 + 15 of tokens g and g + 8 (k0 % 16 == 0,
+          // k % 64 == 0: the 16 bits sit in one word at bit 0 or 16)
+          if (ta) {
+            const int64_t e = static_cast<int64_t>(g) * k + k0;
+            const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
+            a0 &= pair_keep_mask(w >> (2 * c));
+            a2 &= pair_keep_mask(w >> (8 + 2 * c));
+          }
+          if (tb) {
+            const int64_t e = static_cast<int64_t>(g + 8) * k + k0;
+            const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
+            a1 &= pair_keep_mask(w >> (2 * c));
+            a3 &= pair_keep_mask(w >> (8 + 2 * c));
+          }
         }
-        if (tb) {
-          const int64_t e = static_cast<int64_t>(g + 8) * k + k0;
-          const uint32_t w = __ldg(keep + (e >> 5)) >> (e & 31);
-          a1 &= pair_keep_mask(w >> (2 * c));
-          a3 &= pair_keep_mask(w >> (8 + 2 * c));
-        }
+        mma16816(acc, a0, a1, a2, a3, b0, b1);
       }
-      mma16816(acc, a0, a1, a2, a3, b0, b1);
     }
-  }
-  red[warp][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  __syncthreads();
-  if (warp == 0) {
-    float4 t = red[0][lane];
-    for (int w = 1; w < 8; ++w) {
-      const float4 v = red[w][lane];
-      t.x += v.x;
-      t.y += v.y;
-      t.z += v.z;
-      t.w += v.w;
+    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (active && sub == 0) {
+      float4 t = red[warp * 32 + lane];
+      for (int u = 1; u < wpg; ++u) {
+        const float4 v = red[(warp + u) * 32 + lane];
+        t.x += v.x;
+        t.y += v.y;
+        t.z += v.z;
+        t.w += v.w;
+      }
+      // fragment element e: token g + 8 (e >> 1), rank 8 rgi + 2 c + (e & 1) (< rp)
+      float* dst = p.tpart + static_cast<int64_t>(q) * 16 * p.rp + 8 * rgi + 2 * c;
+      dst[g * p.rp] = t.x;
+      dst[g * p.rp + 1] = t.y;
+      dst[(g + 8) * p.rp] = t.z;
+      dst[(g + 8) * p.rp + 1] = t.w;
     }
-    red[0][lane] = t;
+    __syncthreads();   // red is reused by the next pass (and, after the last, by the flushes)
   }
-  cluster_sync_all();
-  if (q == 0 && warp == 0) {
-    float tot[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (uint32_t p = 0; p < kFtCluster; ++p)
+}
+
+// T_s[tok][j] = BF16(s_down * sum over producers of tpart[.][tok][j]), the
+// producers added in order.  ft_t_load issues the loads (zeros when !live),
+// ft_t_bits adds and rounds.
+__device__ __forceinline__ void ft_t_load(const FtParams& p, int tok, int j, bool live, float (&v)[kFtTProd]) {
+  const float* src = p.tpart + static_cast<int64_t>(tok) * p.rp + j;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) tot[e] += ld_cluster_f32(reinterpret_cast<const float*>(&red[0][lane]) + e, p);
-    // fragment element e: token g + 8 (e >> 1), rank j0 + 2 c + (e & 1)
+  for (int q = 0; q < kFtTProd; ++q)
+    v[q] = (live && q < p.tprod) ? __ldcg(src + static_cast<int64_t>(q) * 16 * p.rp) : 0.0f;
+}
+__device__ __forceinline__ uint16_t ft_t_bits(const FtParams& p, const float (&v)[kFtTProd]) {
+  float t = v[0];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int tok = g + 8 * (e >> 1), j = j0 + 2 * c + (e & 1);
-      if (tok < M && j < rp)
-        T[static_cast<int64_t>(tok) * rp + j] =
-            static_cast<uint16_t>(pack_bf16x2(j < r ? s * tot[e] : 0.0f, 0.0f) & 0xFFFFu);
-    }
-  }
-  if (q == 0 && blockIdx.x / kFtCluster == gridDim.x / kFtCluster - 1) {
-    for (int i = threadIdx.x; i < M * rp; i += blockDim.x) {
-      const int tok = i / rp, j = i - tok * rp;
-      if (j >= j0 + 8) T[static_cast<int64_t>(tok) * rp + j] = 0;
-    }
-  }
-  cluster_sync_all();   // peers keep their shared memory until CTA 0 has read it
+  for (int q = 1; q < kFtTProd; ++q) t += v[q];
+  return static_cast<uint16_t>(pack_bf16x2(p.s_down * t, 0.0f) & 0xFFFFu);
+}
+__device__ __forceinline__ uint16_t ft_t_value(const FtParams& p, int tok, int j, bool live) {
+  float v[kFtTProd];
+  ft_t_load(p, tok, j, live, v);
+  return ft_t_bits(p, v);
 }
 
 // ============================================================================
@@ -380,8 +399,15 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
 // takes rows 16 w .. 16 w + 15 of the block.  All global loads of a batch are
 // issued before any is used (a row block has a few contributors and r / 16
 // LoRA steps).
-template <int NTOK>
-__device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, int lane) {
+// T_s of the row block's projection in shared memory: token tok's columns at
+// ts + tok * kTsWords (32-bit pairs), zero past M tokens and past r columns
+constexpr int kTsWords = 132;   // 128 pairs (r <= 256) + 4: a warp's pair loads hit 32 distinct banks
+
+// between() runs after the partial sums are added and before the LoRA term
+// reads ts; it fills ts and ends with a CTA barrier.
+template <int NTOK, class Between>
+__device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, int lane, const uint32_t* ts,
+                                          Between between) {
   constexpr int TG = NTOK / 8;
   constexpr int kC = 4;    // contributors per batch
   constexpr int kS = 4;    // LoRA K steps (16 ranks each) per batch
@@ -419,10 +445,10 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
 #pragma unroll
         for (int e = 0; e < 4; ++e) v[t][e] += pv[u][t][e];
   }
-  // LoRA term: rows of B are the A operand, T_s^T the B operand.  The row
-  // block's projection g uses T_s columns [g r, (g + 1) r).
+  between();
+  // LoRA term: rows of B are the A operand, T_s^T (the row block's
+  // projection's columns, in shared memory) the B operand.
   const bool even = (p.r & 1) == 0;
-  const int toff = group_of(p.sc, static_cast<int64_t>(rb) * kFtRows) * p.r;
   auto bpair = [&](int64_t n, int j) -> uint32_t {
     if (n >= p.d || j >= p.r) return 0u;
     const uint16_t* src = p.B + n * p.r + j;
@@ -443,10 +469,9 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
         const int tok = 8 * t + g;
-        const uint16_t* trow = p.T + static_cast<int64_t>(tok) * p.rp + toff;
-        // columns past this projection's r meet zero rows of B; keep the reads inside T_s
-        bf[u][t][0] = (ok && tok < p.M && toff + j0 + 1 < p.rp) ? ld_pair(trow + j0) : 0u;
-        bf[u][t][1] = (ok && tok < p.M && toff + j0 + 9 < p.rp) ? ld_pair(trow + j0 + 8) : 0u;
+        const uint32_t* trow = ts + tok * kTsWords;
+        bf[u][t][0] = ok ? trow[j0 >> 1] : 0u;
+        bf[u][t][1] = ok ? trow[(j0 >> 1) + 4] : 0u;
       }
     }
 #pragma unroll
@@ -468,11 +493,41 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
 }
 
 // One CTA per row block, 16 warps; launched as the programmatic dependent of
-// the main kernel.
+// the main kernel.  The T_s values a thread produces (one of the row block's
+// projection, one of the saved M x rp output) have their loads issued before
+// the partial sums' loads, so both arrive in one round trip.
 template <int NTOK>
 __global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) {
-  griddep_wait();   // the main kernel's partial sums (and, through it, T_s)
-  ft_finish<NTOK>(p, blockIdx.x, threadIdx.x >> 5, threadIdx.x & 31);
+  __shared__ uint32_t ts[16 * kTsWords];
+  griddep_wait();   // the main kernel's partial sums of W^ X and of X A^T
+  const int tid = threadIdx.x;
+  const int toff = group_of(p.sc, static_cast<int64_t>(blockIdx.x) * kFtRows) * p.r;
+  const int ncol = (p.r + 15) / 16 * 16;   // columns the LoRA steps read (zero past r)
+  const int nts = 16 * ncol;
+  const int tt = tid / ncol, tj = tid - tt * ncol;
+  float tv[kFtTProd];
+  ft_t_load(p, tt, toff + tj, tid < nts && tt < p.M && tj < p.r, tv);
+  const int64_t nT = p.M * p.rp, e0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + tid;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int st0 = static_cast<int>(e0 / p.rp), sj0 = static_cast<int>(e0 - static_cast<int64_t>(st0) * p.rp);
+  float sv[kFtTProd];
+  ft_t_load(p, st0, sj0, e0 < nT && sj0 < p.rA, sv);
+  uint16_t* ts16 = reinterpret_cast<uint16_t*>(ts);
+  ft_finish<NTOK>(p, blockIdx.x, tid >> 5, tid & 31, ts, [&]() {
+    // the row block's projection's T_s columns (zero past M tokens and past r)
+    if (tid < nts) ts16[tt * 2 * kTsWords + tj] = ft_t_bits(p, tv);
+    for (int i = tid + blockDim.x; i < nts; i += blockDim.x) {
+      const int tok = i / ncol, j = i - tok * ncol;
+      ts16[tok * 2 * kTsWords + j] = ft_t_value(p, tok, toff + j, tok < p.M && j < p.r);
+    }
+    // this CTA's share of the saved T_s (zero past rA columns)
+    if (e0 < nT) p.T[e0] = ft_t_bits(p, sv);
+    for (int64_t e = e0 + stride; e < nT; e += stride) {
+      const int tok = static_cast<int>(e / p.rp), j = static_cast<int>(e - static_cast<int64_t>(tok) * p.rp);
+      p.T[e] = ft_t_value(p, tok, j, j < p.rA);
+    }
+    __syncthreads();
+  });
 }
 
 // CM selects how the block constants arrive: 0 = any mode (c2 loaded one item
@@ -483,7 +538,7 @@ __global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) 
 template <int NTOK, int CM>
 __global__ void __launch_bounds__(kFtThreads, 1)
     k_qlora_fewtok(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_c2, const FtParams p) {
+                   const __grid_constant__ CUtensorMap tm_c2, const __grid_constant__ FtParams p) {
   using Cfg = FtCfg<NTOK>;
   constexpr int TG = Cfg::kTG;
   extern __shared__ __align__(1024) uint8_t ft_smem[];
@@ -532,6 +587,9 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     }
   }
   __syncthreads();
+  // Launched as a programmatic dependent: the set-up above overlaps the kernel
+  // before; from here on inputs are read (X, the codes and constants, keep bits)
+  griddep_wait();
 
   // warp = (row set rs: 64 rows) x (block bk: 64 columns of the item)
   const int rs = warp & 3, bk = warp >> 2;
@@ -547,7 +605,6 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // this lane's 16 columns of X (token 8 t + g) in the 128-byte-swizzled X chunk of block bk
   const uint32_t x_off = kFtCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
   const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
-  float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
   float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;   // of the current row block's projection
 
   // ---- TMA issue of item j into stage sj: the code tile, the item's 256
@@ -567,6 +624,10 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   };
   if (threadIdx.x == 0)
     for (int j = 0; j < n_items && j < S; ++j) issue_item(j, j);
+  float* scratch = reinterpret_cast<float*>(gptr(L.scratch));
+  // the first tprod CTAs compute partial sums of X A^T after their last item;
+  // their shares of X and A are brought into L2 now, behind the first items' copies
+  if (static_cast<int>(blockIdx.x) < p.tprod) ft_down_prefetch(p, blockIdx.x);
 
   // ---- block constants.  This lane computes s^ for rows lane and lane + 32 of
   // its row set and block bk of each item.
@@ -806,8 +867,8 @@ __global__ void __launch_bounds__(kFtThreads, 1)
       set_rows(rb);
     }
   }
-  griddep_wait();   // this grid completes after the down kernel, which the finish kernel relies on
-  __syncthreads();
+  __syncthreads();   // the flushes' reads of the scratch slots are done
+  if (static_cast<int>(blockIdx.x) < p.tprod) ft_down_part(p, blockIdx.x, reinterpret_cast<float4*>(scratch), warp, lane);
   if (threadIdx.x == 0 && *abort_flag) {
     // let the copies still in flight land before the CTA exits
     for (int sj = 0; sj < S; ++sj) {
@@ -827,11 +888,11 @@ __global__ void __launch_bounds__(kFtThreads, 1)
 namespace {
 
 struct FtPlan {
-  int ntok, KC, RB, items, G, segmax;
-  size_t part_bytes;
+  int ntok, KC, RB, items, G, segmax, tprod;
+  size_t part_bytes, tpart_bytes;
 };
 
-FtPlan ft_plan(int64_t M, int64_t d, int64_t k) {
+FtPlan ft_plan(int64_t M, int64_t d, int64_t k, int rp) {
   FtPlan f{};
   f.ntok = M <= 8 ? 8 : 16;
   f.KC = static_cast<int>(ceil_div(k, kFtK));
@@ -841,6 +902,8 @@ FtPlan ft_plan(int64_t M, int64_t d, int64_t k) {
   const int per = static_cast<int>(ceil_div(f.items, f.G));
   f.segmax = static_cast<int>(ceil_div(per, f.KC)) + 1;
   f.part_bytes = static_cast<size_t>(f.G) * f.segmax * f.ntok * kFtRows * 4;
+  f.tprod = f.G < kFtTProd ? f.G : kFtTProd;
+  f.tpart_bytes = static_cast<size_t>(f.tprod) * 16 * rp * 4;
   return f;
 }
 
@@ -892,14 +955,14 @@ bool fewtok_eligible(int64_t M, int64_t d, int64_t k) {
          ceil_div(d, kFtRows) * kFtRows * (k / 64) < (int64_t{1} << 31);
 }
 
-size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k) {
-  const FtPlan f = ft_plan(M, d, k);
-  return align_up(f.part_bytes, 256);
+size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k, int rp) {
+  const FtPlan f = ft_plan(M, d, k, rp);
+  return align_up(f.part_bytes, 256) + align_up(f.tpart_bytes, 256);
 }
 
 template <int NTOK>
 static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm, uint16_t* T, float* part,
-                     cudaStream_t st, const char** why, const uint32_t* keep) {
+                     float* tpart, cudaStream_t st, const char** why, const uint32_t* keep) {
   CUtensorMap tx, tc2;
   if (!map_x(&tx, a.X, a.M, a.k, NTOK)) {
     *why = "tensor map encoding failed (few-token X)";
@@ -910,16 +973,6 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   const bool c2_tma = a.q->double_quant && kpb % 16 == 0 && (reinterpret_cast<uintptr_t>(a.q->c2) & 15u) == 0 &&
                       map_c2(&tc2, a.q->c2, kpb, a.d);
   if (!c2_tma) tc2 = tx;   // unused
-  {
-    ProfScope ps_(QLORA_KC_LORA_GEMM, st);
-    const float s_down = (keep && a.drop) ? a.s * a.drop->dscale : a.s;
-    k_lora_down_fewtok<<<static_cast<unsigned>(kFtCluster * ceil_div(a.r, 8)), 256, 0, st>>>(
-        a.X, a.A, static_cast<int>(a.M), a.k, a.r, a.rp, s_down, T, keep);
-  }
-  if (cudaGetLastError() != cudaSuccess) {
-    *why = "few-token down-projection launch";
-    return QLORA_ERR_CUDA;
-  }
   // Int8 or E4M3 c2 through TMA take the kernels without per-item mode branches
   auto kern = !c2_tma ? k_qlora_fewtok<NTOK, 0> : a.q->double_quant == 2 ? k_qlora_fewtok<NTOK, 2>
                                                                          : k_qlora_fewtok<NTOK, 1>;
@@ -934,6 +987,13 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
   p.kpb = static_cast<int32_t>(a.k / 64);
   p.r = a.r_group > 0 ? a.r_group : a.r;
   p.rp = a.rp;
+  p.rA = a.r;
+  p.X = a.X;
+  p.A = a.A;
+  p.keep = keep;
+  p.s_down = (keep && a.drop) ? a.s * a.drop->dscale : a.s;
+  p.tpart = tpart;
+  p.tprod = f.tprod;
   p.sc.dq = a.q->double_quant;
   p.sc.ngrp = a.ngrp;
   for (int i = 0; i < 3; ++i) p.sc.gstart[i] = a.gstart[i];
@@ -984,11 +1044,12 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
 
 int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensorMap* tm_codes, cudaStream_t st,
                       const char** why, const uint32_t* keep) {
-  const FtPlan f = ft_plan(a.M, a.d, a.k);
+  const FtPlan f = ft_plan(a.M, a.d, a.k, a.rp);
   char* w = static_cast<char*>(ws);
   float* part = reinterpret_cast<float*>(w);
-  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, st, why, keep)
-                     : ft_launch<16>(a, f, *tm_codes, T, part, st, why, keep);
+  float* tpart = reinterpret_cast<float*>(w + align_up(f.part_bytes, 256));
+  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, tpart, st, why, keep)
+                     : ft_launch<16>(a, f, *tm_codes, T, part, tpart, st, why, keep);
 }
 
 }  // namespace qlora

@@ -1427,7 +1427,7 @@ static Plan make_plan(int64_t M, int64_t d, int64_t k, int32_t r, bool bwd, bool
   pl.off_T = need_T ? take(static_cast<size_t>(M) * rp * 2) : 0;
   if (!bwd && fewtok_eligible(M, d, k)) {
     pl.fewtok = true;
-    pl.off_main = take(fewtok_workspace_bytes(M, d, k));
+    pl.off_main = take(fewtok_workspace_bytes(M, d, k, rp));
   } else if (!bwd) {
     pl.nt = swap_nt(M);
     const int steps = static_cast<int>(k / 64);

@@ -92,7 +92,7 @@ int launch_linear_bwd(const LinearArgs& a, cudaStream_t st, const char** why);
 // as (k/2 bytes) x d rows, box 128 x 256, 128-byte swizzle.
 constexpr int kFewTokMax = 16;
 bool fewtok_eligible(int64_t M, int64_t d, int64_t k);
-size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k);
+size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k, int rp);
 int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensorMap* tm_codes, cudaStream_t st,
                       const char** why, const uint32_t* keep);
 

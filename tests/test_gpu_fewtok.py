@@ -2,8 +2,9 @@
 
 This path streams the packed codes through a TMA ring, expands them with a
 code-byte table and multiplies with register-resident tensor-core fragments;
-the block scale is applied to each block's partial sum and row blocks shared
-by several CTAs are combined by the last CTA to finish them.  The shapes below
+the block scale is applied to each block's partial sum, row blocks shared by
+several CTAs are combined by a finish kernel, and T_s = BF16(s X A^T) comes
+from partial sums that sixteen CTAs of the main kernel compute.  The shapes below
 cover ragged rows (d not a multiple of the 256-row item), ragged K (k not a
 multiple of the 256-column item), odd and large ranks, double quantisation
 off, row blocks split over many CTAs and a single item.
@@ -36,7 +37,7 @@ def _fwd(L, alpha, dq=True, save_T=True):
 
 def _check(L, Y, T, alpha, dq=True):
     r = L["A"].shape[0]
-    qo = O.quantize_tensor(L["W0"].reshape(-1), double_quant=dq)
+    qo = O.quantize_tensor(L["W0"].reshape(-1), double_quant=bool(dq), dq_fp8=(dq == 2))
     Wh = O.dequantize_tensor(qo).reshape(L["W0"].shape)
     Y_ref, T_ref = O.qlora_forward(L["X"], Wh, L["A"], L["B"], alpha, r)
     assert_close(host_f32(Y), Y_ref, "Y")
@@ -55,6 +56,7 @@ def _check(L, Y, T, alpha, dq=True):
     (16, 64, 64, 256),       # one NF4 block per row, largest rank
     (4, 1024, 16384, 16),    # each row block shared by ~37 CTAs
     (2, 4096, 576, 16),      # many row blocks, two items each
+    (5, 776, 3072, 16),      # c2 through TMA with c1 groups changing inside rows (48 blocks per row)
 ])
 def test_fewtok_shapes(M, d, k, r):
     L = synth.layer(M, d, k, r, seed=100 + M + r)
@@ -68,6 +70,14 @@ def test_fewtok_dq_off():
     _check(L, Y, T, 32.0, dq=False)
 
 
+def test_fewtok_e4m3_groups_inside_rows():
+    """E4M3 second-level constants through TMA, with c1 groups of 256 blocks
+    starting inside rows (48 blocks per row) and ragged rows."""
+    L = synth.layer(3, 520, 3072, 8, seed=9)
+    _, Y, T = _fwd(L, 16.0, dq=2)
+    _check(L, Y, T, 16.0, dq=2)
+
+
 def test_fewtok_without_saved_T():
     L = synth.layer(7, 512, 1024, 16, seed=8)
     _, Y, T = _fwd(L, 16.0, save_T=False)
@@ -77,8 +87,8 @@ def test_fewtok_without_saved_T():
 
 def test_fewtok_zero_adapter_and_repeat():
     """B = 0: Y equals the alpha = 0 run bit for bit.  A second identical call
-    gives identical bits (the per-row-block tickets are cleared every call and
-    the partial sums are added in a fixed order)."""
+    gives identical bits (the partial sums of W^ X and of X A^T are added in a
+    fixed order)."""
     M, d, k, r = 6, 1024, 4096, 16
     L = synth.layer(M, d, k, r, seed=11)
     L["B"] = np.zeros_like(L["B"])

@@ -43,6 +43,7 @@ def _oracle_q(W, dq):
     (300, (256, 256), 512, 16, 2),         # E4M3 second-level constants
     (64, (256, 512, 256), 1024, 16, 1),    # swapped forward (17..128 tokens)
     (8, (256, 256, 256), 512, 16, 1),      # few-token forward (<= 16 tokens)
+    (8, (256, 512, 256), 1024, 16, 1),     # few-token forward, c2 through TMA, one mean per projection
     (1, (512, 256), 256, 8, 1),            # a single token
     (130, (256, 256, 256, 256), 512, 64, 1),   # four projections, n r = 256
 ])
