@@ -61,23 +61,33 @@ namespace {
 
 constexpr int kFtWarps = 16;                                // 4 per SM sub-partition: up to 128 registers
 constexpr int kFtThreads = kFtWarps * 32;
-constexpr int kFtRows = 256;                                // weight rows per item
 constexpr int kFtK = 256;                                   // weights per row per item
-constexpr uint32_t kFtCodeBytes = kFtRows * kFtK / 2;       // 32 KB of codes per item
+constexpr int kFtMaxTok = 32;                               // tokens this path takes
 constexpr int kFtMaxStages = 5;
 constexpr uint32_t kFtTableBytes = 65536;
 constexpr uint32_t kFtSmemBytes = 227u * 1024u;             // the whole window; placed in the kernel
-constexpr uint32_t kFtC2Box = 16u * kFtRows;                // c2 of 16 blocks x 256 rows (four items)
 constexpr int kFtC2Slots = 2;
 
+// NTOK = 8 or 16 tokens: items of 256 weight rows, each warp 64 rows (four
+// 16-row MMA groups).  NTOK = 32: items of 128 rows, each warp 32 rows (two
+// groups), so that a warp's partial sums (rows x 32 tokens) still fit in
+// registers.  Row blocks (the rows whose partial sums a CTA writes and the
+// finish kernel combines) are one item high.
 template <int NTOK>
 struct FtCfg {
-  static constexpr int kTG = NTOK / 8;                            // token groups of 8 (MMA N)
+  static constexpr int kTG = NTOK / 8;                             // token groups of 8 (MMA N)
+  static constexpr int kRows = NTOK == 32 ? 128 : 256;             // weight rows per item
+  static constexpr int kSetRows = kRows / 4;                       // rows of a warp (its row set)
+  static constexpr int kRG = kSetRows / 16;                        // 16-row MMA groups of a warp
+  static constexpr int kLaneRows = kSetRows / 32;                  // rows whose s^ one lane computes
+  static constexpr uint32_t kCodeBytes = kRows * kFtK / 2;         // codes of an item
   static constexpr uint32_t kXBox = NTOK * 128u;                   // 64 columns of X for NTOK tokens
-  static constexpr uint32_t kStageBytes = kFtCodeBytes + 4u * kXBox;
-  static constexpr uint32_t kScratch = 4u * 4u * kTG * 32u * 16u;  // [row set][row group, token group][lane] float4
+  static constexpr uint32_t kStageBytes = kCodeBytes + 4u * kXBox;
+  static constexpr uint32_t kC2Box = 16u * kRows;                  // c2 of 16 blocks (four items)
+  static constexpr uint32_t kScratch = 4u * kRG * kTG * 32u * 16u;  // [row set][row group, token group][lane] float4
   static constexpr uint32_t kMisc = 128;                           // barriers and flags
 };
+constexpr int ft_rows(int ntok) { return ntok == 32 ? 128 : 256; }
 
 constexpr int kFtTProd = 32;   // CTAs of the main kernel that compute partial sums of X A^T
 
@@ -95,7 +105,7 @@ struct FtParams {
   uint16_t* T;          // M x rp, T_s (written by the finish kernel)
   uint16_t* Y;          // M x d
   float* partial;       // [G][segmax][NTOK][256]
-  float* tpart;         // [tprod][16][rp]: each producer CTA's sums of X A^T over its share of K
+  float* tpart;         // [tprod][32][rp]: each producer CTA's sums of X A^T over its share of K
   int32_t items, KC, G, segmax, tprod;
   int32_t c2_tma;       // c2 arrives through the TMA ring (double quantisation, kpb % 16 == 0)
 };
@@ -146,7 +156,7 @@ __device__ __forceinline__ FtLayout ft_layout(uint32_t raw) {
           return false;
         };
         FtLayout L{};
-        if (take(kFtC2Slots * kFtC2Box, 128u, L.c2) && take(Cfg::kScratch, 16u, L.scratch) &&
+        if (take(kFtC2Slots * Cfg::kC2Box, 128u, L.c2) && take(Cfg::kScratch, 16u, L.scratch) &&
             take(Cfg::kMisc, 16u, L.misc)) {
           L.table = T;
           L.lo0 = lo0;
@@ -248,7 +258,10 @@ __device__ __forceinline__ void ft_down_prefetch(const FtParams& p, int q) {
   }
 }
 
-__device__ __noinline__ void ft_down_part(const FtParams& p, int q, float4* red, int warp, int lane) {
+// NH token halves of 16 (NH = 2 for the 32-token kernel, whose scratch holds
+// the 16 KB of red that two halves need)
+template <int NH>
+__device__ __forceinline__ void ft_down_part(const FtParams& p, int q, float4* red, int warp, int lane) {
   const int g = lane >> 2, c = lane & 3;
   const int64_t k = p.k;
   const int nrg = (p.rA + 7) >> 3;                        // rank groups of 8
@@ -258,13 +271,12 @@ __device__ __noinline__ void ft_down_part(const FtParams& p, int q, float4* red,
   const int64_t n16 = k >> 4;
   const int64_t q0 = n16 * q / p.tprod, q1 = n16 * (q + 1) / p.tprod;
   const int64_t s0 = q0 + (q1 - q0) * sub / wpg, s1 = q0 + (q1 - q0) * (sub + 1) / wpg;
-  const bool ta = g < p.M, tb = g + 8 < p.M;
-  const uint16_t* xa = p.X + static_cast<int64_t>(g) * k + 2 * c;
-  const uint16_t* xb = p.X + static_cast<int64_t>(g + 8) * k + 2 * c;
   for (int rg0 = 0; rg0 < nrg; rg0 += per_pass) {
     const int rgi = rg0 + slot;
     const bool active = slot < per_pass && rgi < nrg;
-    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float acc[NH][4];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.0f;
     if (active) {
       const int j0 = 8 * rgi;
       const bool jv = j0 + g < p.rA;
@@ -272,45 +284,58 @@ __device__ __noinline__ void ft_down_part(const FtParams& p, int q, float4* red,
 #pragma unroll 8
       for (int64_t st = s0; st < s1; ++st) {
         const int64_t k0 = 16 * st;
-        uint32_t a0 = ta ? ld_pair(xa + k0) : 0u, a2 = ta ? ld_pair(xa + k0 + 8) : 0u;
-        uint32_t a1 = tb ? ld_pair(xb + k0) : 0u, a3 = tb ? ld_pair(xb + k0 + 8) : 0u;
         const uint32_t b0 = jv ? ld_pair(ar + k0) : 0u, b1 = jv ? ld_pair(ar + k0 + 8) : 0u;
-        if (p.keep) {
-          // keep bits of columns k0 .. k0 + 15 of tokens g and g + 8 (k0 % 16 == 0,
-          // k % 64 == 0: the 16 bits sit in one word at bit 0 or 16)
-          if (ta) {
-            const int64_t e = static_cast<int64_t>(g) * k + k0;
-            const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
-            a0 &= pair_keep_mask(w >> (2 * c));
-            a2 &= pair_keep_mask(w >> (8 + 2 * c));
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          // tokens 16 h + g (fragment rows 0..7) and 16 h + g + 8 (rows 8..15)
+          const int ta_tok = 16 * h + g, tb_tok = ta_tok + 8;
+          const bool ta = ta_tok < p.M, tb = tb_tok < p.M;
+          const uint16_t* xa = p.X + static_cast<int64_t>(ta_tok) * k + 2 * c + k0;
+          const uint16_t* xb = p.X + static_cast<int64_t>(tb_tok) * k + 2 * c + k0;
+          uint32_t a0 = ta ? ld_pair(xa) : 0u, a2 = ta ? ld_pair(xa + 8) : 0u;
+          uint32_t a1 = tb ? ld_pair(xb) : 0u, a3 = tb ? ld_pair(xb + 8) : 0u;
+          if (p.keep) {
+            // keep bits of columns k0 .. k0 + 15 of the two tokens (k0 % 16 == 0,
+            // k % 64 == 0: the 16 bits sit in one word at bit 0 or 16)
+            if (ta) {
+              const int64_t e = static_cast<int64_t>(ta_tok) * k + k0;
+              const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
+              a0 &= pair_keep_mask(w >> (2 * c));
+              a2 &= pair_keep_mask(w >> (8 + 2 * c));
+            }
+            if (tb) {
+              const int64_t e = static_cast<int64_t>(tb_tok) * k + k0;
+              const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
+              a1 &= pair_keep_mask(w >> (2 * c));
+              a3 &= pair_keep_mask(w >> (8 + 2 * c));
+            }
           }
-          if (tb) {
-            const int64_t e = static_cast<int64_t>(g + 8) * k + k0;
-            const uint32_t w = __ldg(p.keep + (e >> 5)) >> (e & 31);
-            a1 &= pair_keep_mask(w >> (2 * c));
-            a3 &= pair_keep_mask(w >> (8 + 2 * c));
-          }
+          mma16816(acc[h], a0, a1, a2, a3, b0, b1);
         }
-        mma16816(acc, a0, a1, a2, a3, b0, b1);
       }
     }
-    red[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+#pragma unroll
+    for (int h = 0; h < NH; ++h)
+      red[(h * kFtWarps + warp) * 32 + lane] = make_float4(acc[h][0], acc[h][1], acc[h][2], acc[h][3]);
     __syncthreads();
     if (active && sub == 0) {
-      float4 t = red[warp * 32 + lane];
-      for (int u = 1; u < wpg; ++u) {
-        const float4 v = red[(warp + u) * 32 + lane];
-        t.x += v.x;
-        t.y += v.y;
-        t.z += v.z;
-        t.w += v.w;
+#pragma unroll
+      for (int h = 0; h < NH; ++h) {
+        float4 t = red[(h * kFtWarps + warp) * 32 + lane];
+        for (int u = 1; u < wpg; ++u) {
+          const float4 v = red[(h * kFtWarps + warp + u) * 32 + lane];
+          t.x += v.x;
+          t.y += v.y;
+          t.z += v.z;
+          t.w += v.w;
+        }
+        // fragment element e: token 16 h + g + 8 (e >> 1), rank 8 rgi + 2 c + (e & 1) (< rp)
+        float* dst = p.tpart + (static_cast<int64_t>(q) * kFtMaxTok + 16 * h) * p.rp + 8 * rgi + 2 * c;
+        dst[g * p.rp] = t.x;
+        dst[g * p.rp + 1] = t.y;
+        dst[(g + 8) * p.rp] = t.z;
+        dst[(g + 8) * p.rp + 1] = t.w;
       }
-      // fragment element e: token g + 8 (e >> 1), rank 8 rgi + 2 c + (e & 1) (< rp)
-      float* dst = p.tpart + static_cast<int64_t>(q) * 16 * p.rp + 8 * rgi + 2 * c;
-      dst[g * p.rp] = t.x;
-      dst[g * p.rp + 1] = t.y;
-      dst[(g + 8) * p.rp] = t.z;
-      dst[(g + 8) * p.rp + 1] = t.w;
     }
     __syncthreads();   // red is reused by the next pass (and, after the last, by the flushes)
   }
@@ -323,7 +348,7 @@ __device__ __forceinline__ void ft_t_load(const FtParams& p, int tok, int j, boo
   const float* src = p.tpart + static_cast<int64_t>(tok) * p.rp + j;
 #pragma unroll
   for (int q = 0; q < kFtTProd; ++q)
-    v[q] = (live && q < p.tprod) ? __ldcg(src + static_cast<int64_t>(q) * 16 * p.rp) : 0.0f;
+    v[q] = (live && q < p.tprod) ? __ldcg(src + static_cast<int64_t>(q) * kFtMaxTok * p.rp) : 0.0f;
 }
 __device__ __forceinline__ uint16_t ft_t_bits(const FtParams& p, const float (&v)[kFtTProd]) {
   float t = v[0];
@@ -346,15 +371,17 @@ __device__ __forceinline__ uint16_t ft_t_value(const FtParams& p, int tok, int j
 // (slot [row set][row group, token group][lane] of 16 bytes, so that a warp's
 // stores and loads cover consecutive banks) and the block-0 warp adds them in
 // order.  MMA row g of row group rg is weight row 16 rg + pg (and + 8).
-template <int TG>
-__device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch, float* part, int rs, int bk,
-                                         int lane, int pg) {
-  float4* scr = reinterpret_cast<float4*>(scratch) + rs * 4 * TG * 32 + lane;
+template <int NTOK>
+__device__ __forceinline__ void ft_flush(float (&acc)[FtCfg<NTOK>::kRG][FtCfg<NTOK>::kTG][4], float* scratch,
+                                         float* part, int rs, int bk, int lane, int pg) {
+  using Cfg = FtCfg<NTOK>;
+  constexpr int TG = Cfg::kTG, RG = Cfg::kRG, R = Cfg::kRows;
+  float4* scr = reinterpret_cast<float4*>(scratch) + rs * RG * TG * 32 + lane;
   for (int b = 1; b < 4; ++b) {
     __syncthreads();   // the slot is free (block-0 warps have read the previous round)
     if (bk == b) {
 #pragma unroll
-      for (int rg = 0; rg < 4; ++rg)
+      for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
         for (int t = 0; t < TG; ++t)
           scr[(rg * TG + t) * 32] = make_float4(acc[rg][t][0], acc[rg][t][1], acc[rg][t][2], acc[rg][t][3]);
@@ -362,7 +389,7 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
     __syncthreads();
     if (bk == 0) {
 #pragma unroll
-      for (int rg = 0; rg < 4; ++rg)
+      for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
         for (int t = 0; t < TG; ++t) {
           const float4 v = scr[(rg * TG + t) * 32];
@@ -376,19 +403,19 @@ __device__ __forceinline__ void ft_flush(float (&acc)[4][TG][4], float* scratch,
   if (bk == 0) {
     const int c = lane & 3;
 #pragma unroll
-    for (int rg = 0; rg < 4; ++rg)
+    for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
-        const int row = 64 * rs + 16 * rg + pg;
+        const int row = Cfg::kSetRows * rs + 16 * rg + pg;
         const int tok = 8 * t + 2 * c;
-        part[tok * kFtRows + row] = acc[rg][t][0];
-        part[(tok + 1) * kFtRows + row] = acc[rg][t][1];
-        part[tok * kFtRows + row + 8] = acc[rg][t][2];
-        part[(tok + 1) * kFtRows + row + 8] = acc[rg][t][3];
+        part[tok * R + row] = acc[rg][t][0];
+        part[(tok + 1) * R + row] = acc[rg][t][1];
+        part[tok * R + row + 8] = acc[rg][t][2];
+        part[(tok + 1) * R + row + 8] = acc[rg][t][3];
       }
   }
 #pragma unroll
-  for (int rg = 0; rg < 4; ++rg)
+  for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
     for (int t = 0; t < TG; ++t)
 #pragma unroll
@@ -409,10 +436,11 @@ template <int NTOK, class Between>
 __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, int lane, const uint32_t* ts,
                                           Between between) {
   constexpr int TG = NTOK / 8;
-  constexpr int kC = 4;    // contributors per batch
-  constexpr int kS = 4;    // LoRA K steps (16 ranks each) per batch
+  constexpr int R = FtCfg<NTOK>::kRows;
+  constexpr int kC = TG <= 2 ? 4 : 2;   // contributors per batch
+  constexpr int kS = 4;                 // LoRA K steps (16 ranks each) per batch
   const int g = lane >> 2, c = lane & 3;
-  const int64_t na = static_cast<int64_t>(rb) * kFtRows + 16 * warp + g, nb = na + 8;
+  const int64_t na = static_cast<int64_t>(rb) * R + 16 * warp + g, nb = na + 8;
   const int ra = 16 * warp + g;
   float v[TG][4];
 #pragma unroll
@@ -428,14 +456,14 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
       const int cc = c0 + u;
       const bool ok = cc <= cl;
       const int seg = ok ? rb - first_item(cc, p.items, p.G) / p.KC : 0;
-      const float* part = p.partial + (static_cast<int64_t>(ok ? cc : cf) * p.segmax + seg) * NTOK * kFtRows;
+      const float* part = p.partial + (static_cast<int64_t>(ok ? cc : cf) * p.segmax + seg) * NTOK * R;
 #pragma unroll
       for (int t = 0; t < TG; ++t) {
         const int tok = 8 * t + 2 * c;
-        pv[u][t][0] = ok ? part[tok * kFtRows + ra] : 0.0f;
-        pv[u][t][1] = ok ? part[(tok + 1) * kFtRows + ra] : 0.0f;
-        pv[u][t][2] = ok ? part[tok * kFtRows + ra + 8] : 0.0f;
-        pv[u][t][3] = ok ? part[(tok + 1) * kFtRows + ra + 8] : 0.0f;
+        pv[u][t][0] = ok ? part[tok * R + ra] : 0.0f;
+        pv[u][t][1] = ok ? part[(tok + 1) * R + ra] : 0.0f;
+        pv[u][t][2] = ok ? part[tok * R + ra + 8] : 0.0f;
+        pv[u][t][3] = ok ? part[(tok + 1) * R + ra + 8] : 0.0f;
       }
     }
 #pragma unroll
@@ -492,18 +520,18 @@ __device__ __forceinline__ void ft_finish(const FtParams& p, int rb, int warp, i
   }
 }
 
-// One CTA per row block, 16 warps; launched as the programmatic dependent of
-// the main kernel.  The T_s values a thread produces (one of the row block's
+// One CTA per row block, one warp per 16 rows; launched as the programmatic
+// dependent of the main kernel.  The T_s values a thread produces (one of the row block's
 // projection, one of the saved M x rp output) have their loads issued before
 // the partial sums' loads, so both arrive in one round trip.
 template <int NTOK>
 __global__ void __launch_bounds__(kFtThreads) k_fewtok_finish(const FtParams p) {
-  __shared__ uint32_t ts[16 * kTsWords];
+  __shared__ uint32_t ts[NTOK * kTsWords];
   griddep_wait();   // the main kernel's partial sums of W^ X and of X A^T
   const int tid = threadIdx.x;
-  const int toff = group_of(p.sc, static_cast<int64_t>(blockIdx.x) * kFtRows) * p.r;
+  const int toff = group_of(p.sc, static_cast<int64_t>(blockIdx.x) * FtCfg<NTOK>::kRows) * p.r;
   const int ncol = (p.r + 15) / 16 * 16;   // columns the LoRA steps read (zero past r)
-  const int nts = 16 * ncol;
+  const int nts = NTOK * ncol;
   const int tt = tid / ncol, tj = tid - tt * ncol;
   float tv[kFtTProd];
   ft_t_load(p, tt, toff + tj, tid < nts && tt < p.M && tj < p.r, tv);
@@ -600,10 +628,10 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // then spreads the 8-byte code loads of each half-warp over all 32 banks
   const int pg = ((g & 3) << 1) | (g >> 2);
   // this lane's 8 code bytes of row 64 rs + pg in the 128-byte-swizzled tile
-  const uint32_t code_off = static_cast<uint32_t>(64 * rs + pg) * 128u +
+  const uint32_t code_off = static_cast<uint32_t>(Cfg::kSetRows * rs + pg) * 128u +
                             16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ pg) + 8u * static_cast<uint32_t>(c & 1);
   // this lane's 16 columns of X (token 8 t + g) in the 128-byte-swizzled X chunk of block bk
-  const uint32_t x_off = kFtCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
+  const uint32_t x_off = Cfg::kCodeBytes + static_cast<uint32_t>(bk) * Cfg::kXBox + static_cast<uint32_t>(g) * 128u;
   const uint32_t x_c0 = 16u * static_cast<uint32_t>((2 * c) ^ g), x_c1 = 16u * static_cast<uint32_t>((2 * c + 1) ^ g);
   float mean = p.sc.dq ? __ldg(p.sc.mean) : 0.0f;   // of the current row block's projection
 
@@ -614,12 +642,12 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   auto issue_item = [&](int j, int sj) {
     const int gi = it0 + j, irb = gi / p.KC, ikc = gi - irb * p.KC;
     const bool c2n = p.c2_tma && (j == 0 || (ikc & 3) == 0);
-    mbar_arrive_expect_tx(&full[sj], Cfg::kStageBytes + (c2n ? kFtC2Box : 0u));
+    mbar_arrive_expect_tx(&full[sj], Cfg::kStageBytes + (c2n ? Cfg::kC2Box : 0u));
     uint8_t* dst = gptr(stage(sj));
-    tma_load_2d(dst, &tm_codes, &full[sj], ikc * (kFtK / 2), irb * kFtRows);
-    tma_load_3d(dst + kFtCodeBytes, &tm_x, &full[sj], 0, 0, 4 * ikc);
+    tma_load_2d(dst, &tm_codes, &full[sj], ikc * (kFtK / 2), irb * Cfg::kRows);
+    tma_load_3d(dst + Cfg::kCodeBytes, &tm_x, &full[sj], 0, 0, 4 * ikc);
     if (c2n)
-      tma_load_2d(gptr(L.c2 + ((gi >> 2) & 1) * kFtC2Box), &tm_c2, &full[sj], 4 * (ikc & ~3), irb * kFtRows);
+      tma_load_2d(gptr(L.c2 + ((gi >> 2) & 1) * Cfg::kC2Box), &tm_c2, &full[sj], 4 * (ikc & ~3), irb * Cfg::kRows);
     last_item[sj] = j;
   };
   if (threadIdx.x == 0)
@@ -629,8 +657,8 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // their shares of X and A are brought into L2 now, behind the first items' copies
   if (static_cast<int>(blockIdx.x) < p.tprod) ft_down_prefetch(p, blockIdx.x);
 
-  // ---- block constants.  This lane computes s^ for rows lane and lane + 32 of
-  // its row set and block bk of each item.
+  // ---- block constants.  This lane computes s^ for row lane (and, with
+  // 64-row sets, lane + 32) of its row set and block bk of each item.
   const bool dq = p.sc.dq != 0, c2_tma = p.c2_tma != 0;
   // Per row: flat index of block 0 of the row, the current group of 256
   // blocks and its constant c1 with the correctly rounded reciprocal (s^ =
@@ -643,12 +671,12 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   RowConst rw[2];
   int32_t nxt = 0;       // (CM != 0) the block index at which a row of this lane enters another group
   auto set_rows = [&](int rbx) {
-    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + lane;
-    // a 256-row block lies in one projection of a grouped weight
-    if (dq && p.sc.ngrp > 1) mean = group_mean(p.sc, static_cast<int64_t>(rbx) * kFtRows);
+    const int64_t r0 = static_cast<int64_t>(rbx) * Cfg::kRows + Cfg::kSetRows * rs + lane;
+    // a row block (256 or 128 rows) lies in one projection of a grouped weight
+    if (dq && p.sc.ngrp > 1) mean = group_mean(p.sc, static_cast<int64_t>(rbx) * Cfg::kRows);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      rw[h].valid = r0 + 32 * h < p.d;
+      rw[h].valid = h < Cfg::kLaneRows && r0 + 32 * h < p.d;
       rw[h].base = static_cast<int32_t>((r0 + 32 * h) * p.kpb);
       rw[h].grp = -1;
       // rows past d: finite placeholders (their sums are never written)
@@ -701,23 +729,26 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   auto prefetch = [&](int rbx, int kcx) {
     if (dq && c2_tma) return;
     const int64_t blk = 4ll * kcx + bk;
-    const int64_t r0 = static_cast<int64_t>(rbx) * kFtRows + 64 * rs + lane;
+    const int64_t r0 = static_cast<int64_t>(rbx) * Cfg::kRows + Cfg::kSetRows * rs + lane;
     const bool bv = blk < p.kpb;
     if (dq) {
       const uint32_t a = (bv && r0 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + r0 * p.kpb + blk)) : 0u;
-      const uint32_t b = (bv && r0 + 32 < p.d) ? static_cast<uint8_t>(__ldg(p.sc.c2 + (r0 + 32) * p.kpb + blk)) : 0u;
+      const uint32_t b = (Cfg::kLaneRows == 2 && bv && r0 + 32 < p.d)
+                             ? static_cast<uint8_t>(__ldg(p.sc.c2 + (r0 + 32) * p.kpb + blk))
+                             : 0u;
       nc2 = a | (b << 8);
     } else {
       nab0 = (bv && r0 < p.d) ? __ldg(p.sc.absmax + r0 * p.kpb + blk) : 0.0f;
-      nab1 = (bv && r0 + 32 < p.d) ? __ldg(p.sc.absmax + (r0 + 32) * p.kpb + blk) : 0.0f;
+      nab1 = (Cfg::kLaneRows == 2 && bv && r0 + 32 < p.d) ? __ldg(p.sc.absmax + (r0 + 32) * p.kpb + blk) : 0.0f;
     }
   };
   set_rows(it0 / p.KC);
   if (n_items > 0) prefetch(it0 / p.KC, it0 - (it0 / p.KC) * p.KC);
 
-  float acc[4][TG][4];
+  constexpr int RG = Cfg::kRG;
+  float acc[RG][TG][4];
 #pragma unroll
-  for (int rg = 0; rg < 4; ++rg)
+  for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
     for (int t = 0; t < TG; ++t)
 #pragma unroll
@@ -726,8 +757,9 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // ---- leaving a row block: the CTA's partial sums out
   int seg = 0;
   auto leave_block = [&](int) {
-    ft_flush<TG>(acc, scratch, p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * kFtRows, rs,
-                 bk, lane, pg);
+    ft_flush<NTOK>(acc, scratch,
+                   p.partial + (static_cast<int64_t>(blockIdx.x) * p.segmax + seg) * NTOK * Cfg::kRows, rs, bk,
+                   lane, pg);
     ++seg;
   };
 
@@ -745,18 +777,22 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     mbar_wait(&full[st], ph, abort_flag, DEV_WAIT_TIMEOUT_TMA);
     const uint32_t sb = stage(st);
     if ((CM != 0 || p.c2_tma) && (i == 0 || (kc & 3) == 0)) {
-      // first item of a group of four: the group's c2, rows lane and lane + 32
+      // first item of a group of four: the group's c2, rows lane (and lane + 32)
       // of the row set; byte 4 t + bk is block bk of item t of the group
-      const uint32_t cb = L.c2 + (((it0 + i) >> 2) & 1) * kFtC2Box + static_cast<uint32_t>(64 * rs + lane) * 16u;
-      const uint4 ra = lds128(cb), rb8 = lds128(cb + 32u * 16u);
+      const uint32_t cb =
+          L.c2 + (((it0 + i) >> 2) & 1) * Cfg::kC2Box + static_cast<uint32_t>(Cfg::kSetRows * rs + lane) * 16u;
       const uint32_t sel = 0x40u + 0x11u * static_cast<uint32_t>(bk);   // byte bk of each word
+      const uint4 ra = lds128(cb);
       c2w0 = prmt(prmt(ra.x, ra.y, sel), prmt(ra.z, ra.w, sel), 0x5410u);
-      c2w1 = prmt(prmt(rb8.x, rb8.y, sel), prmt(rb8.z, rb8.w, sel), 0x5410u);
+      if constexpr (Cfg::kLaneRows == 2) {
+        const uint4 rb8 = lds128(cb + 32u * 16u);
+        c2w1 = prmt(prmt(rb8.x, rb8.y, sel), prmt(rb8.z, rb8.w, sel), 0x5410u);
+      }
     }
 
-    uint2 cw[4][2];
+    uint2 cw[RG][2];
 #pragma unroll
-    for (int rg = 0; rg < 4; ++rg)
+    for (int rg = 0; rg < RG; ++rg)
 #pragma unroll
       for (int h = 0; h < 2; ++h) cw[rg][h] = lds64(sb + code_off + static_cast<uint32_t>(16 * rg + 8 * h) * 128u);
     uint4 xv[TG][2];
@@ -825,7 +861,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     // row set, computed by lanes (16 rg + pg) mod 32 and + 8 (s^ of rows 0..31
     // in sm0, of rows 32..63 in sm1).
 #pragma unroll
-    for (int rg = 0; rg < 4; ++rg) {
+    for (int rg = 0; rg < RG; ++rg) {
       float tmq[TG][4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -868,7 +904,8 @@ __global__ void __launch_bounds__(kFtThreads, 1)
     }
   }
   __syncthreads();   // the flushes' reads of the scratch slots are done
-  if (static_cast<int>(blockIdx.x) < p.tprod) ft_down_part(p, blockIdx.x, reinterpret_cast<float4*>(scratch), warp, lane);
+  if (static_cast<int>(blockIdx.x) < p.tprod)
+    ft_down_part<NTOK == 32 ? 2 : 1>(p, blockIdx.x, reinterpret_cast<float4*>(scratch), warp, lane);
   if (threadIdx.x == 0 && *abort_flag) {
     // let the copies still in flight land before the CTA exits
     for (int sj = 0; sj < S; ++sj) {
@@ -894,16 +931,17 @@ struct FtPlan {
 
 FtPlan ft_plan(int64_t M, int64_t d, int64_t k, int rp) {
   FtPlan f{};
-  f.ntok = M <= 8 ? 8 : 16;
+  f.ntok = M <= 8 ? 8 : M <= 16 ? 16 : 32;
+  const int rows = ft_rows(f.ntok);
   f.KC = static_cast<int>(ceil_div(k, kFtK));
-  f.RB = static_cast<int>(ceil_div(d, kFtRows));
+  f.RB = static_cast<int>(ceil_div(d, rows));
   f.items = f.KC * f.RB;
   f.G = f.items < 148 ? f.items : 148;
   const int per = static_cast<int>(ceil_div(f.items, f.G));
   f.segmax = static_cast<int>(ceil_div(per, f.KC)) + 1;
-  f.part_bytes = static_cast<size_t>(f.G) * f.segmax * f.ntok * kFtRows * 4;
+  f.part_bytes = static_cast<size_t>(f.G) * f.segmax * f.ntok * rows * 4;
   f.tprod = f.G < kFtTProd ? f.G : kFtTProd;
-  f.tpart_bytes = static_cast<size_t>(f.tprod) * 16 * rp * 4;
+  f.tpart_bytes = static_cast<size_t>(f.tprod) * kFtMaxTok * rp * 4;
   return f;
 }
 
@@ -930,8 +968,8 @@ bool map_x(CUtensorMap* m, const uint16_t* X, int64_t M, int64_t k, int ntok) {
                                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// c2 (d x kpb int8) in boxes of 16 blocks x 256 rows
-bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d) {
+// c2 (d x kpb int8) in boxes of 16 blocks x `rows` rows
+bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d, int rows) {
   void* fp = nullptr;
   cudaDriverEntryPointQueryResult q;
   if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
@@ -939,7 +977,7 @@ bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d) {
     return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(kpb), static_cast<cuuint64_t>(d)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(kpb)};
-  cuuint32_t box[2] = {16u, static_cast<cuuint32_t>(kFtRows)};
+  cuuint32_t box[2] = {16u, static_cast<cuuint32_t>(rows)};
   cuuint32_t estr[2] = {1, 1};
   return reinterpret_cast<EncodeTiledFn>(fp)(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(c2), dims,
                                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -947,12 +985,30 @@ bool map_c2(CUtensorMap* m, const int8_t* c2, int64_t kpb, int64_t d) {
                                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// packed codes (d rows of k / 2 bytes) in boxes of 128 bytes (256 weights) x
+// `rows` rows, 128-byte swizzle
+bool map_codes(CUtensorMap* m, const uint8_t* codes, int64_t d, int64_t k, int rows) {
+  void* fp = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fp == nullptr)
+    return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(k / 2), static_cast<cuuint64_t>(d)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(k / 2)};
+  cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return reinterpret_cast<EncodeTiledFn>(fp)(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+                                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool fewtok_eligible(int64_t M, int64_t d, int64_t k) {
   // block indices of every row of every row block (rows past d included) fit in 31 bits
-  return M >= 1 && M <= kFewTokMax && d >= 1 && k >= 64 && k % 64 == 0 &&
-         ceil_div(d, kFtRows) * kFtRows * (k / 64) < (int64_t{1} << 31);
+  return M >= 1 && M <= kFtMaxTok && d >= 1 && k >= 64 && k % 64 == 0 &&
+         ceil_div(d, 256) * 256 * (k / 64) < (int64_t{1} << 31);
 }
 
 size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k, int rp) {
@@ -961,17 +1017,24 @@ size_t fewtok_workspace_bytes(int64_t M, int64_t d, int64_t k, int rp) {
 }
 
 template <int NTOK>
-static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm, uint16_t* T, float* part,
+static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm256, uint16_t* T, float* part,
                      float* tpart, cudaStream_t st, const char** why, const uint32_t* keep) {
-  CUtensorMap tx, tc2;
+  constexpr int R = FtCfg<NTOK>::kRows;
+  CUtensorMap tx, tc2, tm128;
   if (!map_x(&tx, a.X, a.M, a.k, NTOK)) {
     *why = "tensor map encoding failed (few-token X)";
     return QLORA_ERR_CUDA;
   }
+  // the caller's code map has 256-row boxes; 128-row items need their own
+  if (R != 256 && !map_codes(&tm128, a.q->codes, a.d, a.k, R)) {
+    *why = "tensor map encoding failed (few-token codes)";
+    return QLORA_ERR_CUDA;
+  }
+  const CUtensorMap& tm = R == 256 ? tm256 : tm128;
   // c2 through TMA when its rows are 16-byte multiples and its base is 16-byte aligned
   const int64_t kpb = a.k / 64;
   const bool c2_tma = a.q->double_quant && kpb % 16 == 0 && (reinterpret_cast<uintptr_t>(a.q->c2) & 15u) == 0 &&
-                      map_c2(&tc2, a.q->c2, kpb, a.d);
+                      map_c2(&tc2, a.q->c2, kpb, a.d, R);
   if (!c2_tma) tc2 = tx;   // unused
   // Int8 or E4M3 c2 through TMA take the kernels without per-item mode branches
   auto kern = !c2_tma ? k_qlora_fewtok<NTOK, 0> : a.q->double_quant == 2 ? k_qlora_fewtok<NTOK, 2>
@@ -1030,6 +1093,7 @@ static int ft_launch(const LinearArgs& a, const FtPlan& f, const CUtensorMap& tm
     return QLORA_ERR_CUDA;
   }
   cfg.gridDim = dim3(static_cast<unsigned>(f.RB));
+  cfg.blockDim = dim3(static_cast<unsigned>(R / 16 * 32));   // one warp per 16 rows of the row block
   cfg.dynamicSmemBytes = 0;
   {
     ProfScope ps_(QLORA_KC_AUX, st);
@@ -1048,8 +1112,9 @@ int launch_fewtok_fwd(const LinearArgs& a, uint16_t* T, void* ws, const CUtensor
   char* w = static_cast<char*>(ws);
   float* part = reinterpret_cast<float*>(w);
   float* tpart = reinterpret_cast<float*>(w + align_up(f.part_bytes, 256));
-  return f.ntok == 8 ? ft_launch<8>(a, f, *tm_codes, T, part, tpart, st, why, keep)
-                     : ft_launch<16>(a, f, *tm_codes, T, part, tpart, st, why, keep);
+  return f.ntok == 8    ? ft_launch<8>(a, f, *tm_codes, T, part, tpart, st, why, keep)
+         : f.ntok == 16 ? ft_launch<16>(a, f, *tm_codes, T, part, tpart, st, why, keep)
+                        : ft_launch<32>(a, f, *tm_codes, T, part, tpart, st, why, keep);
 }
 
 }  // namespace qlora

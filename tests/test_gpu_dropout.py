@@ -82,8 +82,9 @@ def _check(L, out, alpha, drop):
     (256, 512, 1024, 64, 0.5),     # a large p: the mask decides much of the adapter term
     (130, 264, 192, 5, 0.3),       # r not a multiple of 8
     (128, 384, 512, 256, 0.1),     # largest rank (four K chunks of the adapter term)
-    (33, 1024, 2048, 16, 0.05),    # swapped forward (17..128 tokens)
-    (8, 1024, 2048, 16, 0.2),      # few-token forward (<= 16 tokens)
+    (33, 1024, 2048, 16, 0.05),    # swapped forward (33..128 tokens)
+    (8, 1024, 2048, 16, 0.2),      # few-token forward (<= 32 tokens)
+    (20, 520, 1024, 16, 0.1),      # few-token forward with 17..32 tokens
     (1, 512, 256, 8, 0.4),         # a single token
 ])
 def test_dropout_layer(M, d, k, r, p):

@@ -1,4 +1,4 @@
-"""GPU parity of the few-token forward (M <= 16 tokens) against the CPU oracle.
+"""GPU parity of the few-token forward (M <= 32 tokens) against the CPU oracle.
 
 This path streams the packed codes through a TMA ring, expands them with a
 code-byte table and multiplies with register-resident tensor-core fragments;
@@ -57,6 +57,13 @@ def _check(L, Y, T, alpha, dq=True):
     (4, 1024, 16384, 16),    # each row block shared by ~37 CTAs
     (2, 4096, 576, 16),      # many row blocks, two items each
     (5, 776, 3072, 16),      # c2 through TMA with c1 groups changing inside rows (48 blocks per row)
+    # 17..32 tokens: items of 128 rows, each warp 32 rows of 32 token slots
+    (17, 392, 320, 5),       # ragged rows (not a multiple of 128) and K, odd rank
+    (24, 776, 3072, 16),     # c2 through TMA, c1 groups changing inside rows
+    (32, 1000, 2048, 64),
+    (32, 128, 64, 256),      # one NF4 block per row, largest rank
+    (20, 4096, 576, 16),     # many row blocks
+    (29, 1024, 16384, 16),   # each row block shared by many CTAs
 ])
 def test_fewtok_shapes(M, d, k, r):
     L = synth.layer(M, d, k, r, seed=100 + M + r)
@@ -68,6 +75,17 @@ def test_fewtok_dq_off():
     L = synth.layer(5, 600, 960, 16, seed=7)
     _, Y, T = _fwd(L, 32.0, dq=False)
     _check(L, Y, T, 32.0, dq=False)
+
+
+def test_fewtok_32_tokens_dq_off_and_e4m3():
+    """17..32 tokens with single-level constants (loaded one item ahead) and
+    with E4M3 second-level constants through TMA."""
+    L = synth.layer(25, 600, 960, 16, seed=17)
+    _, Y, T = _fwd(L, 32.0, dq=False)
+    _check(L, Y, T, 32.0, dq=False)
+    L = synth.layer(30, 520, 3072, 8, seed=19)
+    _, Y, T = _fwd(L, 16.0, dq=2)
+    _check(L, Y, T, 16.0, dq=2)
 
 
 def test_fewtok_e4m3_groups_inside_rows():
@@ -85,11 +103,12 @@ def test_fewtok_without_saved_T():
     _check(L, Y, None, 16.0)
 
 
-def test_fewtok_zero_adapter_and_repeat():
+@pytest.mark.parametrize("M", [6, 32])
+def test_fewtok_zero_adapter_and_repeat(M):
     """B = 0: Y equals the alpha = 0 run bit for bit.  A second identical call
     gives identical bits (the partial sums of W^ X and of X A^T are added in a
     fixed order)."""
-    M, d, k, r = 6, 1024, 4096, 16
+    d, k, r = 1024, 4096, 16
     L = synth.layer(M, d, k, r, seed=11)
     L["B"] = np.zeros_like(L["B"])
     q, Y0, _ = _fwd(L, 16.0)

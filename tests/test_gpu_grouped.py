@@ -41,9 +41,10 @@ def _oracle_q(W, dq):
     (600, (512, 256), 704, 64, 1),         # two projections (gate, up), ragged K
     (200, (256, 256, 256), 256, 8, 0),     # single-level constants
     (300, (256, 256), 512, 16, 2),         # E4M3 second-level constants
-    (64, (256, 512, 256), 1024, 16, 1),    # swapped forward (17..128 tokens)
-    (8, (256, 256, 256), 512, 16, 1),      # few-token forward (<= 16 tokens)
+    (64, (256, 512, 256), 1024, 16, 1),    # swapped forward (33..128 tokens)
+    (8, (256, 256, 256), 512, 16, 1),      # few-token forward (<= 32 tokens)
     (8, (256, 512, 256), 1024, 16, 1),     # few-token forward, c2 through TMA, one mean per projection
+    (24, (256, 256, 512), 1024, 16, 1),    # few-token forward with 17..32 tokens (128-row items)
     (1, (512, 256), 256, 8, 1),            # a single token
     (130, (256, 256, 256, 256), 512, 64, 1),   # four projections, n r = 256
 ])
