@@ -1,22 +1,23 @@
-// qlora_fewtok.cu -- the QLoRA forward for a few tokens (M <= 16).
+// qlora_fewtok.cu -- the QLoRA forward for a few tokens (M <= 32).
 //
 // "LoRA and QLoRA" (chkda.github.io/posts/lora_qlora), "Double quantization
 // and double dequantization": Y = X doubleDequant(c1, c2, W_NF4)^T + X L1 L2,
 // with the LoRA term written as (alpha/r) (X A^T) B^T ("How does alpha/r
 // control adapter strength?").
 //
-// With a handful of tokens each 4-bit weight takes part in at most 16
+// With a handful of tokens each 4-bit weight takes part in at most 32
 // products, so the layer is bound by streaming the packed codes from HBM
 // (half a byte per weight).  This path keeps the expanded weights in registers
 // and is organised around keeping enough bytes in flight:
 //
-//   * Work items are 256 weight rows x 256 columns (32 KB of codes), split
-//     evenly over one CTA per SM.  TMA brings each item's code tile and the
+//   * Work items are 256 weight rows x 256 columns (32 KB of codes; 128 rows
+//     for 17..32 tokens, so that a warp's partial sums stay in registers),
+//     split evenly over one CTA per SM.  TMA brings each item's code tile and the
 //     matching 256 columns of X (one 3-D box) through a ring of up to five
 //     stages; the refill of the stage of item i with item i + S is issued by
 //     warp i mod 16, so issuing costs no single warp more than its share.  The
 //     8-bit block constants c2 come with the first item of each group of four
-//     (16 blocks x 256 rows, two slots).  A row's group constant c1 changes
+//     (16 blocks x the item's rows, two slots).  A row's group constant c1 changes
 //     at most every 256 blocks and is reloaded only when it does.  (Without
 //     TMA-able c2 rows, or without double quantisation, the per-block
 //     constants are loaded one item ahead.)
@@ -26,7 +27,8 @@
 //     256 bytes apart from a 64 KB-aligned base, so a single byte permute
 //     turns a code byte into its lookup address.
 //   * Products run on mma.sync m16n8k16 (bf16 operands, fp32 accumulation):
-//     the weights are the register-resident A operand and 8 tokens the N side.
+//     the weights are the register-resident A operand and 8 tokens the N side
+//     (one, two or four token groups).
 //     Inside a 64-weight block the K order is permuted so that each lane's own
 //     code bytes fill its fragment slots; X is read with the same permutation.
 //     Tensor-core instructions that take their operands from shared memory

@@ -32,7 +32,7 @@
 //   k_qlora_pair<true>    dX, 512 tokens x 256 input columns per pair; the
 //                         dequant warps write W in the MN-major swizzled layout
 //                         (the reduction runs over W's rows).
-//   k_qlora_swap<NT>      17..128 tokens: W rows are the MMA's M side (128 per
+//   k_qlora_swap<NT>      33..128 tokens: W rows are the MMA's M side (128 per
 //                         tile), the tokens its N side, so the tensor core is
 //                         not padded to 128 tokens; split over K.
 //   k_thin<false,*>       T_s and U_s (K-major activations; A read K-major, B
@@ -177,7 +177,7 @@ __device__ __forceinline__ uint32_t ext_b(const MainParams& p, const ExtWindow& 
 }
 
 // ============================================================================
-// Swapped forward (17..128 tokens): the weight rows are the MMA's M side (128
+// Swapped forward (33..128 tokens): the weight rows are the MMA's M side (128
 // per CTA), the NT tokens its N side.  K step 128 (two NF4 blocks per weight
 // row); the LoRA extension steps are 64 wide.
 // ============================================================================
@@ -1393,7 +1393,7 @@ struct Plan {
   size_t off_T, off_Bt, off_U, off_main, total;
 };
 
-// Swapped forward (17..128 tokens): split K only as far as one wave of CTAs
+// Swapped forward (33..128 tokens): split K only as far as one wave of CTAs
 // (one per SM) is filled.  Each CTA pays a fixed set-up and drain per launch
 // and a split adds an fp32 partial pass, so a second, partly empty wave of
 // whole-K CTAs beats many short split CTAs: on 28672 x 8192 at M = 32, one
