@@ -48,8 +48,10 @@
 //     their last item; the finish kernel adds the 32 in order (every CTA for
 //     its row block's columns, and all CTAs together for the saved T_s).
 //
-// The finish kernel is launched with programmatic dependent launch, so it is
-// resident as soon as the main kernel's CTAs drain.
+// Both kernels are programmatic dependents: the streaming kernel builds its
+// lookup table and barriers while the kernel before it drains and waits for
+// it before reading any input; the finish kernel is scheduled as the
+// streaming kernel's CTAs exit.
 #include <cstdio>
 
 #include "nf4_scale.cuh"
@@ -229,11 +231,11 @@ __device__ __forceinline__ uint32_t ld_pair(const uint16_t* p) { return *reinter
 }  // namespace
 
 // ============================================================================
-// Partial sums of X A^T for M <= 16 tokens on mma.sync, computed by the first
-// tprod CTAs of the main kernel after their last item (their shares of X and A
-// were prefetched into L2 at the start): tokens are the M side (16 rows), 8
-// ranks the N side.  Producer q
-// takes the 16-column steps [n16 q / tprod, n16 (q + 1) / tprod) of K; its
+// Partial sums of X A^T on mma.sync, computed by the first tprod CTAs of the
+// main kernel after their last item (their shares of X and A were prefetched
+// into L2 at the start): 16 tokens are the M side (one or two halves of 16),
+// 8 ranks the N side.  Producer q takes the 16-column steps
+// [n16 q / tprod, n16 (q + 1) / tprod) of K; its
 // warps split the rank groups of 8 and, within one, the steps; the warps of a
 // rank group add their sums in warp order through shared memory and write
 // tpart[q][token][rank].  The finish kernel adds the producers' sums in order,
@@ -621,7 +623,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // before; from here on inputs are read (X, the codes and constants, keep bits)
   griddep_wait();
 
-  // warp = (row set rs: 64 rows) x (block bk: 64 columns of the item)
+  // warp = (row set rs: a quarter of the item's rows) x (block bk: 64 columns of the item)
   const int rs = warp & 3, bk = warp >> 2;
   const int g = lane >> 2, c = lane & 3;
   const uint32_t lanebase = L.table + static_cast<uint32_t>(lane) * 4u;
