@@ -108,7 +108,7 @@ struct FtParams {
   const uint16_t* B;    // d x r (projections' rows stacked)
   uint16_t* T;          // M x rp, T_s (written by the finish kernel)
   uint16_t* Y;          // M x d
-  float* partial;       // [G][segmax][NTOK][256]
+  float* partial;       // [G][segmax][NTOK][rows of a row block]
   float* tpart;         // [tprod][32][rp]: each producer CTA's sums of X A^T over its share of K
   int32_t items, KC, G, segmax, tprod;
   int32_t c2_tma;       // c2 arrives through the TMA ring (double quantisation, kpb % 16 == 0)
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kFtThreads, 1)
   // it, pg = 0, 2, 4, 6, 1, 3, 5, 7 for g = 0..7: the rows' 128-byte swizzle
   // then spreads the 8-byte code loads of each half-warp over all 32 banks
   const int pg = ((g & 3) << 1) | (g >> 2);
-  // this lane's 8 code bytes of row 64 rs + pg in the 128-byte-swizzled tile
+  // this lane's 8 code bytes of row kSetRows rs + pg in the 128-byte-swizzled tile
   const uint32_t code_off = static_cast<uint32_t>(Cfg::kSetRows * rs + pg) * 128u +
                             16u * static_cast<uint32_t>((2 * bk + (c >> 1)) ^ pg) + 8u * static_cast<uint32_t>(c & 1);
   // this lane's 16 columns of X (token 8 t + g) in the 128-byte-swizzled X chunk of block bk
