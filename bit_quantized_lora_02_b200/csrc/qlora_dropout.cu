@@ -102,10 +102,18 @@ constexpr int kUpCols = 128;
 constexpr int kRChunk = 64;
 constexpr int kUStride = kRChunk + 8;    // bf16 per row of the U_s tile (16 B pad: conflict-free ldmatrix)
 constexpr int kAStride = kUpCols + 8;    // bf16 per row of the A tile
-constexpr int kRStride = 4 * 40 + 4;     // floats per row of the result tile (quarters padded by 8)
-__device__ __forceinline__ int res_index(int row, int col) { return row * kRStride + col + 8 * (col >> 5); }
+// result tile: 64 rows x 128 fp32, 16-byte chunks XOR-swizzled per row and
+// 32-column quarter q (chunk c of quarter q at (c ^ h) within the quarter,
+// h = 2 ((row mod 4) ^ q) + (q mod 2)).  A half-warp's 8-byte fragment stores
+// (four rows x two chunks) and a quarter-warp's 16-byte epilogue reads (two
+// rows x four quarters) each hit all 32 banks once.
+__device__ __forceinline__ int res_index(int row, int col) {
+  const int chunk = col >> 2, q = chunk >> 3;
+  const int h = (((row & 3) ^ q) << 1) | (q & 1);
+  return row * 128 + (((q << 3) | ((chunk & 7) ^ h)) << 2) + (col & 3);
+}
 constexpr uint32_t kTileBytes = (kUpRows * kUStride + kRChunk * kAStride) * 2;
-constexpr uint32_t kResBytes = kUpRows * kRStride * 4;
+constexpr uint32_t kResBytes = kUpRows * kUpCols * 4;
 constexpr uint32_t kUpSmem = kTileBytes > kResBytes ? kTileBytes : kResBytes;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -216,11 +224,10 @@ __global__ void __launch_bounds__(256, 3)
   }
   __syncthreads();
   if (!live) return;
-  const float* rq = sR + row * kRStride + 40 * quarter;
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
-    const float4 lo = *reinterpret_cast<const float4*>(rq + 8 * ch);
-    const float4 hi = *reinterpret_cast<const float4*>(rq + 8 * ch + 4);
+    const float4 lo = *reinterpret_cast<const float4*>(sR + res_index(row, 32 * quarter + 8 * ch));
+    const float4 hi = *reinterpret_cast<const float4*>(sR + res_index(row, 32 * quarter + 8 * ch + 4));
     const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
     const uint32_t w4[4] = {x4[ch].x, x4[ch].y, x4[ch].z, x4[ch].w};
     uint32_t o[4];

@@ -41,12 +41,18 @@ constexpr int kMergeCols = 128;
 constexpr int kRChunk = 64;
 constexpr int kBStride = kRChunk + 8;         // bf16 per row of the B tile (16 B pad: no ldmatrix conflicts)
 constexpr int kAStride = kMergeCols + 8;      // bf16 per row of the A tile
-// result tile: 8 floats of padding after every 32-column quarter and a row
-// stride of 164 (= 4 mod 32) floats, so the epilogue's reads hit distinct banks
-constexpr int kRStride = 4 * 40 + 4;
-__device__ __forceinline__ int res_index(int row, int col) { return row * kRStride + col + 8 * (col >> 5); }
+// result tile: 64 rows x 128 fp32, 16-byte chunks XOR-swizzled per row and
+// 32-column quarter q (chunk c of quarter q at (c ^ h) within the quarter,
+// h = 2 ((row mod 4) ^ q) + (q mod 2)).  A half-warp's 8-byte fragment stores
+// (four rows x two chunks) and a quarter-warp's 16-byte epilogue reads (two
+// rows x four quarters) each hit all 32 banks once.
+__device__ __forceinline__ int res_index(int row, int col) {
+  const int chunk = col >> 2, q = chunk >> 3;
+  const int h = (((row & 3) ^ q) << 1) | (q & 1);
+  return row * 128 + (((q << 3) | ((chunk & 7) ^ h)) << 2) + (col & 3);
+}
 constexpr uint32_t kTileBytes = (kMergeRows * kBStride + kRChunk * kAStride) * 2;
-constexpr uint32_t kResBytes = kMergeRows * kRStride * 4;
+constexpr uint32_t kResBytes = kMergeRows * kMergeCols * 4;
 constexpr uint32_t kMergeSmem = kTileBytes > kResBytes ? kTileBytes : kResBytes;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -179,17 +185,13 @@ __global__ void __launch_bounds__(256, 3) k_lora_merge(const uint8_t* __restrict
   // the block's reconstructed weights, as doubleDequant stores them:
   // BF16(RN32(C[q] * s^))
   const Nf4Tab tab = make_tab(scale_value(sc.dq, mean, raw, recip), C);
-  // quarter q of the row starts on bank group 8 q (40 floats per quarter), the
-  // next row 4 banks later: a quarter-warp's 16-byte reads (two rows x four
-  // quarters) hit all 32 banks once
-  const float* rq = sR + row * kRStride + 40 * quarter;
   uint16_t* orow = out + n * k + c;
   const uint32_t cw[4] = {cw4.x, cw4.y, cw4.z, cw4.w};
 #pragma unroll
   for (int ch = 0; ch < 4; ++ch) {
     const uint4 wq = dq8(cw[ch], tab);   // 8 bf16 weights, element i in halfword i
-    const float4 lo = *reinterpret_cast<const float4*>(rq + 8 * ch);
-    const float4 hi = *reinterpret_cast<const float4*>(rq + 8 * ch + 4);
+    const float4 lo = *reinterpret_cast<const float4*>(sR + res_index(row, 32 * quarter + 8 * ch));
+    const float4 hi = *reinterpret_cast<const float4*>(sR + res_index(row, 32 * quarter + 8 * ch + 4));
     const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
     const uint32_t w4[4] = {wq.x, wq.y, wq.z, wq.w};
     uint32_t o[4];
